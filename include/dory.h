@@ -1,0 +1,168 @@
+/*
+ * dory.h -- C ABI of the B200 (sm_100a) elastic-depth forward pass of the
+ * Dory1.0-4B looped normalized-GPT.
+ *
+ * What is computed (sources: the Dory1.0-4B pages):
+ *   x0 = N(E[tok]); the input blocks map x0 to x; then for t = 1..k:
+ *   u_t = N(s_{t-1} + x) with s_0 = x, s_t = N(F_theta(u_t)) where F_theta is
+ *   the shared recurrent block; the output blocks run once; logits
+ *   z = s_z * (W_lm s).  Effective depth 32 + 40k sublayers.
+ *     -- "Dory1.0-4B: 循环归一化 GPT" (paper summary), 核心方法.
+ *   Every sublayer updates s <- N(s + alpha (N(h) - s)) with per-channel
+ *   alpha; the gated attention output and the SwiGLU activation are
+ *   L2-normalised before their output projections.
+ *     -- "Dory1.0-4B: A Looped Normalized-GPT" (paperlayer), §2 Architecture.
+ *   Attention: GQA, sliding window 1024 (RoPE base 1e4) and full attention
+ *   (RoPE base 1e7) interleaved 3:1, input-dependent sigmoid output gate.
+ *     -- paper summary, 技术新颖性; MXFP8 explainer, hybrid-attention section.
+ *   KV cache modes per_loop / last_loop: last_loop keeps one cache per
+ *   recurrent attention layer and every loop overwrites it.
+ *     -- paperlayer §6.1 Last-Loop KV Caching; MXFP8 explainer, last-loop.
+ *
+ * Conventions for every entry point:
+ *   - Return 0 (DORY_OK) or a negative DORY_ERR_* code; dory_strerror()
+ *     names it.  A failed call leaves caller buffers unspecified but the
+ *     library state valid.
+ *   - Pointers prefixed d_ are device pointers (global memory of the current
+ *     device); others are host pointers.  The caller allocates and owns every
+ *     device buffer (weights, cache, workspace, outputs); the library keeps
+ *     non-owning pointers plus small host-side plans.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued asynchronously; no entry point synchronises the device except
+ *     dory_sync_status().
+ */
+#ifndef DORY_H_
+#define DORY_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DORY_OK 0
+#define DORY_ERR_ARG (-1)         /* null pointer, bad size, bad name/shape  */
+#define DORY_ERR_UNSUPPORTED (-2) /* shape or format not compiled in         */
+#define DORY_ERR_CACHE (-3)       /* kv_mode / loop count / context overflow */
+#define DORY_ERR_CUDA (-4)        /* a CUDA call or launch failed            */
+#define DORY_ERR_TIMEOUT (-5)     /* a bounded device wait gave up           */
+#define DORY_ERR_WORKSPACE (-6)   /* workspace too small                     */
+#define DORY_ERR_DEVICE (-7)      /* a device-side check recorded an error   */
+
+typedef enum { DORY_KV_PER_LOOP = 0, DORY_KV_LAST_LOOP = 1 } dory_kv_mode;
+typedef enum { DORY_W_BF16 = 0, DORY_W_MXFP8 = 1, DORY_W_NVFP4 = 2 } dory_wfmt;
+
+/* Model shape.  A block is an attention sublayer followed by an MLP
+ * sublayer; blocks are numbered 0..n_blocks-1 in execution order (input,
+ * recurrent, output).  layer_types[i] = 0 (sliding window) or 1 (full).
+ * Requirements (else DORY_ERR_UNSUPPORTED): head_dim in {64, 128, 160},
+ * n_q_heads % n_kv_heads == 0 with at most 8 query heads per KV head, d,
+ * ffn and n_q_heads*head_dim multiples of 256, vocab and the q/k/v/gate row
+ * count multiples of 128, at least one input and one recurrent block. */
+typedef struct {
+  int d, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
+  int n_in_blocks, n_rec_blocks, n_out_blocks;
+  const uint8_t* layer_types; /* host array of n_blocks entries (copied) */
+  int swa_window;
+  double rope_theta_swa, rope_theta_full;
+  int wfmt;                   /* dory_wfmt of the block projections      */
+} dory_config;
+
+/* One named weight tensor in device memory (non-owning).  Names and shapes
+ * (row-major, K = contraction axis last):
+ *   "embed"  bf16 [vocab, d]       "lm_head" bf16 [vocab, d]
+ *   "s_z"    f32  [vocab]
+ *   "blk<i>.w_qkvg"  bf16 [2*Hq*h + 2*Hkv*h, d]  rows: q, k, v, gate
+ *   "blk<i>.s_q"     f32 [Hq, h]     "blk<i>.s_k" f32 [Hkv, h]
+ *   "blk<i>.w_o"     bf16 [d, Hq*h]  "blk<i>.alpha_a" f32 [d]
+ *   "blk<i>.w_gu"    bf16 [2*ffn, d] rows: gate then up
+ *   "blk<i>.w_down"  bf16 [d, ffn]   "blk<i>.alpha_m" f32 [d]
+ * alpha, s_q, s_k, s_z are the effective values used in the forward pass.
+ * Every device pointer must be 16-byte aligned. */
+typedef struct {
+  const char* name;
+  const void* d_ptr;
+  int64_t bytes;
+} dory_tensor;
+
+typedef struct dory_model dory_model;
+typedef struct dory_cache dory_cache;
+
+/* Validate the config and the weight table and build the host-side plan.
+ * Every tensor listed above must be present with exactly its byte size.
+ * No device memory is allocated; no kernel runs.  *out is released with
+ * dory_free().  Errors: DORY_ERR_ARG (missing/mis-sized tensor, bad shape),
+ * DORY_ERR_UNSUPPORTED (wfmt other than BF16, head_dim too large). */
+int dory_init_weights(const dory_config* cfg, const dory_tensor* tensors,
+                      int n_tensors, dory_model** out);
+
+/* Bytes of device memory a KV cache needs for `batch` sequences of up to
+ * `max_ctx` tokens, calls of up to `max_chunk` tokens per sequence, and (in
+ * per_loop mode) up to `max_loops` loops.  Layout: a small header, the full
+ * attention layers as 64-token pages behind a block table, the
+ * sliding-window layers as rings of min(max_ctx, window + max_chunk - 1)
+ * positions.  In last_loop mode the size does not depend on max_loops. */
+int dory_kv_cache_bytes(const dory_model* m, int batch, int max_ctx,
+                        int max_chunk, int max_loops, int kv_mode,
+                        int64_t* bytes);
+
+/* Bind a caller-owned device buffer (>= dory_kv_cache_bytes, 256-byte
+ * aligned) as an empty cache and enqueue its initialisation on `stream`.
+ * The kv_mode is fixed for the life of the cache. */
+int dory_kv_cache_bind(dory_model* m, void* d_buf, int64_t bytes, int batch,
+                       int max_ctx, int max_chunk, int max_loops, int kv_mode,
+                       void* stream, dory_cache** out);
+
+/* Tokens currently held per sequence (host mirror; all sequences of a cache
+ * advance together). */
+int dory_cache_length(const dory_cache* c, int* n_ctx);
+
+/* Forget all cached tokens (per_loop caches also forget their loop count). */
+int dory_cache_reset(dory_cache* c, void* stream);
+
+/* Workspace bytes for calls of `batch` sequences x up to `max_chunk`
+ * tokens.  The workspace holds activations only; its contents between
+ * calls are meaningless except for dory_copy_state(). */
+int dory_workspace_bytes(const dory_model* m, int batch, int max_chunk,
+                         int64_t* bytes);
+
+/* Append T tokens per sequence (d_tokens int32 [B, T], row-major) and run
+ * the looped forward pass over them with `n_loops` recurrent loops.
+ * B must equal the bound batch, 1 <= T <= max_chunk, n_ctx + T <= max_ctx,
+ * kv_mode must equal the cache's; a per_loop cache takes the loop count of
+ * its first call and rejects any other (DORY_ERR_CACHE).
+ * Outputs (either may be NULL): d_logits f32 [B, T, vocab] if logits_all
+ * else [B, vocab] (last token); d_argmax int32 [B, T] or [B] (greedy, lowest
+ * index on ties). */
+int dory_prefill(dory_model* m, dory_cache* c, const int32_t* d_tokens, int B,
+                 int T, int n_loops, int kv_mode, int logits_all,
+                 float* d_logits, int32_t* d_argmax, void* d_workspace,
+                 int64_t ws_bytes, void* stream);
+
+/* One decode step: one token per sequence (d_tokens int32 [B]).  Same rules
+ * as dory_prefill with T = 1.  The step is replayed from a CUDA graph once
+ * its launch plan has been seen with the same pointers, B and n_loops. */
+int dory_decode_step(dory_model* m, dory_cache* c, const int32_t* d_tokens,
+                     int B, int n_loops, int kv_mode, float* d_logits,
+                     int32_t* d_argmax, void* d_workspace, int64_t ws_bytes,
+                     void* stream);
+
+/* Copy the final residual state s (input of the LM head, f32) of the last
+ * call that used this workspace: [B, T, d] for a logits_all prefill, else
+ * [B, d]. */
+int dory_copy_state(const dory_model* m, const void* d_workspace, int B,
+                    int T, int logits_all, float* d_out, void* stream);
+
+/* Synchronise `stream` and report the device error word (bounded waits and
+ * device-side checks): DORY_OK, DORY_ERR_TIMEOUT or DORY_ERR_DEVICE; a
+ * failed synchronisation returns DORY_ERR_CUDA.  The word is cleared. */
+int dory_sync_status(dory_model* m, void* stream);
+
+const char* dory_strerror(int code);
+void dory_cache_free(dory_cache* c);
+void dory_free(dory_model* m);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DORY_H_ */

@@ -1,0 +1,659 @@
+// Host side of the C ABI declared in include/dory.h: validation, weight
+// table, KV-cache and workspace layout, the per-call launch plan and CUDA
+// graph replay of decode steps.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <cmath>
+#include <map>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "dory.h"
+#include "dory_internal.h"
+
+using namespace dory;
+
+static __device__ int g_dory_status;   // or-ed ERRBIT_* from device checks
+
+namespace {
+
+struct BlockW {
+  const bf16 *w_qkvg, *w_o, *w_gu, *w_down;
+  const float *s_q, *s_k, *alpha_a, *alpha_m;
+};
+
+typedef std::tuple<int, int, const void*, const void*, const void*,
+                   const void*, const void*> GraphKey;
+
+struct GraphEntry {
+  int seen = 0;
+  cudaGraphExec_t exec = nullptr;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+struct dory_model {
+  Dims dm;
+  int n_in, n_rec, n_out, nblk;
+  std::vector<uint8_t> ltype;
+  double th_swa, th_full;
+  const bf16* embed;
+  const bf16* lm_head;
+  const float* s_z;
+  std::vector<BlockW> blk;
+  int num_sms = 148;
+  int device = 0;
+  int* d_status = nullptr;
+  bool use_graphs = true;
+  cudaStream_t cap_stream = nullptr;
+  std::map<GraphKey, GraphEntry> graphs;
+};
+
+struct dory_cache {
+  dory_model* m;
+  int B, max_ctx, max_chunk, max_loops, kv_mode;
+  int n_ctx = 0;
+  int loops_bound = 0;
+  int pages_per_seq;
+  int swa_cap;
+  int* d_nctx;
+  int* d_block_table;
+  std::vector<int> slot_base;   // per block: first entry in `slots`
+  std::vector<KVSlot> slots;
+};
+
+namespace {
+
+bool is_rec(const dory_model* m, int i) {
+  return i >= m->n_in && i < m->n_in + m->n_rec;
+}
+
+// Number of cache slots of block i: per_loop recurrent blocks keep one per
+// loop; every other block keeps one.
+int slots_of(const dory_model* m, int i, int kv_mode, int max_loops) {
+  return (is_rec(m, i) && kv_mode == DORY_KV_PER_LOOP) ? max_loops : 1;
+}
+
+struct CacheLayout {
+  size_t header, table, total;
+  std::vector<size_t> k_off, v_off;
+  std::vector<int> ring, cap;
+  std::vector<int> base;
+  int pages_per_seq, swa_cap;
+};
+
+CacheLayout cache_layout(const dory_model* m, int B, int max_ctx,
+                         int max_chunk, int max_loops, int kv_mode) {
+  CacheLayout L;
+  const Dims& dm = m->dm;
+  L.pages_per_seq = (max_ctx + kPage - 1) / kPage;
+  L.swa_cap = std::min(max_ctx, dm.window + max_chunk - 1);
+  L.header = 256;
+  L.table = align256((size_t)B * L.pages_per_seq * sizeof(int));
+  size_t off = L.header + L.table;
+  for (int i = 0; i < m->nblk; ++i) {
+    L.base.push_back((int)L.k_off.size());
+    const int n = slots_of(m, i, kv_mode, max_loops);
+    for (int s = 0; s < n; ++s) {
+      const bool full = m->ltype[i] == 1;
+      const size_t per =
+          full ? (size_t)B * L.pages_per_seq * dm.Hkv * kPage * dm.hd * 2
+               : (size_t)B * dm.Hkv * L.swa_cap * dm.hd * 2;
+      L.k_off.push_back(off);
+      off += align256(per);
+      L.v_off.push_back(off);
+      off += align256(per);
+      L.ring.push_back(full ? 0 : 1);
+      L.cap.push_back(full ? 0 : L.swa_cap);
+    }
+  }
+  L.total = off;
+  return L;
+}
+
+int gemv_split(int K, int n_items) {
+  int S = 1;
+  while (S < 8 && K % (2 * S * 256) == 0 && K / (2 * S) >= 1024 &&
+         (long)n_items * S < 8192)
+    S *= 2;
+  return S;
+}
+
+struct WS {
+  float *s0, *s1, *sfin, *x, *qkvg, *q, *gate, *h, *gu, *part_o, *part_ml,
+      *rope, *amax_val;
+  bf16 *s_bf, *a, *mact;
+  int* amax_idx;
+  size_t total;
+};
+
+constexpr int kMaxS = 8;
+constexpr int kArgmaxSlots = 2048;
+
+WS ws_layout(const dory_model* m, int B, int T, char* base) {
+  const Dims& dm = m->dm;
+  const size_t M = (size_t)B * T;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  WS w;
+  w.s0 = (float*)take(M * dm.d * 4);
+  w.s1 = (float*)take(M * dm.d * 4);
+  w.sfin = (float*)take(M * dm.d * 4);
+  w.x = (float*)take(M * dm.d * 4);
+  w.s_bf = (bf16*)take(M * dm.d * 2);
+  w.qkvg = (float*)take(kMaxS * M * dm.rows_qkvg * 4);
+  w.q = (float*)take(M * dm.qdim * 4);
+  w.gate = (float*)take(M * dm.qdim * 4);
+  w.a = (bf16*)take(M * dm.qdim * 2);
+  w.h = (float*)take(kMaxS * M * dm.d * 4);
+  w.gu = (float*)take(M > 8 || T > 1 ? M * 2 * (size_t)dm.F * 4 : 0);
+  w.mact = (bf16*)take(M * dm.F * 2);
+  w.part_o = (float*)take((size_t)B * dm.Hq * kMaxSplits * dm.hd * 4);
+  w.part_ml = (float*)take((size_t)B * dm.Hq * kMaxSplits * 2 * 4);
+  w.rope = (float*)take((size_t)2 * T * (dm.hd / 2) * 2 * 4);
+  w.amax_val = (float*)take((size_t)B * kArgmaxSlots * 4);
+  w.amax_idx = (int*)take((size_t)B * kArgmaxSlots * 4);
+  w.total = off;
+  return w;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? DORY_OK : DORY_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* dory_strerror(int code) {
+  switch (code) {
+    case DORY_OK: return "ok";
+    case DORY_ERR_ARG: return "invalid argument";
+    case DORY_ERR_UNSUPPORTED: return "unsupported shape or format";
+    case DORY_ERR_CACHE: return "kv cache mismatch or overflow";
+    case DORY_ERR_CUDA: return "CUDA error";
+    case DORY_ERR_TIMEOUT: return "bounded device wait timed out";
+    case DORY_ERR_WORKSPACE: return "workspace too small";
+    case DORY_ERR_DEVICE: return "device-side check failed";
+    default: return "unknown error";
+  }
+}
+
+int dory_init_weights(const dory_config* cfg, const dory_tensor* tensors,
+                      int n_tensors, dory_model** out) {
+  if (!cfg || !out || (n_tensors > 0 && !tensors)) return DORY_ERR_ARG;
+  *out = nullptr;
+  const int d = cfg->d, Hq = cfg->n_q_heads, Hkv = cfg->n_kv_heads,
+            hd = cfg->head_dim, F = cfg->ffn, V = cfg->vocab;
+  if (d <= 0 || Hq <= 0 || Hkv <= 0 || hd <= 0 || F <= 0 || V <= 0)
+    return DORY_ERR_ARG;
+  if (cfg->n_in_blocks < 1 || cfg->n_rec_blocks < 1 || cfg->n_out_blocks < 0)
+    return DORY_ERR_ARG;
+  if (!cfg->layer_types || cfg->swa_window < 1) return DORY_ERR_ARG;
+  if (!(cfg->rope_theta_swa > 1.0) || !(cfg->rope_theta_full > 1.0))
+    return DORY_ERR_ARG;
+  if (Hq % Hkv) return DORY_ERR_ARG;
+  if (cfg->wfmt != DORY_W_BF16) return DORY_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (!(hd == 64 || hd == 128 || hd == 160) || G > 8 || G * hd > 1024)
+    return DORY_ERR_UNSUPPORTED;
+  if (d % 256 || F % 256 || (Hq * hd) % 256 || V % 128 || d > 8192 ||
+      F > 32768)
+    return DORY_ERR_UNSUPPORTED;
+  const int rows = 2 * Hq * hd + 2 * Hkv * hd;
+  if (rows % 128) return DORY_ERR_UNSUPPORTED;
+
+  dory_model* m = new dory_model();
+  m->dm = Dims{d, Hq, Hkv, hd, F, V, Hq * hd, Hkv * hd, rows, cfg->swa_window};
+  m->n_in = cfg->n_in_blocks;
+  m->n_rec = cfg->n_rec_blocks;
+  m->n_out = cfg->n_out_blocks;
+  m->nblk = m->n_in + m->n_rec + m->n_out;
+  m->ltype.assign(cfg->layer_types, cfg->layer_types + m->nblk);
+  for (uint8_t t : m->ltype)
+    if (t > 1) { delete m; return DORY_ERR_ARG; }
+  m->th_swa = cfg->rope_theta_swa;
+  m->th_full = cfg->rope_theta_full;
+
+  std::map<std::string, std::pair<const void*, int64_t>> tab;
+  for (int i = 0; i < n_tensors; ++i) {
+    if (!tensors[i].name || !tensors[i].d_ptr ||
+        ((uintptr_t)tensors[i].d_ptr & 15)) {
+      delete m;
+      return DORY_ERR_ARG;
+    }
+    tab[tensors[i].name] = {tensors[i].d_ptr, tensors[i].bytes};
+  }
+  bool ok = true;
+  auto get = [&](const std::string& n, int64_t bytes) -> const void* {
+    auto it = tab.find(n);
+    if (it == tab.end() || it->second.second != bytes) {
+      ok = false;
+      return nullptr;
+    }
+    return it->second.first;
+  };
+  m->embed = (const bf16*)get("embed", (int64_t)V * d * 2);
+  m->lm_head = (const bf16*)get("lm_head", (int64_t)V * d * 2);
+  m->s_z = (const float*)get("s_z", (int64_t)V * 4);
+  m->blk.resize(m->nblk);
+  for (int i = 0; i < m->nblk; ++i) {
+    const std::string p = "blk" + std::to_string(i) + ".";
+    BlockW& b = m->blk[i];
+    b.w_qkvg = (const bf16*)get(p + "w_qkvg", (int64_t)rows * d * 2);
+    b.s_q = (const float*)get(p + "s_q", (int64_t)Hq * hd * 4);
+    b.s_k = (const float*)get(p + "s_k", (int64_t)Hkv * hd * 4);
+    b.w_o = (const bf16*)get(p + "w_o", (int64_t)d * Hq * hd * 2);
+    b.alpha_a = (const float*)get(p + "alpha_a", (int64_t)d * 4);
+    b.w_gu = (const bf16*)get(p + "w_gu", (int64_t)2 * F * d * 2);
+    b.w_down = (const bf16*)get(p + "w_down", (int64_t)d * F * 2);
+    b.alpha_m = (const float*)get(p + "alpha_m", (int64_t)d * 4);
+  }
+  if (!ok) { delete m; return DORY_ERR_ARG; }
+
+  if (cudaGetDevice(&m->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&m->num_sms, cudaDevAttrMultiProcessorCount,
+                             m->device) != cudaSuccess ||
+      cudaGetSymbolAddress((void**)&m->d_status, g_dory_status) != cudaSuccess) {
+    delete m;
+    return DORY_ERR_CUDA;
+  }
+  const char* ng = getenv("DORY_NO_GRAPH");
+  m->use_graphs = !(ng && ng[0] == '1');
+  *out = m;
+  return DORY_OK;
+}
+
+void dory_free(dory_model* m) {
+  if (!m) return;
+  for (auto& kv : m->graphs)
+    if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+  if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
+  delete m;
+}
+
+int dory_kv_cache_bytes(const dory_model* m, int batch, int max_ctx,
+                        int max_chunk, int max_loops, int kv_mode,
+                        int64_t* bytes) {
+  if (!m || !bytes || batch < 1 || max_ctx < 1 || max_chunk < 1 ||
+      max_chunk > max_ctx || (kv_mode != 0 && kv_mode != 1))
+    return DORY_ERR_ARG;
+  if (kv_mode == DORY_KV_PER_LOOP && max_loops < 1) return DORY_ERR_ARG;
+  if (kv_mode == DORY_KV_LAST_LOOP) max_loops = 1;
+  *bytes = (int64_t)cache_layout(m, batch, max_ctx, max_chunk, max_loops,
+                                 kv_mode).total;
+  return DORY_OK;
+}
+
+int dory_kv_cache_bind(dory_model* m, void* d_buf, int64_t bytes, int batch,
+                       int max_ctx, int max_chunk, int max_loops, int kv_mode,
+                       void* stream, dory_cache** out) {
+  if (!out) return DORY_ERR_ARG;
+  *out = nullptr;
+  int64_t need = 0;
+  int rc = dory_kv_cache_bytes(m, batch, max_ctx, max_chunk, max_loops,
+                               kv_mode, &need);
+  if (rc) return rc;
+  if (!d_buf || ((uintptr_t)d_buf & 255) || bytes < need) return DORY_ERR_ARG;
+  if (kv_mode == DORY_KV_LAST_LOOP) max_loops = 1;
+  CacheLayout L = cache_layout(m, batch, max_ctx, max_chunk, max_loops, kv_mode);
+  dory_cache* c = new dory_cache();
+  c->m = m;
+  c->B = batch;
+  c->max_ctx = max_ctx;
+  c->max_chunk = max_chunk;
+  c->max_loops = max_loops;
+  c->kv_mode = kv_mode;
+  c->pages_per_seq = L.pages_per_seq;
+  c->swa_cap = L.swa_cap;
+  char* base = (char*)d_buf;
+  c->d_nctx = (int*)base;
+  c->d_block_table = (int*)(base + L.header);
+  c->slot_base = L.base;
+  for (size_t i = 0; i < L.k_off.size(); ++i)
+    c->slots.push_back(KVSlot{(bf16*)(base + L.k_off[i]),
+                              (bf16*)(base + L.v_off[i]), L.ring[i], L.cap[i]});
+  launch_cache_init(c->d_nctx, c->d_block_table, batch, L.pages_per_seq,
+                    (cudaStream_t)stream);
+  if (cudaGetLastError() != cudaSuccess) { delete c; return DORY_ERR_CUDA; }
+  *out = c;
+  return DORY_OK;
+}
+
+int dory_cache_length(const dory_cache* c, int* n_ctx) {
+  if (!c || !n_ctx) return DORY_ERR_ARG;
+  *n_ctx = c->n_ctx;
+  return DORY_OK;
+}
+
+int dory_cache_reset(dory_cache* c, void* stream) {
+  if (!c) return DORY_ERR_ARG;
+  c->n_ctx = 0;
+  c->loops_bound = 0;
+  launch_cache_init(c->d_nctx, c->d_block_table, c->B, c->pages_per_seq,
+                    (cudaStream_t)stream);
+  return cuda_rc(cudaGetLastError());
+}
+
+void dory_cache_free(dory_cache* c) {
+  if (!c) return;
+  dory_model* m = c->m;
+  for (auto it = m->graphs.begin(); it != m->graphs.end();) {
+    if (std::get<6>(it->first) == (const void*)c) {
+      if (it->second.exec) cudaGraphExecDestroy(it->second.exec);
+      it = m->graphs.erase(it);
+    } else {
+      ++it;
+    }
+  }
+  delete c;
+}
+
+int dory_workspace_bytes(const dory_model* m, int batch, int max_chunk,
+                         int64_t* bytes) {
+  if (!m || !bytes || batch < 1 || max_chunk < 1) return DORY_ERR_ARG;
+  *bytes = (int64_t)ws_layout(m, batch, max_chunk, nullptr).total;
+  return DORY_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+struct CallCtx {
+  dory_model* m;
+  dory_cache* c;
+  WS w;
+  int B, T, M, n_loops, logits_all;
+  const int* tokens;
+  float* logits;
+  int* argmax;
+  cudaStream_t st;
+};
+
+KVSlot slot_for(const dory_cache* c, int i, int t) {
+  int idx = c->slot_base[i];
+  if (is_rec(c->m, i) && c->kv_mode == DORY_KV_PER_LOOP) idx += t - 1;
+  return c->slots[idx];
+}
+
+bool use_gemv(int B, int T) { return T == 1 && B <= 8; }
+
+// Enqueue one forward pass: embedding, input blocks, n_loops passes of the
+// recurrent blocks with re-injection, output blocks, LM head.
+void enqueue_forward(const CallCtx& x) {
+  dory_model* m = x.m;
+  const Dims& dm = m->dm;
+  const WS& w = x.w;
+  const bool gemv = use_gemv(x.B, x.T);
+  const CacheGeo geo{x.c->d_nctx, x.c->d_block_table, x.c->pages_per_seq,
+                     x.c->max_ctx};
+  const int half = dm.hd / 2;
+  const float q_scale = sqrtf((float)dm.hd) * 1.4426950408889634f;
+  launch_rope_table(w.rope, geo, x.T, dm.hd, m->th_swa, m->th_full, x.st);
+  launch_embed(x.tokens, m->embed, x.M, dm.d, w.s0, w.s_bf, m->d_status, dm.V,
+               x.st);
+  float* cur = w.s0;
+  float* other = w.s1;
+  const float* prev_alpha = nullptr;
+  int prev_S = 1;
+
+  std::vector<std::pair<int, int>> order;
+  for (int i = 0; i < m->n_in; ++i) order.push_back({i, 0});
+  for (int t = 1; t <= x.n_loops; ++t)
+    for (int i = m->n_in; i < m->n_in + m->n_rec; ++i) order.push_back({i, t});
+  for (int i = m->n_in + m->n_rec; i < m->nblk; ++i) order.push_back({i, 0});
+
+  for (size_t k = 0; k < order.size(); ++k) {
+    const int i = order[k].first, t = order[k].second;
+    const BlockW& bw = m->blk[i];
+    int rj = RJ_NONE;
+    if (i == m->n_in) rj = (t == 1) ? RJ_FIRST : RJ_NEXT;
+    const bool full = m->ltype[i] == 1;
+    const KVSlot kv = slot_for(x.c, i, t);
+
+    // ---- attention sublayer -------------------------------------------
+    int S_qkvg = 1;
+    if (gemv) {
+      GemvArgs g{};
+      g.W = bw.w_qkvg; g.K = dm.d; g.n_items = dm.rows_qkvg; g.B = x.B;
+      g.epi = EPI_F32; g.S = S_qkvg = gemv_split(dm.d, dm.rows_qkvg);
+      g.out = w.qkvg;
+      if (k == 0) {
+        g.pro = PRO_BF16; g.xin = w.s_bf; g.xin_stride = dm.d;
+      } else {
+        g.pro = PRO_UPDATE; g.s_in = cur; g.h_in = w.h; g.h_S = prev_S;
+        g.alpha = prev_alpha; g.s_out = other; g.reinject = rj; g.x_buf = w.x;
+        std::swap(cur, other);
+      }
+      launch_gemv(g, gemv_grid(g, m->num_sms), x.st);
+    } else {
+      if (k > 0) {
+        launch_update_rows(cur, w.h, prev_alpha, other, w.s_bf, w.x, rj, x.M,
+                           dm.d, x.st);
+        std::swap(cur, other);
+      }
+      launch_gemm_bf16(w.s_bf, dm.d, bw.w_qkvg, w.qkvg, dm.rows_qkvg, x.M,
+                       dm.rows_qkvg, dm.d, nullptr, x.st);
+    }
+    QkvPostArgs qa{};
+    qa.qkvg = w.qkvg; qa.S = S_qkvg; qa.M = x.M; qa.T = x.T; qa.B = x.B;
+    qa.dm = dm; qa.s_q = bw.s_q; qa.s_k = bw.s_k;
+    qa.rope = w.rope + (full ? (size_t)x.T * half * 2 : 0);
+    qa.q_scale = q_scale; qa.q_out = w.q; qa.gate_out = w.gate;
+    qa.kv = kv; qa.g = geo; qa.err = m->d_status;
+    launch_qkv_post(qa, x.st);
+    AttnArgs aa{};
+    aa.q = w.q; aa.gate = w.gate; aa.B = x.B; aa.T = x.T; aa.dm = dm;
+    aa.window = full ? 0 : dm.window; aa.kv = kv; aa.g = geo;
+    aa.part_o = w.part_o; aa.part_ml = w.part_ml; aa.a_out = w.a;
+    aa.err = m->d_status;
+    if (x.T == 1) {
+      launch_attn_decode(aa, x.st);
+      launch_attn_combine(aa, x.st);
+    } else {
+      launch_attn_prefill(aa, x.st);
+    }
+    int S_o = 1;
+    if (gemv) {
+      GemvArgs g{};
+      g.W = bw.w_o; g.K = dm.qdim; g.n_items = dm.d; g.B = x.B; g.epi = EPI_F32;
+      g.S = S_o = gemv_split(dm.qdim, dm.d); g.out = w.h;
+      g.pro = PRO_BF16; g.xin = w.a; g.xin_stride = dm.qdim;
+      launch_gemv(g, gemv_grid(g, m->num_sms), x.st);
+    } else {
+      launch_gemm_bf16(w.a, dm.qdim, bw.w_o, w.h, dm.d, x.M, dm.d, dm.qdim,
+                       nullptr, x.st);
+    }
+
+    // ---- MLP sublayer ---------------------------------------------------
+    if (gemv) {
+      GemvArgs g{};
+      g.W = bw.w_gu; g.K = dm.d; g.n_items = dm.F; g.B = x.B;
+      g.epi = EPI_SWIGLU; g.pair_off = dm.F; g.S = 1; g.out_bf = w.mact;
+      g.pro = PRO_UPDATE; g.s_in = cur; g.h_in = w.h; g.h_S = S_o;
+      g.alpha = bw.alpha_a; g.s_out = other; g.reinject = RJ_NONE; g.x_buf = w.x;
+      std::swap(cur, other);
+      launch_gemv(g, gemv_grid(g, m->num_sms), x.st);
+      GemvArgs g2{};
+      g2.W = bw.w_down; g2.K = dm.F; g2.n_items = dm.d; g2.B = x.B;
+      g2.epi = EPI_F32; g2.S = prev_S = gemv_split(dm.F, dm.d); g2.out = w.h;
+      g2.pro = PRO_BF16; g2.xin = w.mact; g2.xin_stride = dm.F;
+      launch_gemv(g2, gemv_grid(g2, m->num_sms), x.st);
+    } else {
+      launch_update_rows(cur, w.h, bw.alpha_a, other, w.s_bf, w.x, RJ_NONE,
+                         x.M, dm.d, x.st);
+      std::swap(cur, other);
+      launch_gemm_bf16(w.s_bf, dm.d, bw.w_gu, w.gu, 2 * dm.F, x.M, 2 * dm.F,
+                       dm.d, nullptr, x.st);
+      launch_swiglu(w.gu, w.mact, x.M, dm.F, x.st);
+      launch_gemm_bf16(w.mact, dm.F, bw.w_down, w.h, dm.d, x.M, dm.d, dm.F,
+                       nullptr, x.st);
+      prev_S = 1;
+    }
+    prev_alpha = bw.alpha_m;
+  }
+
+  // ---- final update and LM head ------------------------------------------
+  if (gemv) {
+    GemvArgs g{};
+    g.W = m->lm_head; g.K = dm.d; g.n_items = dm.V; g.B = x.B; g.S = 1;
+    g.epi = EPI_LMHEAD; g.pro = PRO_UPDATE; g.s_in = cur; g.h_in = w.h;
+    g.h_S = prev_S; g.alpha = prev_alpha; g.s_out = w.sfin;
+    g.reinject = RJ_NONE; g.x_buf = w.x;
+    g.out = x.logits; g.out_stride = dm.V; g.col_scale = m->s_z;
+    g.amax_val = w.amax_val; g.amax_idx = w.amax_idx;
+    const int grid = gemv_grid(g, m->num_sms);
+    launch_gemv(g, grid, x.st);
+    if (x.argmax)
+      launch_argmax_partials(w.amax_val, w.amax_idx, x.B, grid, x.argmax, x.st);
+  } else {
+    launch_update_rows(cur, w.h, prev_alpha, w.sfin, w.s_bf, w.x, RJ_NONE, x.M,
+                       dm.d, x.st);
+    if (x.logits_all) {
+      launch_gemm_bf16(w.s_bf, dm.d, m->lm_head, x.logits, dm.V, x.M, dm.V,
+                       dm.d, m->s_z, x.st);
+      if (x.argmax) launch_argmax_rows(x.logits, x.M, dm.V, x.argmax, x.st);
+    } else {
+      for (int b0 = 0; b0 < x.B; b0 += 8) {
+        GemvArgs g{};
+        g.W = m->lm_head; g.K = dm.d; g.n_items = dm.V; g.S = 1;
+        g.B = std::min(8, x.B - b0); g.epi = EPI_LMHEAD; g.pro = PRO_BF16;
+        g.xin = w.s_bf + ((size_t)b0 * x.T + x.T - 1) * dm.d;
+        g.xin_stride = x.T * dm.d;
+        g.out = x.logits ? x.logits + (size_t)b0 * dm.V : nullptr;
+        g.out_stride = dm.V; g.col_scale = m->s_z;
+        g.amax_val = w.amax_val; g.amax_idx = w.amax_idx;
+        const int grid = gemv_grid(g, m->num_sms);
+        launch_gemv(g, grid, x.st);
+        if (x.argmax)
+          launch_argmax_partials(w.amax_val, w.amax_idx, g.B, grid,
+                                 x.argmax + b0, x.st);
+      }
+    }
+  }
+  launch_advance(x.c->d_nctx, x.T, x.st);
+}
+
+int run_call(dory_model* m, dory_cache* c, const int32_t* tokens, int B,
+             int T, int n_loops, int kv_mode, int logits_all, float* logits,
+             int32_t* argmax, void* ws, int64_t ws_bytes, void* stream,
+             bool decode) {
+  if (!m || !c || c->m != m || !tokens || !ws) return DORY_ERR_ARG;
+  if (B != c->B || T < 1 || T > c->max_chunk || n_loops < 1) return DORY_ERR_ARG;
+  if (logits_all && !logits) return DORY_ERR_ARG;
+  if ((uintptr_t)ws & 255) return DORY_ERR_ARG;
+  if (kv_mode != c->kv_mode) return DORY_ERR_CACHE;
+  if (kv_mode == DORY_KV_PER_LOOP &&
+      (n_loops > c->max_loops || (c->loops_bound && c->loops_bound != n_loops)))
+    return DORY_ERR_CACHE;
+  if ((int64_t)c->n_ctx + T > c->max_ctx) return DORY_ERR_CACHE;
+  const WS w = ws_layout(m, B, T, (char*)ws);
+  if ((int64_t)w.total > ws_bytes) return DORY_ERR_WORKSPACE;
+  CallCtx x{m, c, w, B, T, B * T, n_loops, logits_all, tokens, logits, argmax,
+            (cudaStream_t)stream};
+  cudaGetLastError();   // clear stale errors from earlier, unrelated calls
+
+  bool done = false;
+  if (decode && m->use_graphs) {
+    const GraphKey key(B, n_loops, tokens, logits, argmax, ws, c);
+    if (m->graphs.size() > 64 && !m->graphs.count(key)) {
+      for (auto& kv : m->graphs)
+        if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+      m->graphs.clear();
+    }
+    GraphEntry& ge = m->graphs[key];
+    if (!ge.exec && ge.seen >= 1) {
+      if (!m->cap_stream &&
+          cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) !=
+              cudaSuccess)
+        return DORY_ERR_CUDA;
+      CallCtx cx = x;
+      cx.st = m->cap_stream;
+      cudaGraph_t graph = nullptr;
+      if (cudaStreamBeginCapture(m->cap_stream,
+                                 cudaStreamCaptureModeThreadLocal) ==
+          cudaSuccess) {
+        enqueue_forward(cx);
+        const cudaError_t e1 = cudaStreamEndCapture(m->cap_stream, &graph);
+        if (e1 == cudaSuccess && graph &&
+            cudaGraphInstantiate(&ge.exec, graph, 0) != cudaSuccess)
+          ge.exec = nullptr;
+        if (graph) cudaGraphDestroy(graph);
+      }
+      cudaGetLastError();
+      if (!ge.exec) ge.seen = -1000000;   // never try this key again
+    }
+    if (ge.exec) {
+      if (cudaGraphLaunch(ge.exec, x.st) != cudaSuccess) return DORY_ERR_CUDA;
+      done = true;
+    } else {
+      ge.seen++;
+    }
+  }
+  if (!done) enqueue_forward(x);
+  if (cudaGetLastError() != cudaSuccess) return DORY_ERR_CUDA;
+  c->n_ctx += T;
+  if (kv_mode == DORY_KV_PER_LOOP && !c->loops_bound) c->loops_bound = n_loops;
+  return DORY_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dory_prefill(dory_model* m, dory_cache* c, const int32_t* d_tokens, int B,
+                 int T, int n_loops, int kv_mode, int logits_all,
+                 float* d_logits, int32_t* d_argmax, void* d_workspace,
+                 int64_t ws_bytes, void* stream) {
+  return run_call(m, c, d_tokens, B, T, n_loops, kv_mode, logits_all ? 1 : 0,
+                  d_logits, d_argmax, d_workspace, ws_bytes, stream, false);
+}
+
+int dory_decode_step(dory_model* m, dory_cache* c, const int32_t* d_tokens,
+                     int B, int n_loops, int kv_mode, float* d_logits,
+                     int32_t* d_argmax, void* d_workspace, int64_t ws_bytes,
+                     void* stream) {
+  return run_call(m, c, d_tokens, B, 1, n_loops, kv_mode, 0, d_logits,
+                  d_argmax, d_workspace, ws_bytes, stream, true);
+}
+
+int dory_copy_state(const dory_model* m, const void* d_workspace, int B,
+                    int T, int logits_all, float* d_out, void* stream) {
+  if (!m || !d_workspace || !d_out || B < 1 || T < 1) return DORY_ERR_ARG;
+  const WS w = ws_layout(m, B, T, (char*)d_workspace);
+  const size_t row = (size_t)m->dm.d * sizeof(float);
+  cudaError_t e;
+  if (use_gemv(B, T) || logits_all)
+    e = cudaMemcpyAsync(d_out, w.sfin, row * B * (logits_all ? T : 1),
+                        cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
+  else
+    e = cudaMemcpy2DAsync(d_out, row, w.sfin + (size_t)(T - 1) * m->dm.d,
+                          row * T, row, B, cudaMemcpyDeviceToDevice,
+                          (cudaStream_t)stream);
+  return cuda_rc(e);
+}
+
+int dory_sync_status(dory_model* m, void* stream) {
+  if (!m) return DORY_ERR_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dory_status, sizeof(int)) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  if (v) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(g_dory_status, &zero, sizeof(int));
+  }
+  if (v & ERRBIT_TIMEOUT) return DORY_ERR_TIMEOUT;
+  if (v) return DORY_ERR_DEVICE;
+  return DORY_OK;
+}
+
+}  // extern "C"

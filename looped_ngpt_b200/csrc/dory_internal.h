@@ -1,0 +1,151 @@
+// Internal interface between the C-ABI host layer (dory_api.cu) and the
+// sm_100a kernels.  Not installed; not part of the public ABI.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace dory {
+
+typedef __nv_bfloat16 bf16;
+
+// Device error bits (or-ed into the status word the host reads back).
+enum : int {
+  ERRBIT_BOUNDS = 1,   // a position or index fell outside its buffer
+  ERRBIT_TIMEOUT = 2,  // a bounded wait gave up
+};
+
+constexpr int kPage = 64;           // tokens per page of a full-attention cache
+constexpr int kMaxSplits = 64;      // decode attention: key splits per head
+constexpr int kMaxHeadDim = 256;
+
+struct Dims {
+  int d, Hq, Hkv, hd, F, V;
+  int qdim, kvdim, rows_qkvg;
+  int window;
+};
+
+// One attention layer-slot of the KV cache.  ring = 1: sliding-window ring
+// [B][Hkv][cap][hd]; ring = 0: pages [n_pages][Hkv][kPage][hd] reached
+// through the cache's block table.
+struct KVSlot {
+  bf16* K;
+  bf16* V;
+  int ring;
+  int cap;
+};
+
+struct CacheGeo {
+  int* n_ctx;                // device: tokens held per sequence
+  const int* block_table;    // device: [B][pages_per_seq]
+  int pages_per_seq;
+  int max_ctx;
+};
+
+__device__ __forceinline__ size_t kv_index(const KVSlot& s, const CacheGeo& g,
+                                           int Hkv, int hd, int b, int kvh,
+                                           int p) {
+  if (s.ring) {
+    int slot = p % s.cap;
+    return ((size_t)(b * Hkv + kvh) * s.cap + slot) * hd;
+  }
+  int page = g.block_table[b * g.pages_per_seq + p / kPage];
+  return (((size_t)page * Hkv + kvh) * kPage + (p % kPage)) * hd;
+}
+
+// ---------------------------------------------------------------- GEMV ----
+enum GemvPro : int { PRO_BF16 = 0, PRO_UPDATE = 1 };
+enum GemvEpi : int { EPI_F32 = 0, EPI_SWIGLU = 1, EPI_LMHEAD = 2 };
+enum Reinject : int { RJ_NONE = 0, RJ_FIRST = 1, RJ_NEXT = 2 };
+
+struct GemvArgs {
+  const bf16* W;       // [N_rows, K] row-major
+  int K;               // contraction length (multiple of 256 * S)
+  int n_items;         // output rows (EPI_SWIGLU: pairs n, n + pair_off)
+  int S;               // split-K factor (EPI_F32 only)
+  int B;               // batch rows, <= 8
+  int pair_off;        // EPI_SWIGLU
+  // prologue
+  int pro;
+  const bf16* xin;     // PRO_BF16: [B][xin_stride]
+  int xin_stride;
+  const float* s_in;   // PRO_UPDATE: current state [B][K]
+  const float* h_in;   // sublayer output partials [h_S][B][K]
+  int h_S;
+  const float* alpha;  // [K]
+  float* s_out;        // [B][K] (written by block 0)
+  int reinject;
+  float* x_buf;        // [B][K] input-block output (RJ_FIRST writes it)
+  // epilogue
+  int epi;
+  float* out;          // EPI_F32: [S][B][n_items]; EPI_LMHEAD: logits
+                       // [B][out_stride] or null
+  int out_stride;
+  bf16* out_bf;        // EPI_SWIGLU: [B][pair_off]
+  const float* col_scale;   // EPI_LMHEAD: s_z [n_items]
+  float* amax_val;     // EPI_LMHEAD: [B][gridDim]
+  int* amax_idx;
+};
+int gemv_grid(const GemvArgs& a, int num_sms);
+void launch_gemv(const GemvArgs& a, int grid, cudaStream_t st);
+
+// ------------------------------------------------------------- rowwise ----
+// RoPE cos/sin for positions n_ctx + t, t < T; table [2][T][hd/2][2].
+void launch_rope_table(float* table, const CacheGeo& g, int T, int hd,
+                       double theta_swa, double theta_full, cudaStream_t st);
+// x0 = N(E[tok]) -> s (f32) and s_bf (bf16), rows M.
+void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
+                  bf16* s_bf, int* err, int vocab, cudaStream_t st);
+// RoPE + per-head L2 norm + q/k scales + sigmoid gate + K/V cache write.
+struct QkvPostArgs {
+  const float* qkvg; int S; int M; int T; int B;
+  Dims dm;
+  const float* s_q; const float* s_k;
+  const float* rope;   // table of this layer's type [T][hd/2][2]
+  float q_scale;       // extra factor folded into q (softmax temperature)
+  float* q_out;        // [M][qdim]
+  float* gate_out;     // [M][qdim]
+  KVSlot kv; CacheGeo g;
+  int* err;
+};
+void launch_qkv_post(const QkvPostArgs& a, cudaStream_t st);
+// Prefill: s_new = N(s + alpha (N(h) - s)) per row (+ loop re-injection).
+void launch_update_rows(const float* s_in, const float* h, const float* alpha,
+                        float* s_out, bf16* s_bf, float* x_buf, int reinject,
+                        int M, int d, cudaStream_t st);
+// m = silu(gu[:, :F]) * gu[:, F:] (bf16), rows M.
+void launch_swiglu(const float* gu, bf16* m, int M, int F, cudaStream_t st);
+// Final greedy argmax over [B][n] partials or full logits rows.
+void launch_argmax_partials(const float* val, const int* idx, int B, int n,
+                            int* out, cudaStream_t st);
+void launch_argmax_rows(const float* logits, int rows, int V, int* out,
+                        cudaStream_t st);
+void launch_advance(int* n_ctx, int T, cudaStream_t st);
+void launch_cache_init(int* n_ctx, int* block_table, int B, int pages_per_seq,
+                       cudaStream_t st);
+
+// ----------------------------------------------------------- attention ----
+struct AttnArgs {
+  const float* q;      // [M][qdim], scaled by sqrt(hd) * log2(e)
+  const float* gate;   // [M][qdim] sigmoid(g)
+  int B, T;
+  Dims dm;
+  int window;          // 0 = full attention
+  KVSlot kv; CacheGeo g;
+  float* part_o;       // decode: [B][Hq][kMaxSplits][hd]
+  float* part_ml;      // decode: [B][Hq][kMaxSplits][2]
+  bf16* a_out;         // [M][qdim] = gate * attention output
+  int* err;
+};
+void launch_attn_decode(const AttnArgs& a, cudaStream_t st);
+void launch_attn_combine(const AttnArgs& a, cudaStream_t st);
+void launch_attn_prefill(const AttnArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- GEMM ----
+// C[M, N] (f32, row stride ldc) = A[M, K] (bf16, row stride lda) * W[N, K]^T
+// optionally times col_scale[n].  M any, N % 128 == 0, K % 32 == 0.
+void launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
+                      int M, int N, int K, const float* col_scale,
+                      cudaStream_t st);
+
+}  // namespace dory

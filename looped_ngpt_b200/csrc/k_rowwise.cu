@@ -1,0 +1,272 @@
+// Row-wise kernels of the looped nGPT forward pass: embedding, RoPE table,
+// RoPE + per-head QK L2 norm + K/V cache write, the prefill nGPT update,
+// SwiGLU, greedy argmax and cache bookkeeping.  All are HBM/L2-bound and
+// touch each element once.
+#include "common.cuh"
+
+namespace dory {
+
+namespace {
+
+// cos/sin of (n_ctx + t) * theta^(-2i/hd) for both attention types.  The
+// angle is formed in double precision: at positions ~1e5 a float angle
+// would be off by ~1e-2 rad.
+__global__ void rope_table_kernel(float* table, const int* n_ctx, int T,
+                                  int half, double th_swa, double th_full) {
+  const int total = 2 * T * half;
+  const int p0 = *n_ctx;
+  for (int id = blockIdx.x * blockDim.x + threadIdx.x; id < total;
+       id += gridDim.x * blockDim.x) {
+    const int type = id / (T * half);
+    const int rem = id - type * T * half;
+    const int t = rem / half, i = rem - t * half;
+    const double theta = type ? th_full : th_swa;
+    const double inv = pow(theta, -2.0 * i / (2.0 * half));
+    double s, c;
+    sincos((double)(p0 + t) * inv, &s, &c);
+    table[2 * id] = (float)c;
+    table[2 * id + 1] = (float)s;
+  }
+}
+
+// x0 = N(E[tok]); one block per row.
+__global__ void embed_kernel(const int* tokens, const bf16* E, int d,
+                             int vocab, float* s, bf16* s_bf, int* err) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  int tok = tokens[row];
+  if (tok < 0 || tok >= vocab) {
+    if (threadIdx.x == 0) atomicOr(err, ERRBIT_BOUNDS);
+    tok = 0;
+  }
+  const bf16* e = E + (size_t)tok * d;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    const float v = __bfloat162float(e[i]);
+    ss += v * v;
+  }
+  const float inv = 1.f / fmaxf(sqrtf(block_sum(ss, red)), 1e-12f);
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    const float v = __bfloat162float(e[i]) * inv;
+    s[(size_t)row * d + i] = v;
+    s_bf[(size_t)row * d + i] = __float2bfloat16_rn(v);
+  }
+}
+
+constexpr int kPairs = kMaxHeadDim / 64;   // rotate-half pairs per lane
+
+// One warp per (row, head item).  Items: [0, Hq) q heads, [Hq, Hq+Hkv) k
+// heads, [Hq+Hkv, Hq+2Hkv) v heads, [Hq+2Hkv, 2Hq+2Hkv) gate heads.
+__global__ void qkv_post_kernel(const QkvPostArgs a) {
+  const Dims& dm = a.dm;
+  const int lane = threadIdx.x & 31;
+  const int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int n_items = 2 * dm.Hq + 2 * dm.Hkv;
+  const int row = blockIdx.y;
+  if (item >= n_items) return;
+  const int b = row / a.T, t = row - b * a.T;
+  const int p = *a.g.n_ctx + t;
+  const int hd = dm.hd, half = hd / 2;
+  const size_t part = (size_t)a.M * dm.rows_qkvg;
+  const float* src = a.qkvg + (size_t)row * dm.rows_qkvg;
+
+  int col0, kind, head;
+  if (item < dm.Hq) { kind = 0; head = item; col0 = head * hd; }
+  else if (item < dm.Hq + dm.Hkv) {
+    kind = 1; head = item - dm.Hq; col0 = dm.qdim + head * hd;
+  } else if (item < dm.Hq + 2 * dm.Hkv) {
+    kind = 2; head = item - dm.Hq - dm.Hkv; col0 = dm.qdim + dm.kvdim + head * hd;
+  } else {
+    kind = 3; head = item - dm.Hq - 2 * dm.Hkv;
+    col0 = dm.qdim + 2 * dm.kvdim + head * hd;
+  }
+  auto load = [&](int c) {
+    float v = 0.f;
+    for (int s = 0; s < a.S; ++s) v += src[s * part + col0 + c];
+    return v;
+  };
+
+  if (kind == 3) {
+    for (int c = lane; c < hd; c += 32)
+      a.gate_out[(size_t)row * dm.qdim + head * hd + c] = sigmoidf_(load(c));
+    return;
+  }
+  if (p >= a.g.max_ctx) {
+    if (lane == 0) atomicOr(a.err, ERRBIT_BOUNDS);
+    return;
+  }
+  if (kind == 2) {
+    bf16* dst = a.kv.V + kv_index(a.kv, a.g, dm.Hkv, hd, b, head, p);
+    for (int c = lane; c < hd; c += 32) dst[c] = __float2bfloat16_rn(load(c));
+    return;
+  }
+  // q or k: rotate-half RoPE, then L2 norm over the head, then scale.
+  float r1[kPairs], r2[kPairs];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < kPairs; ++j) {
+    const int i = lane + 32 * j;
+    r1[j] = r2[j] = 0.f;
+    if (i < half) {
+      const float x1 = load(i), x2 = load(i + half);
+      const float c = a.rope[(t * half + i) * 2], s = a.rope[(t * half + i) * 2 + 1];
+      r1[j] = x1 * c - x2 * s;
+      r2[j] = x2 * c + x1 * s;
+      ss += r1[j] * r1[j] + r2[j] * r2[j];
+    }
+  }
+  const float inv = 1.f / fmaxf(sqrtf(warp_sum(ss)), 1e-12f);
+  if (kind == 0) {
+    const float* sc = a.s_q + head * hd;
+    float* dst = a.q_out + (size_t)row * dm.qdim + head * hd;
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+      const int i = lane + 32 * j;
+      if (i < half) {
+        dst[i] = r1[j] * inv * sc[i] * a.q_scale;
+        dst[i + half] = r2[j] * inv * sc[i + half] * a.q_scale;
+      }
+    }
+  } else {
+    const float* sc = a.s_k + head * hd;
+    bf16* dst = a.kv.K + kv_index(a.kv, a.g, dm.Hkv, hd, b, head, p);
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+      const int i = lane + 32 * j;
+      if (i < half) {
+        dst[i] = __float2bfloat16_rn(r1[j] * inv * sc[i]);
+        dst[i + half] = __float2bfloat16_rn(r2[j] * inv * sc[i + half]);
+      }
+    }
+  }
+}
+
+__global__ void update_rows_kernel(const float* s_in, const float* h,
+                                   const float* alpha, float* s_out,
+                                   bf16* s_bf, float* x_buf, int reinject,
+                                   int d) {
+  extern __shared__ float tmp[];
+  __shared__ float red[32];
+  const size_t o = (size_t)blockIdx.x * d;
+  ngpt_update_row(s_in + o, h + o, 1, 0, alpha, d, reinject,
+                  reinject == RJ_NONE ? nullptr : x_buf + o, s_out + o,
+                  s_bf + o, tmp, red);
+}
+
+__global__ void swiglu_kernel(const float* gu, bf16* m, int M, int F) {
+  const size_t total = (size_t)M * F;
+  for (size_t id = blockIdx.x * (size_t)blockDim.x + threadIdx.x; id < total;
+       id += (size_t)gridDim.x * blockDim.x) {
+    const size_t r = id / F, c = id - r * F;
+    const float g = gu[r * 2 * F + c], u = gu[r * 2 * F + F + c];
+    m[id] = __float2bfloat16_rn(g * sigmoidf_(g) * u);
+  }
+}
+
+// Lowest index among the maxima; NaN entries never win.
+__device__ __forceinline__ void better(float& v, int& i, float cv, int ci) {
+  if (cv > v || (cv == v && ci < i)) { v = cv; i = ci; }
+}
+
+__device__ void block_argmax(float v, int i, int* out) {
+  __shared__ float sv[32];
+  __shared__ int si[32];
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+    better(v, i, ov, oi);
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) { sv[w] = v; si[w] = i; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int k = 0; k < (int)(blockDim.x >> 5); ++k) better(bv, bi, sv[k], si[k]);
+    *out = bi == 0x7fffffff ? 0 : bi;
+  }
+}
+
+__global__ void argmax_partials_kernel(const float* val, const int* idx,
+                                       int n, int* out) {
+  const int b = blockIdx.x;
+  float v = -INFINITY;
+  int i = 0x7fffffff;
+  for (int k = threadIdx.x; k < n; k += blockDim.x)
+    better(v, i, val[b * n + k], idx[b * n + k]);
+  block_argmax(v, i, out + b);
+}
+
+__global__ void argmax_rows_kernel(const float* z, int V, int* out) {
+  const size_t r = blockIdx.x;
+  float v = -INFINITY;
+  int i = 0x7fffffff;
+  for (int k = threadIdx.x; k < V; k += blockDim.x) better(v, i, z[r * V + k], k);
+  block_argmax(v, i, out + r);
+}
+
+__global__ void advance_kernel(int* n_ctx, int T) { *n_ctx += T; }
+
+__global__ void cache_init_kernel(int* n_ctx, int* bt, int total) {
+  const int id = blockIdx.x * blockDim.x + threadIdx.x;
+  if (id == 0) *n_ctx = 0;
+  if (id < total) bt[id] = id;     // sequence b owns pages [b*P, (b+1)*P)
+}
+
+}  // namespace
+
+void launch_rope_table(float* table, const CacheGeo& g, int T, int hd,
+                       double theta_swa, double theta_full, cudaStream_t st) {
+  const int total = 2 * T * (hd / 2);
+  const int blocks = (total + 255) / 256;
+  rope_table_kernel<<<blocks < 1184 ? blocks : 1184, 256, 0, st>>>(
+      table, g.n_ctx, T, hd / 2, theta_swa, theta_full);
+}
+
+void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
+                  bf16* s_bf, int* err, int vocab, cudaStream_t st) {
+  embed_kernel<<<M, 256, 0, st>>>(tokens, E, d, vocab, s, s_bf, err);
+}
+
+void launch_qkv_post(const QkvPostArgs& a, cudaStream_t st) {
+  const int items = 2 * a.dm.Hq + 2 * a.dm.Hkv;
+  dim3 grid((items + 7) / 8, a.M);
+  qkv_post_kernel<<<grid, 256, 0, st>>>(a);
+}
+
+void launch_update_rows(const float* s_in, const float* h, const float* alpha,
+                        float* s_out, bf16* s_bf, float* x_buf, int reinject,
+                        int M, int d, cudaStream_t st) {
+  update_rows_kernel<<<M, 256, d * sizeof(float), st>>>(
+      s_in, h, alpha, s_out, s_bf, x_buf, reinject, d);
+}
+
+void launch_swiglu(const float* gu, bf16* m, int M, int F, cudaStream_t st) {
+  const size_t total = (size_t)M * F;
+  size_t blocks = (total + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  swiglu_kernel<<<(int)blocks, 256, 0, st>>>(gu, m, M, F);
+}
+
+void launch_argmax_partials(const float* val, const int* idx, int B, int n,
+                            int* out, cudaStream_t st) {
+  argmax_partials_kernel<<<B, 256, 0, st>>>(val, idx, n, out);
+}
+
+void launch_argmax_rows(const float* logits, int rows, int V, int* out,
+                        cudaStream_t st) {
+  argmax_rows_kernel<<<rows, 256, 0, st>>>(logits, V, out);
+}
+
+void launch_advance(int* n_ctx, int T, cudaStream_t st) {
+  advance_kernel<<<1, 1, 0, st>>>(n_ctx, T);
+}
+
+void launch_cache_init(int* n_ctx, int* block_table, int B, int pages_per_seq,
+                       cudaStream_t st) {
+  const int total = B * pages_per_seq;
+  cache_init_kernel<<<(total + 255) / 256 + 1, 256, 0, st>>>(n_ctx, block_table,
+                                                             total);
+}
+
+}  // namespace dory
