@@ -62,8 +62,19 @@ def gpu_run(gm, prompt, n_loops, kv_mode, toks, chunks=None, max_ctx=None):
 
 
 def compare(z_gpu, z_ref, label):
+    """Element-wise logits bound, and a valid greedy pick at every position:
+    the GPU's top-1 token must score within LOGIT_TOL of the oracle's best
+    (with random-init weights the top two logits can be closer than BF16
+    rounding, and then either token is a correct argmax).  Returns
+    (max|dz|, raw top-1 agreements, positions) for pooled agreement checks."""
     d = float(np.abs(z_gpu - z_ref).max())
-    top = float(np.mean(np.argmax(z_gpu, -1) == np.argmax(z_ref, -1)))
+    g = np.argmax(z_gpu, -1)
+    r = np.argmax(z_ref, -1)
+    picked = np.take_along_axis(z_ref, g[..., None], -1)[..., 0]
+    slack = float((z_ref.max(-1) - picked).max())
+    agree = int(np.sum(g == r))
+    print(f"{label}: max|dz| {d:.3e}  top-1 {agree}/{g.size}  "
+          f"worst pick slack {slack:.2e}")
     assert d <= LOGIT_TOL, f"{label}: max|dz| {d:.3e} > {LOGIT_TOL}"
-    assert top >= TOP1_MIN, f"{label}: top-1 agreement {top:.4f}"
-    return d, top
+    assert slack <= LOGIT_TOL, f"{label}: a greedy pick is {slack:.3e} below"
+    return d, agree, g.size
