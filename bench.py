@@ -1,0 +1,371 @@
+#!/usr/bin/env python
+"""Benchmark of the elastic-depth forward pass of the Dory-shape looped nGPT.
+
+Workload (one B200 per rank): Dory1.0-4B shapes (d 2560, 16/4 heads of 160,
+blocks 8/20/8, SwiGLU 10240, vocab 131072), seeded random-init BF16 weights,
+batch 1, a 2048-token uniform-random prompt, then greedy decode, last_loop KV
+cache, at k = 1, 2 and 4 loops.  A step is one decode step: one token through
+embedding, 16 + 20k blocks and the LM head.  The headline value is decode
+tokens/s at k = 2 (the recommended default loop count); decode and prefill
+tokens/s at every k and their roofline fractions are in "breakdown".
+
+More than one GPU: independent replicas (one per rank, no collective on the
+data path); the value is the sum of tokens over ranks / the slowest rank's
+time.  `--impl reference` times the CPU oracle on a bounded sample instead.
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("decode tok/s & prefill tok/s at k=1/2/4 (1 B200); "
+          "% of HBM / TC roofline")
+PROMPT = 2048
+HEADLINE_K = 2
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--impl", default="dory", choices=["dory", "reference"])
+    ap.add_argument("--loops", default="1,2,4")
+    ap.add_argument("--kv-mode", default="last_loop")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prompt", type=int, default=PROMPT)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,"
+         "clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 8:
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[4 + i].lower().startswith("active")})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(
+                    ".", "").isdigit() else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------------ ranks --
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device(f"cuda:{local}"))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info()
+             if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+# --------------------------------------------------------------- oracle arm --
+def oracle_decode_sample(w, n_loops, tokens=1):
+    """Time the oracle on a bounded sample of the decode workload: `tokens`
+    decode steps from an empty cache (context 1..tokens)."""
+    from oracle.model import Model
+    from synthetic import DORY
+    m = Model(DORY, w, batch=1, kv_mode="last_loop")
+    t0 = time.perf_counter()
+    tok = 7
+    for _ in range(tokens):
+        z = m.decode_step([tok], n_loops)
+        tok = int(np.argmax(z[0]))
+    dt = time.perf_counter() - t0
+    return tokens / dt, dt
+
+
+# ------------------------------------------------------------------ GPU arm --
+def run_gpu(args, rank, world, local):
+    import torch
+    import looped_ngpt_b200 as lb
+    from synthetic import DORY, make_weights, make_prompt
+
+    hbm_peak, tc_peak, peak_kind = peaks()
+    w = make_weights(DORY, seed=0)
+    dev = torch.device(f"cuda:{local}")
+    gm = lb.DoryModel(DORY, w, device=dev)
+    prompt = torch.from_numpy(make_prompt(DORY, 1, args.prompt)).to(dev)
+    ks = [int(k) for k in args.loops.split(",")]
+    if HEADLINE_K not in ks:
+        ks.append(HEADLINE_K)
+    K, W = args.steps, args.warmup
+    max_ctx = args.prompt + 2 * (W + K) + 16
+    ws = gm.workspace(1, args.prompt)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    out = {"decode_tok_s": {}, "prefill_tok_s": {}, "decode_hbm_frac": {},
+           "prefill_tc_frac": {}, "decode_bytes_per_token": {},
+           "prefill_flops": {}}
+    headline = None
+    for k in ks:
+        cache = gm.new_cache(1, max_ctx, args.prompt, kv_mode=args.kv_mode,
+                             max_loops=k)
+        # prefill: one warm-up call, one timed, one profiled (counts FLOPs)
+        t_pre = None
+        for rep in range(3):
+            cache.reset()
+            if rep == 2:
+                gm.profile(True)
+            torch.cuda.synchronize()
+            e0, e1 = ev(), ev()
+            e0.record()
+            _, am = gm.prefill(cache, prompt, k, ws)
+            e1.record()
+            torch.cuda.synchronize()
+            if rep == 1:
+                t_pre = e0.elapsed_time(e1) / 1e3
+        pst = gm.profile_read()
+        gm.profile(False)
+        pflops = sum(v["flops"] for v in pst.values())
+        out["prefill_tok_s"][f"k{k}"] = args.prompt / t_pre
+        out["prefill_flops"][f"k{k}"] = pflops
+        out["prefill_tc_frac"][f"k{k}"] = pflops / t_pre / (tc_peak * 1e12)
+        # decode: the argmax of each step is written straight into the token
+        # buffer that the next step reads
+        gm.decode_step(cache, am, k, ws, want_logits=False)
+        tok = cache._dec_bufs[0]
+        for _ in range(W):
+            gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
+        clocks = Clocks(local) if k == HEADLINE_K else None
+        torch.cuda.synchronize()
+        barrier(world)
+        if clocks:
+            clocks.start()
+        e0, e1 = ev(), ev()
+        e0.record()
+        for _ in range(K):
+            gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        dt = e0.elapsed_time(e1) / 1e3
+        ck = clocks.stop() if clocks else None
+        # profiled steps (eager, CUDA events around each kernel)
+        gm.profile(True)
+        P = 4
+        for _ in range(P):
+            gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
+        st = gm.profile_read()
+        gm.profile(False)
+        assert gm.sync_status() == 0, "device-side check failed"
+        bytes_tok = sum(v["bytes"] for v in st.values()) / P
+        out["decode_tok_s"][f"k{k}"] = K / dt
+        out["decode_bytes_per_token"][f"k{k}"] = bytes_tok
+        out["decode_hbm_frac"][f"k{k}"] = bytes_tok * K / dt / (hbm_peak * 1e9)
+        if k == HEADLINE_K:
+            headline = dict(dt=dt, clocks=ck, stats=st, P=P, cache=cache,
+                            launches=sum(v["launches"] for v in st.values()) / P)
+    # end-to-end through host buffers at the headline k
+    k = HEADLINE_K
+    cache = headline["cache"]
+    cache.reset()
+    _, am = gm.prefill(cache, prompt, k, ws)
+    host_tok = torch.empty(1, dtype=torch.int32, pin_memory=True)
+    host_out = torch.empty(1, dtype=torch.int32, pin_memory=True)
+    host_tok.copy_(am.cpu())
+    tok = cache._dec_bufs[0]
+    for _ in range(W):
+        tok.copy_(host_tok, non_blocking=True)
+        gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
+        host_out.copy_(tok, non_blocking=True)
+        torch.cuda.synchronize()
+        host_tok.copy_(host_out)
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = time.perf_counter()
+    for _ in range(K):
+        tok.copy_(host_tok, non_blocking=True)
+        gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
+        host_out.copy_(tok, non_blocking=True)
+        torch.cuda.synchronize()
+        host_tok.copy_(host_out)
+    e2e_dt = time.perf_counter() - t0
+    barrier(world)
+    return dict(out=out, headline=headline, e2e_dt=e2e_dt, w=w,
+                hbm_peak=hbm_peak, tc_peak=tc_peak, peak_kind=peak_kind)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return main_reference(args)
+    rank, world, local = dist_setup()
+    r = run_gpu(args, rank, world, local)
+    h = r["headline"]
+    dt = max_over_ranks(h["dt"], world)
+    K, W = args.steps, args.warmup
+    value = world * K / dt
+    e2e_dt = max_over_ranks(r["e2e_dt"], world)
+    st = h["stats"]
+    # dominant kernel: largest share of the profiled step time
+    dom = max(st, key=lambda n: st[n]["ms"])
+    d = st[dom]
+    bound = "hbm" if d["flops"] / max(d["bytes"], 1) < 100 else "tensor"
+    if bound == "hbm":
+        achieved = d["bytes"] / d["launches"] / (d["ms"] / d["launches"] / 1e3) / 1e9
+        peak, unit = r["hbm_peak"], "GB/s"
+    else:
+        achieved = d["flops"] / d["launches"] / (d["ms"] / d["launches"] / 1e3) / 1e12
+        peak, unit = r["tc_peak"], "TFLOP/s"
+    total_ms = sum(v["ms"] for v in st.values())
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, secs = oracle_decode_sample(r["w"], HEADLINE_K, tokens=1)
+        cpu = {"value": tps, "unit": "tok/s", "cores": blas_threads(),
+               "kind": "oracle",
+               "sample": f"1 decode step at k={HEADLINE_K} from an empty "
+                         f"cache, Dory-shape weights ({secs:.1f} s of CPU)"}
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": dt / K * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": (f"Dory-shape BF16 looped nGPT decode, batch 1 "
+                                f"per GPU after a {args.prompt}-token prompt, "
+                                f"k={HEADLINE_K}, {args.kv_mode}"),
+                   "global_batch": world, "seq_len": args.prompt,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "no flush: 12 GB of weights streamed per token > L2"},
+        "roofline": {"bound": bound, "kernel": dom, "achieved": achieved,
+                     "peak": peak, "unit": unit, "frac": achieved / peak,
+                     "peak_source": r["peak_kind"], "traffic": None,
+                     "share_of_step": d["ms"] / total_ms},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * K / e2e_dt, "unit": "tok/s",
+                "h2d_bytes_per_step": 4, "d2h_bytes_per_step": 4},
+        "gpu_launches": int(round(h["launches"] * K)),
+        "clocks": h["clocks"],
+        "breakdown": r["out"],
+        "kernels": {n: {"launches_per_step": v["launches"] / h["P"],
+                        "us_per_step": v["ms"] / h["P"] * 1e3,
+                        "GBps": v["bytes"] / (v["ms"] / 1e3) / 1e9
+                        if v["ms"] > 0 else None}
+                    for n, v in sorted(st.items(), key=lambda kv: -kv[1]["ms"])},
+    }
+    print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main_reference(args):
+    """The oracle on the host cores: bounded decode samples of the same
+    workload (Dory shapes, k=2), same metric and unit."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from synthetic import DORY, make_weights
+    w = make_weights(DORY, seed=0)
+    K, W = max(1, min(args.steps, 2)), max(0, min(args.warmup, 1))
+    for _ in range(W):
+        oracle_decode_sample(w, HEADLINE_K, tokens=1)
+    tps, secs = oracle_decode_sample(w, HEADLINE_K, tokens=K)
+    sample = (f"{K} decode steps at k={HEADLINE_K} from an empty cache, "
+              f"Dory-shape weights, fp64 NumPy ({secs:.1f} s)")
+    line = {"metric": METRIC, "value": tps, "unit": "tok/s", "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": secs / K * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": (f"Dory-shape looped nGPT decode, batch 1, "
+                                    f"k={HEADLINE_K}, last_loop"),
+                       "global_batch": 1, "seq_len": args.prompt,
+                       "parallelism": "none"},
+            "cpu_baseline": {"value": tps, "unit": "tok/s",
+                             "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": tps, "unit": "tok/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

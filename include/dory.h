@@ -158,6 +158,25 @@ int dory_copy_state(const dory_model* m, const void* d_workspace, int B,
  * failed synchronisation returns DORY_ERR_CUDA.  The word is cleared. */
 int dory_sync_status(dory_model* m, void* stream);
 
+/* Per-kernel timing (tracing aid).  While enabled, every call launches its
+ * kernels eagerly (no graph replay), each bracketed by CUDA events on the
+ * call's stream, and records the kernel's algorithmic bytes (weights, KV
+ * entries and activations it must move) and FLOPs. */
+typedef struct {
+  char name[32];      /* kernel class, e.g. "gemv_gateup", "attn_decode"   */
+  int64_t launches;
+  double total_ms;    /* summed event-measured durations                  */
+  double bytes;       /* summed algorithmic bytes                          */
+  double flops;       /* summed algorithmic FLOPs                          */
+} dory_kernel_stat;
+
+int dory_profile_enable(dory_model* m, int on);
+
+/* Synchronise `stream`, aggregate the recorded launches by kernel class
+ * into out[0..max) (*n = classes written) and clear the record. */
+int dory_profile_read(dory_model* m, dory_kernel_stat* out, int max, int* n,
+                      void* stream);
+
 const char* dory_strerror(int code);
 void dory_cache_free(dory_cache* c);
 void dory_free(dory_model* m);

@@ -31,6 +31,12 @@ class DoryTensor(Structure):
     _fields_ = [("name", c_char_p), ("d_ptr", c_void_p), ("bytes", c_int64)]
 
 
+class DoryKernelStat(Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", c_int64),
+                ("total_ms", c_double), ("bytes", c_double),
+                ("flops", c_double)]
+
+
 _P = c_void_p
 _I64P = POINTER(c_int64)
 SIGNATURES = {
@@ -49,6 +55,9 @@ SIGNATURES = {
                                  c_int64, _P]),
     "dory_copy_state": (c_int, [_P, _P, c_int, c_int, c_int, _P, _P]),
     "dory_sync_status": (c_int, [_P, _P]),
+    "dory_profile_enable": (c_int, [_P, c_int]),
+    "dory_profile_read": (c_int, [_P, POINTER(DoryKernelStat), c_int,
+                                  POINTER(c_int), _P]),
     "dory_strerror": (c_char_p, [c_int]),
     "dory_cache_free": (None, [_P]),
     "dory_free": (None, [_P]),

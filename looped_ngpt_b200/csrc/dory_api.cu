@@ -51,6 +51,16 @@ struct dory_model {
   bool use_graphs = true;
   cudaStream_t cap_stream = nullptr;
   std::map<GraphKey, GraphEntry> graphs;
+  // per-kernel timing (dory_profile_enable)
+  struct ProfRec {
+    std::string name;
+    cudaEvent_t a, b;
+    double bytes, flops;
+  };
+  bool prof = false;
+  std::vector<ProfRec> prof_recs;
+  std::vector<cudaEvent_t> ev_pool;
+  size_t ev_used = 0;
 };
 
 struct dory_cache {
@@ -171,6 +181,44 @@ int cuda_rc(cudaError_t e) { return e == cudaSuccess ? DORY_OK : DORY_ERR_CUDA; 
 
 extern "C" {
 
+int dory_profile_enable(dory_model* m, int on) {
+  if (!m) return DORY_ERR_ARG;
+  m->prof = on != 0;
+  return DORY_OK;
+}
+
+int dory_profile_read(dory_model* m, dory_kernel_stat* out, int max, int* n,
+                      void* stream) {
+  if (!m || !n || (max > 0 && !out)) return DORY_ERR_ARG;
+  *n = 0;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  std::vector<dory_kernel_stat> agg;
+  std::map<std::string, size_t> where;
+  for (auto& r : m->prof_recs) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) continue;
+    auto it = where.find(r.name);
+    if (it == where.end()) {
+      dory_kernel_stat st{};
+      std::snprintf(st.name, sizeof(st.name), "%s", r.name.c_str());
+      where[r.name] = agg.size();
+      agg.push_back(st);
+      it = where.find(r.name);
+    }
+    dory_kernel_stat& st = agg[it->second];
+    st.launches += 1;
+    st.total_ms += ms;
+    st.bytes += r.bytes;
+    st.flops += r.flops;
+  }
+  m->prof_recs.clear();
+  m->ev_used = 0;
+  cudaGetLastError();
+  for (size_t i = 0; i < agg.size() && (int)i < max; ++i) out[(*n)++] = agg[i];
+  return DORY_OK;
+}
+
 const char* dory_strerror(int code) {
   switch (code) {
     case DORY_OK: return "ok";
@@ -275,6 +323,7 @@ void dory_free(dory_model* m) {
   for (auto& kv : m->graphs)
     if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
+  for (cudaEvent_t e : m->ev_pool) cudaEventDestroy(e);
   delete m;
 }
 
@@ -366,11 +415,64 @@ int dory_workspace_bytes(const dory_model* m, int batch, int max_chunk,
 
 namespace {
 
+// Brackets one launch with CUDA events when profiling is on.
+struct Prof {
+  dory_model* m;
+  cudaStream_t st;
+  long idx = -1;
+  Prof(dory_model* mm, cudaStream_t s, const char* name, double bytes,
+       double flops)
+      : m(mm), st(s) {
+    if (!m->prof) return;
+    while (m->ev_pool.size() < m->ev_used + 2) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) return;
+      m->ev_pool.push_back(e);
+    }
+    dory_model::ProfRec r{name, m->ev_pool[m->ev_used], m->ev_pool[m->ev_used + 1],
+                          bytes, flops};
+    m->ev_used += 2;
+    cudaEventRecord(r.a, st);
+    m->prof_recs.push_back(r);
+    idx = (long)m->prof_recs.size() - 1;
+  }
+  ~Prof() {
+    if (idx >= 0) cudaEventRecord(m->prof_recs[idx].b, st);
+  }
+};
+
+double gemv_bytes(const GemvArgs& g, int rows) {
+  const double w = (double)rows * g.K * 2;
+  const double in = g.pro == PRO_UPDATE ? (double)g.B * g.K * 4 * (3 + g.h_S)
+                                        : (double)g.B * g.K * 2;
+  double out;
+  if (g.epi == EPI_SWIGLU) out = (double)g.B * g.n_items * 2;
+  else if (g.epi == EPI_LMHEAD) out = g.out ? (double)g.B * g.n_items * 4 : 0;
+  else out = (double)g.S * g.B * g.n_items * 4;
+  return w + in + out;
+}
+
+void gemv_run(dory_model* m, const GemvArgs& g, int grid, cudaStream_t st,
+              const char* name) {
+  const int rows = g.epi == EPI_SWIGLU ? 2 * g.n_items : g.n_items;
+  Prof p(m, st, name, gemv_bytes(g, rows), 2.0 * rows * g.K * g.B);
+  launch_gemv(g, grid, st);
+}
+
+void gemm_run(dory_model* m, const bf16* A, int lda, const bf16* W, float* C,
+              int ldc, int M, int N, int K, const float* scale,
+              cudaStream_t st, const char* name) {
+  Prof p(m, st, name,
+         (double)M * K * 2 + (double)N * K * 2 + (double)M * N * 4,
+         2.0 * M * N * K);
+  launch_gemm_bf16(A, lda, W, C, ldc, M, N, K, scale, st);
+}
+
 struct CallCtx {
   dory_model* m;
   dory_cache* c;
   WS w;
-  int B, T, M, n_loops, logits_all;
+  int B, T, M, n_loops, logits_all, n_ctx0;
   const int* tokens;
   float* logits;
   int* argmax;
@@ -396,9 +498,15 @@ void enqueue_forward(const CallCtx& x) {
                      x.c->max_ctx};
   const int half = dm.hd / 2;
   const float q_scale = sqrtf((float)dm.hd) * 1.4426950408889634f;
-  launch_rope_table(w.rope, geo, x.T, dm.hd, m->th_swa, m->th_full, x.st);
-  launch_embed(x.tokens, m->embed, x.M, dm.d, w.s0, w.s_bf, m->d_status, dm.V,
-               x.st);
+  {
+    Prof p(m, x.st, "rope_table", 16.0 * x.T * half, 0);
+    launch_rope_table(w.rope, geo, x.T, dm.hd, m->th_swa, m->th_full, x.st);
+  }
+  {
+    Prof p(m, x.st, "embed", (double)x.M * dm.d * 8, 0);
+    launch_embed(x.tokens, m->embed, x.M, dm.d, w.s0, w.s_bf, m->d_status,
+                 dm.V, x.st);
+  }
   float* cur = w.s0;
   float* other = w.s1;
   const float* prev_alpha = nullptr;
@@ -432,15 +540,16 @@ void enqueue_forward(const CallCtx& x) {
         g.alpha = prev_alpha; g.s_out = other; g.reinject = rj; g.x_buf = w.x;
         std::swap(cur, other);
       }
-      launch_gemv(g, gemv_grid(g, m->num_sms), x.st);
+      gemv_run(m, g, gemv_grid(g, m->num_sms), x.st, "gemv_qkvg");
     } else {
       if (k > 0) {
+        Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
         launch_update_rows(cur, w.h, prev_alpha, other, w.s_bf, w.x, rj, x.M,
                            dm.d, x.st);
         std::swap(cur, other);
       }
-      launch_gemm_bf16(w.s_bf, dm.d, bw.w_qkvg, w.qkvg, dm.rows_qkvg, x.M,
-                       dm.rows_qkvg, dm.d, nullptr, x.st);
+      gemm_run(m, w.s_bf, dm.d, bw.w_qkvg, w.qkvg, dm.rows_qkvg, x.M,
+               dm.rows_qkvg, dm.d, nullptr, x.st, "gemm_qkvg");
     }
     QkvPostArgs qa{};
     qa.qkvg = w.qkvg; qa.S = S_qkvg; qa.M = x.M; qa.T = x.T; qa.B = x.B;
@@ -448,16 +557,39 @@ void enqueue_forward(const CallCtx& x) {
     qa.rope = w.rope + (full ? (size_t)x.T * half * 2 : 0);
     qa.q_scale = q_scale; qa.q_out = w.q; qa.gate_out = w.gate;
     qa.kv = kv; qa.g = geo; qa.err = m->d_status;
-    launch_qkv_post(qa, x.st);
+    {
+      Prof p(m, x.st, "qkv_post",
+             (double)x.M * (dm.rows_qkvg * 4.0 * S_qkvg + dm.qdim * 8.0 +
+                            dm.kvdim * 4.0), 0);
+      launch_qkv_post(qa, x.st);
+    }
     AttnArgs aa{};
     aa.q = w.q; aa.gate = w.gate; aa.B = x.B; aa.T = x.T; aa.dm = dm;
     aa.window = full ? 0 : dm.window; aa.kv = kv; aa.g = geo;
     aa.part_o = w.part_o; aa.part_ml = w.part_ml; aa.a_out = w.a;
     aa.err = m->d_status;
     if (x.T == 1) {
-      launch_attn_decode(aa, x.st);
+      const double nk = full ? x.n_ctx0 + 1.0
+                             : std::min(x.n_ctx0 + 1.0, (double)dm.window);
+      {
+        Prof p(m, x.st, "attn_decode",
+               x.B * (dm.Hkv * nk * dm.hd * 4.0 + dm.qdim * 4.0),
+               4.0 * x.B * dm.Hq * nk * dm.hd);
+        launch_attn_decode(aa, x.st);
+      }
+      Prof p(m, x.st, "attn_combine", x.B * dm.qdim * 10.0, 0);
       launch_attn_combine(aa, x.st);
     } else {
+      double vis = 0;
+      for (int t = 0; t < x.T; ++t) {
+        const double q = x.n_ctx0 + t + 1.0;
+        vis += full ? q : std::min(q, (double)dm.window);
+      }
+      const double lo = full ? 0 : std::max(0, x.n_ctx0 - dm.window + 1);
+      const double keys = x.n_ctx0 + x.T - lo;
+      Prof p(m, x.st, "attn_prefill",
+             x.B * (dm.Hkv * keys * dm.hd * 4.0) + x.M * dm.qdim * 10.0,
+             4.0 * x.B * dm.Hq * vis * dm.hd);
       launch_attn_prefill(aa, x.st);
     }
     int S_o = 1;
@@ -466,10 +598,10 @@ void enqueue_forward(const CallCtx& x) {
       g.W = bw.w_o; g.K = dm.qdim; g.n_items = dm.d; g.B = x.B; g.epi = EPI_F32;
       g.S = S_o = gemv_split(dm.qdim, dm.d); g.out = w.h;
       g.pro = PRO_BF16; g.xin = w.a; g.xin_stride = dm.qdim;
-      launch_gemv(g, gemv_grid(g, m->num_sms), x.st);
+      gemv_run(m, g, gemv_grid(g, m->num_sms), x.st, "gemv_o");
     } else {
-      launch_gemm_bf16(w.a, dm.qdim, bw.w_o, w.h, dm.d, x.M, dm.d, dm.qdim,
-                       nullptr, x.st);
+      gemm_run(m, w.a, dm.qdim, bw.w_o, w.h, dm.d, x.M, dm.d, dm.qdim, nullptr,
+               x.st, "gemm_o");
     }
 
     // ---- MLP sublayer ---------------------------------------------------
@@ -480,21 +612,27 @@ void enqueue_forward(const CallCtx& x) {
       g.pro = PRO_UPDATE; g.s_in = cur; g.h_in = w.h; g.h_S = S_o;
       g.alpha = bw.alpha_a; g.s_out = other; g.reinject = RJ_NONE; g.x_buf = w.x;
       std::swap(cur, other);
-      launch_gemv(g, gemv_grid(g, m->num_sms), x.st);
+      gemv_run(m, g, gemv_grid(g, m->num_sms), x.st, "gemv_gateup");
       GemvArgs g2{};
       g2.W = bw.w_down; g2.K = dm.F; g2.n_items = dm.d; g2.B = x.B;
       g2.epi = EPI_F32; g2.S = prev_S = gemv_split(dm.F, dm.d); g2.out = w.h;
       g2.pro = PRO_BF16; g2.xin = w.mact; g2.xin_stride = dm.F;
-      launch_gemv(g2, gemv_grid(g2, m->num_sms), x.st);
+      gemv_run(m, g2, gemv_grid(g2, m->num_sms), x.st, "gemv_down");
     } else {
-      launch_update_rows(cur, w.h, bw.alpha_a, other, w.s_bf, w.x, RJ_NONE,
-                         x.M, dm.d, x.st);
+      {
+        Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
+        launch_update_rows(cur, w.h, bw.alpha_a, other, w.s_bf, w.x, RJ_NONE,
+                           x.M, dm.d, x.st);
+      }
       std::swap(cur, other);
-      launch_gemm_bf16(w.s_bf, dm.d, bw.w_gu, w.gu, 2 * dm.F, x.M, 2 * dm.F,
-                       dm.d, nullptr, x.st);
-      launch_swiglu(w.gu, w.mact, x.M, dm.F, x.st);
-      launch_gemm_bf16(w.mact, dm.F, bw.w_down, w.h, dm.d, x.M, dm.d, dm.F,
-                       nullptr, x.st);
+      gemm_run(m, w.s_bf, dm.d, bw.w_gu, w.gu, 2 * dm.F, x.M, 2 * dm.F, dm.d,
+               nullptr, x.st, "gemm_gateup");
+      {
+        Prof p(m, x.st, "swiglu", (double)x.M * dm.F * 10, 0);
+        launch_swiglu(w.gu, w.mact, x.M, dm.F, x.st);
+      }
+      gemm_run(m, w.mact, dm.F, bw.w_down, w.h, dm.d, x.M, dm.d, dm.F, nullptr,
+               x.st, "gemm_down");
       prev_S = 1;
     }
     prev_alpha = bw.alpha_m;
@@ -510,16 +648,24 @@ void enqueue_forward(const CallCtx& x) {
     g.out = x.logits; g.out_stride = dm.V; g.col_scale = m->s_z;
     g.amax_val = w.amax_val; g.amax_idx = w.amax_idx;
     const int grid = gemv_grid(g, m->num_sms);
-    launch_gemv(g, grid, x.st);
-    if (x.argmax)
+    gemv_run(m, g, grid, x.st, "gemv_lmhead");
+    if (x.argmax) {
+      Prof p(m, x.st, "argmax", x.B * grid * 8.0, 0);
       launch_argmax_partials(w.amax_val, w.amax_idx, x.B, grid, x.argmax, x.st);
+    }
   } else {
-    launch_update_rows(cur, w.h, prev_alpha, w.sfin, w.s_bf, w.x, RJ_NONE, x.M,
-                       dm.d, x.st);
+    {
+      Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
+      launch_update_rows(cur, w.h, prev_alpha, w.sfin, w.s_bf, w.x, RJ_NONE,
+                         x.M, dm.d, x.st);
+    }
     if (x.logits_all) {
-      launch_gemm_bf16(w.s_bf, dm.d, m->lm_head, x.logits, dm.V, x.M, dm.V,
-                       dm.d, m->s_z, x.st);
-      if (x.argmax) launch_argmax_rows(x.logits, x.M, dm.V, x.argmax, x.st);
+      gemm_run(m, w.s_bf, dm.d, m->lm_head, x.logits, dm.V, x.M, dm.V, dm.d,
+               m->s_z, x.st, "gemm_lmhead");
+      if (x.argmax) {
+        Prof p(m, x.st, "argmax", (double)x.M * dm.V * 4, 0);
+        launch_argmax_rows(x.logits, x.M, dm.V, x.argmax, x.st);
+      }
     } else {
       for (int b0 = 0; b0 < x.B; b0 += 8) {
         GemvArgs g{};
@@ -531,13 +677,16 @@ void enqueue_forward(const CallCtx& x) {
         g.out_stride = dm.V; g.col_scale = m->s_z;
         g.amax_val = w.amax_val; g.amax_idx = w.amax_idx;
         const int grid = gemv_grid(g, m->num_sms);
-        launch_gemv(g, grid, x.st);
-        if (x.argmax)
+        gemv_run(m, g, grid, x.st, "gemv_lmhead");
+        if (x.argmax) {
+          Prof p(m, x.st, "argmax", g.B * grid * 8.0, 0);
           launch_argmax_partials(w.amax_val, w.amax_idx, g.B, grid,
                                  x.argmax + b0, x.st);
+        }
       }
     }
   }
+  Prof p(m, x.st, "advance", 8, 0);
   launch_advance(x.c->d_nctx, x.T, x.st);
 }
 
@@ -556,12 +705,12 @@ int run_call(dory_model* m, dory_cache* c, const int32_t* tokens, int B,
   if ((int64_t)c->n_ctx + T > c->max_ctx) return DORY_ERR_CACHE;
   const WS w = ws_layout(m, B, T, (char*)ws);
   if ((int64_t)w.total > ws_bytes) return DORY_ERR_WORKSPACE;
-  CallCtx x{m, c, w, B, T, B * T, n_loops, logits_all, tokens, logits, argmax,
-            (cudaStream_t)stream};
+  CallCtx x{m, c, w, B, T, B * T, n_loops, logits_all, c->n_ctx, tokens,
+            logits, argmax, (cudaStream_t)stream};
   cudaGetLastError();   // clear stale errors from earlier, unrelated calls
 
   bool done = false;
-  if (decode && m->use_graphs) {
+  if (decode && m->use_graphs && !m->prof) {
     const GraphKey key(B, n_loops, tokens, logits, argmax, ws, c);
     if (m->graphs.size() > 64 && !m->graphs.count(key)) {
       for (auto& kv : m->graphs)

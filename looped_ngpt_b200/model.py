@@ -167,6 +167,23 @@ class DoryModel:
             _stream_ptr(stream)))
         return out
 
+    def profile(self, on=True):
+        """dory_profile_enable: per-kernel CUDA-event timing of later calls."""
+        check("dory_profile_enable",
+              _lib.load().dory_profile_enable(self.handle, 1 if on else 0))
+
+    def profile_read(self, stream=None):
+        """dory_profile_read -> {kernel class: {launches, ms, bytes, flops}}."""
+        arr = (_lib.DoryKernelStat * 64)()
+        n = ctypes.c_int()
+        check("dory_profile_read", _lib.load().dory_profile_read(
+            self.handle, arr, 64, ctypes.byref(n), _stream_ptr(stream)))
+        return {arr[i].name.decode(): dict(launches=arr[i].launches,
+                                           ms=arr[i].total_ms,
+                                           bytes=arr[i].bytes,
+                                           flops=arr[i].flops)
+                for i in range(n.value)}
+
     def sync_status(self, stream=None):
         return _lib.load().dory_sync_status(self.handle, _stream_ptr(stream))
 

@@ -73,31 +73,23 @@ def make_tensor(shape, name, seed=0):
     raise ValueError(kind)
 
 
-def _one(args):
-    shape, name, seed = args
-    return name, make_tensor(shape, name, seed)
-
-
 def make_weights(shape, seed=0, names=None, workers=None):
     """All (or the listed) tensors as {name: ndarray}.
 
-    ``workers`` > 1 draws tensors in a spawn-started process pool (never a
-    fork: a process forked after CUDA initialisation can hang).
+    ``workers`` > 1 draws tensors on a thread pool: NumPy's generator and the
+    array arithmetic release the GIL, so threads scale without copying the
+    tensors between processes.
     """
     names = list(names) if names is not None else tensor_names(shape)
     if workers is None:
         big = shape.params_per_block() * shape.n_blocks > 50_000_000
-        workers = min(16, os.cpu_count() or 1) if big else 1
+        workers = min(32, os.cpu_count() or 1) if big else 1
     if workers <= 1:
         return {n: make_tensor(shape, n, seed) for n in names}
-    import multiprocessing as mp
-    from concurrent.futures import ProcessPoolExecutor
-    ctx = mp.get_context("spawn")
-    out = {}
-    with ProcessPoolExecutor(max_workers=workers, mp_context=ctx) as ex:
-        for n, t in ex.map(_one, [(shape, n, seed) for n in names]):
-            out[n] = t
-    return out
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        outs = list(ex.map(lambda n: make_tensor(shape, n, seed), names))
+    return dict(zip(names, outs))
 
 
 def make_prompt(shape, batch, length, seed=1):
