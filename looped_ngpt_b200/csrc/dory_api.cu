@@ -6,6 +6,8 @@
 #include <cstring>
 #include <cmath>
 #include <map>
+#include <mutex>
+#include <set>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -51,6 +53,7 @@ struct dory_model {
   bool use_graphs = true;
   cudaStream_t cap_stream = nullptr;
   std::map<GraphKey, GraphEntry> graphs;
+  std::set<dory_cache*> caches;   // bound caches, detached by dory_free
   // per-kernel timing (dory_profile_enable)
   struct ProfRec {
     std::string name;
@@ -320,6 +323,7 @@ int dory_init_weights(const dory_config* cfg, const dory_tensor* tensors,
 
 void dory_free(dory_model* m) {
   if (!m) return;
+  for (dory_cache* c : m->caches) c->m = nullptr;   // caches may outlive m
   for (auto& kv : m->graphs)
     if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
@@ -371,6 +375,7 @@ int dory_kv_cache_bind(dory_model* m, void* d_buf, int64_t bytes, int batch,
   launch_cache_init(c->d_nctx, c->d_block_table, batch, L.pages_per_seq,
                     (cudaStream_t)stream);
   if (cudaGetLastError() != cudaSuccess) { delete c; return DORY_ERR_CUDA; }
+  m->caches.insert(c);
   *out = c;
   return DORY_OK;
 }
@@ -382,7 +387,7 @@ int dory_cache_length(const dory_cache* c, int* n_ctx) {
 }
 
 int dory_cache_reset(dory_cache* c, void* stream) {
-  if (!c) return DORY_ERR_ARG;
+  if (!c || !c->m) return DORY_ERR_ARG;
   c->n_ctx = 0;
   c->loops_bound = 0;
   launch_cache_init(c->d_nctx, c->d_block_table, c->B, c->pages_per_seq,
@@ -393,6 +398,11 @@ int dory_cache_reset(dory_cache* c, void* stream) {
 void dory_cache_free(dory_cache* c) {
   if (!c) return;
   dory_model* m = c->m;
+  if (!m) {             // its model was freed first
+    delete c;
+    return;
+  }
+  m->caches.erase(c);
   for (auto it = m->graphs.begin(); it != m->graphs.end();) {
     if (std::get<6>(it->first) == (const void*)c) {
       if (it->second.exec) cudaGraphExecDestroy(it->second.exec);
@@ -806,3 +816,4 @@ int dory_sync_status(dory_model* m, void* stream) {
 }
 
 }  // extern "C"
+
