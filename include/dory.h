@@ -158,6 +158,32 @@ int dory_copy_state(const dory_model* m, const void* d_workspace, int B,
  * failed synchronisation returns DORY_ERR_CUDA.  The word is cleared. */
 int dory_sync_status(dory_model* m, void* stream);
 
+/* Allocation-free decode step.  The pages have no counterpart: this entry
+ * exists for callers that cannot call cudaMalloc (for example code running
+ * under an allocator that owns all device memory, or a host process that
+ * must not grow its device footprint after start-up), so they cannot provide
+ * the workspace that dory_decode_step takes.  It runs the same kernels as
+ * dory_decode_step with the workspace taken from a library-owned static
+ * device array of DORY_STATIC_WS_BYTES bytes; every GPU that loads the
+ * library holds that array until the process exits.  The caller still
+ * passes the cache, the tokens and the outputs.
+ *   - The first call on a device looks up that device's copy of the array
+ *     (cudaGetSymbolAddress, with the device current); make that first call
+ *     before any stream capture.
+ *   - Returns DORY_ERR_WORKSPACE when dory_workspace_bytes(m, B, 1) exceeds
+ *     DORY_STATIC_WS_BYTES; other errors as dory_decode_step.
+ *   - Calls no cudaMalloc/cudaFree or other allocating routine (with
+ *     profiling off, the default), and launches every kernel directly.
+ *   - All calls share the one array: calls that may overlap on the GPU (on
+ *     different streams, or from several threads) race and must be ordered
+ *     by the caller.  Nothing in the array needs to start at zero: each call
+ *     writes every word it reads before reading it. */
+#define DORY_STATIC_WS_BYTES (8 << 20)
+int dory_decode_step_static(dory_model* m, dory_cache* c,
+                            const int32_t* d_tokens, int B, int n_loops,
+                            int kv_mode, float* d_logits, int32_t* d_argmax,
+                            void* stream);
+
 /* Per-kernel timing (tracing aid).  While enabled, every call launches its
  * kernels eagerly (no graph replay), each bracketed by CUDA events on the
  * call's stream, and records the kernel's algorithmic bytes (weights, KV

@@ -53,6 +53,8 @@ SIGNATURES = {
                              _P, _P, _P, c_int64, _P]),
     "dory_decode_step": (c_int, [_P, _P, _P, c_int, c_int, c_int, _P, _P, _P,
                                  c_int64, _P]),
+    "dory_decode_step_static": (c_int, [_P, _P, _P, c_int, c_int, c_int, _P,
+                                        _P, _P]),
     "dory_copy_state": (c_int, [_P, _P, c_int, c_int, c_int, _P, _P]),
     "dory_sync_status": (c_int, [_P, _P]),
     "dory_profile_enable": (c_int, [_P, c_int]),

@@ -817,3 +817,52 @@ int dory_sync_status(dory_model* m, void* stream) {
 
 }  // extern "C"
 
+// ---------------------------------------------------------------------------
+// Allocation-free decode step (dory_decode_step_static).  Its workspace is a
+// file-scope device array; host code reaches it only through the address
+// that cudaGetSymbolAddress returns for the current device (the symbol's
+// name in host code is a host-side stand-in, not a device address).
+static __device__ __align__(256) unsigned char g_static_ws[DORY_STATIC_WS_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_ws_mu;
+void* g_static_ws_addr[kMaxDevices];
+
+// Device address of this device's copy of g_static_ws, looked up once per
+// device with that device current.
+int static_ws_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DORY_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DORY_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_ws_mu);
+  if (!g_static_ws_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || !p)
+      return DORY_ERR_CUDA;
+    g_static_ws_addr[dev] = p;
+  }
+  *out = g_static_ws_addr[dev];
+  return DORY_OK;
+}
+
+}  // namespace
+
+extern "C" int dory_decode_step_static(dory_model* m, dory_cache* c,
+                                       const int32_t* d_tokens, int B,
+                                       int n_loops, int kv_mode,
+                                       float* d_logits, int32_t* d_argmax,
+                                       void* stream) {
+  if (!m || !c || B < 1) return DORY_ERR_ARG;
+  int64_t need = 0;
+  const int rc0 = dory_workspace_bytes(m, B, 1, &need);
+  if (rc0) return rc0;
+  if (need > (int64_t)DORY_STATIC_WS_BYTES) return DORY_ERR_WORKSPACE;
+  void* ws = nullptr;
+  const int rc = static_ws_address(&ws);
+  if (rc) return rc;
+  // decode = false: the kernels are launched directly, never via a graph.
+  return run_call(m, c, d_tokens, B, 1, n_loops, kv_mode, 0, d_logits,
+                  d_argmax, ws, (int64_t)DORY_STATIC_WS_BYTES, stream, false);
+}
