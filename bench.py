@@ -42,6 +42,15 @@ def parse():
     ap.add_argument("--kv-mode", default="last_loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prompt", type=int, default=PROMPT)
+    ap.add_argument("--profile-decode", type=int, default=0, metavar="K",
+                    help="only: prefill, warm up, then one decode step at "
+                         "k=K inside the NVTX range 'decode_step' (for ncu)")
+    ap.add_argument("--profile-blocks", default="",
+                    help="profile runs only: input,recurrent,output block "
+                         "counts of a reduced-depth Dory-width model")
+    ap.add_argument("--profile-prefill", type=int, default=0, metavar="K",
+                    help="only: one prefill at k=K inside the NVTX range "
+                         "'prefill' (for ncu)")
     return ap.parse_args()
 
 
@@ -269,10 +278,48 @@ def run_gpu(args, rank, world, local):
                 hbm_peak=hbm_peak, tc_peak=tc_peak, peak_kind=peak_kind)
 
 
+def profile_run(args):
+    """A minimal run for profilers: one NVTX-marked decode step or prefill."""
+    import torch
+    import looped_ngpt_b200 as lb
+    from synthetic import DORY, make_weights, make_prompt, dory_with_blocks
+    shape = DORY
+    if args.profile_blocks:
+        shape = dory_with_blocks(*[int(x) for x in args.profile_blocks.split(",")])
+    w = make_weights(shape, seed=0)
+    gm = lb.DoryModel(shape, w, device="cuda:0")
+    prompt = torch.from_numpy(make_prompt(shape, 1, args.prompt)).to("cuda:0")
+    k = args.profile_decode or args.profile_prefill
+    cache = gm.new_cache(1, args.prompt + 64, args.prompt, kv_mode=args.kv_mode,
+                         max_loops=k)
+    ws = gm.workspace(1, args.prompt)
+    if args.profile_prefill:
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_push("prefill")
+        gm.prefill(cache, prompt, k, ws)
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
+        return 0
+    _, am = gm.prefill(cache, prompt, k, ws)
+    gm.decode_step(cache, am, k, ws, want_logits=False)
+    tok = cache._dec_bufs[0]
+    for _ in range(3):
+        gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("decode_step")
+    gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
+    assert gm.sync_status() == 0
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return main_reference(args)
+    if args.profile_decode or args.profile_prefill:
+        return profile_run(args)
     rank, world, local = dist_setup()
     r = run_gpu(args, rank, world, local)
     h = r["headline"]

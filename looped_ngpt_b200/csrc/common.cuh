@@ -48,6 +48,28 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return r;
 }
 
+// Programmatic dependent launch.  Every kernel of the forward pass is
+// launched so that it may start while its predecessor is still running.
+// Rule used throughout: before pdl_wait() a kernel touches only immutable
+// data (weights) or data written by kernels that finished before its
+// predecessor started; it calls pdl_trigger() only after pdl_wait(), so at
+// most one kernel runs ahead of the one it depends on.  Both are no-ops when
+// the kernel was launched without the attribute.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Ask L2 to start fetching [p, p + bytes) (no data returned).  p and bytes
+// must be multiples of 16.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  if (bytes == 0) return;
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ float sigmoidf_(float x) {
   return 1.f / (1.f + __expf(-x));
 }

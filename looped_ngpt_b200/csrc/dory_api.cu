@@ -19,6 +19,16 @@ using namespace dory;
 
 static __device__ int g_dory_status;   // or-ed ERRBIT_* from device checks
 
+namespace dory {
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("DORY_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+}  // namespace dory
+
 namespace {
 
 struct BlockW {
@@ -128,19 +138,13 @@ CacheLayout cache_layout(const dory_model* m, int B, int max_ctx,
   return L;
 }
 
-int gemv_split(int K, int n_items) {
-  int S = 1;
-  while (S < 8 && K % (2 * S * 256) == 0 && K / (2 * S) >= 1024 &&
-         (long)n_items * S < 8192)
-    S *= 2;
-  return S;
-}
 
 struct WS {
   float *s0, *s1, *sfin, *x, *qkvg, *q, *gate, *h, *gu, *part_o, *part_ml,
       *rope, *amax_val;
   bf16 *s_bf, *a, *mact;
   int* amax_idx;
+  int* counters;
   size_t total;
 };
 
@@ -174,6 +178,7 @@ WS ws_layout(const dory_model* m, int B, int T, char* base) {
   w.rope = (float*)take((size_t)2 * T * (dm.hd / 2) * 2 * 4);
   w.amax_val = (float*)take((size_t)B * kArgmaxSlots * 4);
   w.amax_idx = (int*)take((size_t)B * kArgmaxSlots * 4);
+  w.counters = (int*)take((size_t)B * dm.Hkv * 4);
   w.total = off;
   return w;
 }
@@ -252,7 +257,8 @@ int dory_init_weights(const dory_config* cfg, const dory_tensor* tensors,
   if (Hq % Hkv) return DORY_ERR_ARG;
   if (cfg->wfmt != DORY_W_BF16) return DORY_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
-  if (!(hd == 64 || hd == 128 || hd == 160) || G > 8 || G * hd > 1024)
+  if (!(hd == 64 || hd == 128 || hd == 160) ||
+      !(G == 1 || G == 2 || G == 4 || G == 8) || G * hd > 1024)
     return DORY_ERR_UNSUPPORTED;
   if (d % 256 || F % 256 || (Hq * hd) % 256 || V % 128 || d > 8192 ||
       F > 32768)
@@ -462,11 +468,17 @@ double gemv_bytes(const GemvArgs& g, int rows) {
   return w + in + out;
 }
 
-void gemv_run(dory_model* m, const GemvArgs& g, int grid, cudaStream_t st,
-              const char* name) {
+// Launches the GEMV; returns the number of K segments (partials) it writes.
+int gemv_run(dory_model* m, const GemvArgs& g0, cudaStream_t st,
+             const char* name) {
+  GemvArgs g = g0;
+  g.err = m->d_status;
+  g.S = gemv_splits(g);
+  const int grid = gemv_grid(g, m->num_sms);
   const int rows = g.epi == EPI_SWIGLU ? 2 * g.n_items : g.n_items;
   Prof p(m, st, name, gemv_bytes(g, rows), 2.0 * rows * g.K * g.B);
   launch_gemv(g, grid, st);
+  return g.S;
 }
 
 void gemm_run(dory_model* m, const bf16* A, int lda, const bf16* W, float* C,
@@ -508,14 +520,15 @@ void enqueue_forward(const CallCtx& x) {
                      x.c->max_ctx};
   const int half = dm.hd / 2;
   const float q_scale = sqrtf((float)dm.hd) * 1.4426950408889634f;
-  {
+  if (x.T > 1) {
     Prof p(m, x.st, "rope_table", 16.0 * x.T * half, 0);
     launch_rope_table(w.rope, geo, x.T, dm.hd, m->th_swa, m->th_full, x.st);
   }
   {
     Prof p(m, x.st, "embed", (double)x.M * dm.d * 8, 0);
     launch_embed(x.tokens, m->embed, x.M, dm.d, w.s0, w.s_bf, m->d_status,
-                 dm.V, x.st);
+                 dm.V, w.counters, x.B * dm.Hkv, x.T == 1 ? w.rope : nullptr,
+                 geo.n_ctx, dm.hd, m->th_swa, m->th_full, x.st);
   }
   float* cur = w.s0;
   float* other = w.s1;
@@ -541,7 +554,7 @@ void enqueue_forward(const CallCtx& x) {
     if (gemv) {
       GemvArgs g{};
       g.W = bw.w_qkvg; g.K = dm.d; g.n_items = dm.rows_qkvg; g.B = x.B;
-      g.epi = EPI_F32; g.S = S_qkvg = gemv_split(dm.d, dm.rows_qkvg);
+      g.epi = EPI_F32;
       g.out = w.qkvg;
       if (k == 0) {
         g.pro = PRO_BF16; g.xin = w.s_bf; g.xin_stride = dm.d;
@@ -550,7 +563,7 @@ void enqueue_forward(const CallCtx& x) {
         g.alpha = prev_alpha; g.s_out = other; g.reinject = rj; g.x_buf = w.x;
         std::swap(cur, other);
       }
-      gemv_run(m, g, gemv_grid(g, m->num_sms), x.st, "gemv_qkvg");
+      S_qkvg = gemv_run(m, g, x.st, "gemv_qkvg");
     } else {
       if (k > 0) {
         Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
@@ -561,35 +574,37 @@ void enqueue_forward(const CallCtx& x) {
       gemm_run(m, w.s_bf, dm.d, bw.w_qkvg, w.qkvg, dm.rows_qkvg, x.M,
                dm.rows_qkvg, dm.d, nullptr, x.st, "gemm_qkvg");
     }
-    QkvPostArgs qa{};
-    qa.qkvg = w.qkvg; qa.S = S_qkvg; qa.M = x.M; qa.T = x.T; qa.B = x.B;
-    qa.dm = dm; qa.s_q = bw.s_q; qa.s_k = bw.s_k;
-    qa.rope = w.rope + (full ? (size_t)x.T * half * 2 : 0);
-    qa.q_scale = q_scale; qa.q_out = w.q; qa.gate_out = w.gate;
-    qa.kv = kv; qa.g = geo; qa.err = m->d_status;
-    {
-      Prof p(m, x.st, "qkv_post",
-             (double)x.M * (dm.rows_qkvg * 4.0 * S_qkvg + dm.qdim * 8.0 +
-                            dm.kvdim * 4.0), 0);
-      launch_qkv_post(qa, x.st);
-    }
-    AttnArgs aa{};
-    aa.q = w.q; aa.gate = w.gate; aa.B = x.B; aa.T = x.T; aa.dm = dm;
-    aa.window = full ? 0 : dm.window; aa.kv = kv; aa.g = geo;
-    aa.part_o = w.part_o; aa.part_ml = w.part_ml; aa.a_out = w.a;
-    aa.err = m->d_status;
     if (x.T == 1) {
+      DecAttnArgs da{};
+      da.qkvg = w.qkvg; da.S = S_qkvg; da.B = x.B; da.dm = dm;
+      da.s_q = bw.s_q; da.s_k = bw.s_k;
+      da.rope = w.rope + (full ? (size_t)half * 2 : 0);
+      da.q_scale = q_scale; da.window = full ? 0 : dm.window;
+      da.kv = kv; da.g = geo; da.part_o = w.part_o; da.part_ml = w.part_ml;
+      da.counters = w.counters; da.a_out = w.a; da.err = m->d_status;
       const double nk = full ? x.n_ctx0 + 1.0
                              : std::min(x.n_ctx0 + 1.0, (double)dm.window);
-      {
-        Prof p(m, x.st, "attn_decode",
-               x.B * (dm.Hkv * nk * dm.hd * 4.0 + dm.qdim * 4.0),
-               4.0 * x.B * dm.Hq * nk * dm.hd);
-        launch_attn_decode(aa, x.st);
-      }
-      Prof p(m, x.st, "attn_combine", x.B * dm.qdim * 10.0, 0);
-      launch_attn_combine(aa, x.st);
+      Prof p(m, x.st, "attn_decode",
+             x.B * (dm.Hkv * nk * dm.hd * 4.0 + S_qkvg * dm.rows_qkvg * 4.0),
+             4.0 * x.B * dm.Hq * nk * dm.hd);
+      launch_attn_decode_fused(da, x.st);
     } else {
+      QkvPostArgs qa{};
+      qa.qkvg = w.qkvg; qa.S = S_qkvg; qa.M = x.M; qa.T = x.T; qa.B = x.B;
+      qa.dm = dm; qa.s_q = bw.s_q; qa.s_k = bw.s_k;
+      qa.rope = w.rope + (full ? (size_t)x.T * half * 2 : 0);
+      qa.q_scale = q_scale; qa.q_out = w.q; qa.gate_out = w.gate;
+      qa.kv = kv; qa.g = geo; qa.err = m->d_status;
+      {
+        Prof p(m, x.st, "qkv_post",
+               (double)x.M * (dm.rows_qkvg * 4.0 * S_qkvg + dm.qdim * 8.0 +
+                              dm.kvdim * 4.0), 0);
+        launch_qkv_post(qa, x.st);
+      }
+      AttnArgs aa{};
+      aa.q = w.q; aa.gate = w.gate; aa.B = x.B; aa.T = x.T; aa.dm = dm;
+      aa.window = full ? 0 : dm.window; aa.kv = kv; aa.g = geo;
+      aa.a_out = w.a; aa.err = m->d_status;
       double vis = 0;
       for (int t = 0; t < x.T; ++t) {
         const double q = x.n_ctx0 + t + 1.0;
@@ -606,9 +621,9 @@ void enqueue_forward(const CallCtx& x) {
     if (gemv) {
       GemvArgs g{};
       g.W = bw.w_o; g.K = dm.qdim; g.n_items = dm.d; g.B = x.B; g.epi = EPI_F32;
-      g.S = S_o = gemv_split(dm.qdim, dm.d); g.out = w.h;
+      g.out = w.h;
       g.pro = PRO_BF16; g.xin = w.a; g.xin_stride = dm.qdim;
-      gemv_run(m, g, gemv_grid(g, m->num_sms), x.st, "gemv_o");
+      S_o = gemv_run(m, g, x.st, "gemv_o");
     } else {
       gemm_run(m, w.a, dm.qdim, bw.w_o, w.h, dm.d, x.M, dm.d, dm.qdim, nullptr,
                x.st, "gemm_o");
@@ -622,12 +637,12 @@ void enqueue_forward(const CallCtx& x) {
       g.pro = PRO_UPDATE; g.s_in = cur; g.h_in = w.h; g.h_S = S_o;
       g.alpha = bw.alpha_a; g.s_out = other; g.reinject = RJ_NONE; g.x_buf = w.x;
       std::swap(cur, other);
-      gemv_run(m, g, gemv_grid(g, m->num_sms), x.st, "gemv_gateup");
+      gemv_run(m, g, x.st, "gemv_gateup");
       GemvArgs g2{};
       g2.W = bw.w_down; g2.K = dm.F; g2.n_items = dm.d; g2.B = x.B;
-      g2.epi = EPI_F32; g2.S = prev_S = gemv_split(dm.F, dm.d); g2.out = w.h;
+      g2.epi = EPI_F32; g2.out = w.h;
       g2.pro = PRO_BF16; g2.xin = w.mact; g2.xin_stride = dm.F;
-      gemv_run(m, g2, gemv_grid(g2, m->num_sms), x.st, "gemv_down");
+      prev_S = gemv_run(m, g2, x.st, "gemv_down");
     } else {
       {
         Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
@@ -658,10 +673,12 @@ void enqueue_forward(const CallCtx& x) {
     g.out = x.logits; g.out_stride = dm.V; g.col_scale = m->s_z;
     g.amax_val = w.amax_val; g.amax_idx = w.amax_idx;
     const int grid = gemv_grid(g, m->num_sms);
-    gemv_run(m, g, grid, x.st, "gemv_lmhead");
+    gemv_run(m, g, x.st, "gemv_lmhead");
     if (x.argmax) {
       Prof p(m, x.st, "argmax", x.B * grid * 8.0, 0);
-      launch_argmax_partials(w.amax_val, w.amax_idx, x.B, grid, x.argmax, x.st);
+      launch_argmax_partials(w.amax_val, w.amax_idx, x.B, grid, x.argmax,
+                             x.c->d_nctx, x.T, x.st);
+      return;                  // the argmax kernel advanced the cache length
     }
   } else {
     {
@@ -687,11 +704,11 @@ void enqueue_forward(const CallCtx& x) {
         g.out_stride = dm.V; g.col_scale = m->s_z;
         g.amax_val = w.amax_val; g.amax_idx = w.amax_idx;
         const int grid = gemv_grid(g, m->num_sms);
-        gemv_run(m, g, grid, x.st, "gemv_lmhead");
+        gemv_run(m, g, x.st, "gemv_lmhead");
         if (x.argmax) {
           Prof p(m, x.st, "argmax", g.B * grid * 8.0, 0);
           launch_argmax_partials(w.amax_val, w.amax_idx, g.B, grid,
-                                 x.argmax + b0, x.st);
+                                 x.argmax + b0, nullptr, 0, x.st);
         }
       }
     }

@@ -4,10 +4,29 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <utility>
 
 namespace dory {
 
 typedef __nv_bfloat16 bf16;
+
+// Launch with programmatic stream serialization (PDL) unless disabled.
+bool pdl_enabled();
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                            size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Device error bits (or-ed into the status word the host reads back).
 enum : int {
@@ -62,7 +81,7 @@ struct GemvArgs {
   const bf16* W;       // [N_rows, K] row-major
   int K;               // contraction length (multiple of 256 * S)
   int n_items;         // output rows (EPI_SWIGLU: pairs n, n + pair_off)
-  int S;               // split-K factor (EPI_F32 only)
+  int S;               // split-K factor: set to gemv_splits(*this)
   int B;               // batch rows, <= 8
   int pair_off;        // EPI_SWIGLU
   // prologue
@@ -85,7 +104,11 @@ struct GemvArgs {
   const float* col_scale;   // EPI_LMHEAD: s_z [n_items]
   float* amax_val;     // EPI_LMHEAD: [B][gridDim]
   int* amax_idx;
+  int* err;            // device status word (bounded-wait timeouts)
 };
+// K segments per row the launcher will use (outputs are [S][B][n] partials
+// for EPI_F32; 1 for the other epilogues).
+int gemv_splits(const GemvArgs& a);
 int gemv_grid(const GemvArgs& a, int num_sms);
 void launch_gemv(const GemvArgs& a, int grid, cudaStream_t st);
 
@@ -94,8 +117,12 @@ void launch_gemv(const GemvArgs& a, int grid, cudaStream_t st);
 void launch_rope_table(float* table, const CacheGeo& g, int T, int hd,
                        double theta_swa, double theta_full, cudaStream_t st);
 // x0 = N(E[tok]) -> s (f32) and s_bf (bf16), rows M.
+// Block 0 also zeroes `counters` and, if rope != null (one-token calls),
+// writes the RoPE table [2][1][hd/2][2] for position n_ctx.
 void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
-                  bf16* s_bf, int* err, int vocab, cudaStream_t st);
+                  bf16* s_bf, int* err, int vocab, int* counters,
+                  int n_counters, float* rope, const int* n_ctx, int hd,
+                  double theta_swa, double theta_full, cudaStream_t st);
 // RoPE + per-head L2 norm + q/k scales + sigmoid gate + K/V cache write.
 struct QkvPostArgs {
   const float* qkvg; int S; int M; int T; int B;
@@ -117,7 +144,7 @@ void launch_update_rows(const float* s_in, const float* h, const float* alpha,
 void launch_swiglu(const float* gu, bf16* m, int M, int F, cudaStream_t st);
 // Final greedy argmax over [B][n] partials or full logits rows.
 void launch_argmax_partials(const float* val, const int* idx, int B, int n,
-                            int* out, cudaStream_t st);
+                            int* out, int* n_ctx, int T, cudaStream_t st);
 void launch_argmax_rows(const float* logits, int rows, int V, int* out,
                         cudaStream_t st);
 void launch_advance(int* n_ctx, int T, cudaStream_t st);
@@ -137,9 +164,26 @@ struct AttnArgs {
   bf16* a_out;         // [M][qdim] = gate * attention output
   int* err;
 };
-void launch_attn_decode(const AttnArgs& a, cudaStream_t st);
-void launch_attn_combine(const AttnArgs& a, cudaStream_t st);
 void launch_attn_prefill(const AttnArgs& a, cudaStream_t st);
+
+// Decode (one token per sequence): RoPE/QK-norm/KV write, split-KV attention,
+// split merge and gate in one kernel.
+struct DecAttnArgs {
+  const float* qkvg;   // QKVG partials [S][B][rows_qkvg]
+  int S, B;
+  Dims dm;
+  const float* s_q; const float* s_k;
+  const float* rope;   // [hd/2][2] cos/sin of this layer's type at n_ctx
+  float q_scale;
+  int window;
+  KVSlot kv; CacheGeo g;
+  float* part_o;       // [B][Hq][kMaxSplits][hd]
+  float* part_ml;      // [B][Hq][kMaxSplits][2]
+  int* counters;       // [B][Hkv] zero on entry; reset to zero on exit
+  bf16* a_out;         // [B][qdim]
+  int* err;
+};
+void launch_attn_decode_fused(const DecAttnArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- GEMM ----
 // C[M, N] (f32, row stride ldc) = A[M, K] (bf16, row stride lda) * W[N, K]^T

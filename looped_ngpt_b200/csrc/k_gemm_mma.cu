@@ -38,6 +38,8 @@ gemm_mma_kernel(const bf16* __restrict__ A, int lda,
   const int wm = warp >> 2, wn = warp & 3;
   const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
   const int KT = K / BK;
+  pdl_wait();
+  pdl_trigger();
 
   auto load_stage = [&](int s, int kt) {
     const int k0 = kt * BK;
@@ -147,8 +149,8 @@ void launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
     configured = true;
   }
   dim3 grid(N / BN, (M + BM - 1) / BM);
-  gemm_mma_kernel<<<grid, 256, smem, st>>>(A, lda, W, C, ldc, M, N, K,
-                                           col_scale);
+  launch_k(gemm_mma_kernel, grid, dim3(256), smem, st, A, lda, W, C, ldc, M,
+           N, K, col_scale);
 }
 
 }  // namespace dory

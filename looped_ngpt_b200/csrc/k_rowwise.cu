@@ -13,6 +13,8 @@ namespace {
 // would be off by ~1e-2 rad.
 __global__ void rope_table_kernel(float* table, const int* n_ctx, int T,
                                   int half, double th_swa, double th_full) {
+  pdl_wait();
+  pdl_trigger();
   const int total = 2 * T * half;
   const int p0 = *n_ctx;
   for (int id = blockIdx.x * blockDim.x + threadIdx.x; id < total;
@@ -29,11 +31,32 @@ __global__ void rope_table_kernel(float* table, const int* n_ctx, int T,
   }
 }
 
-// x0 = N(E[tok]); one block per row.
+// x0 = N(E[tok]); one block per row.  Block 0 also zeroes the attention
+// ticket counters and, for one-token calls (rope != null), writes the RoPE
+// cos/sin of position n_ctx for both attention types.
 __global__ void embed_kernel(const int* tokens, const bf16* E, int d,
-                             int vocab, float* s, bf16* s_bf, int* err) {
+                             int vocab, float* s, bf16* s_bf, int* err,
+                             int* counters, int n_counters, float* rope,
+                             const int* n_ctx, int half, double th_swa,
+                             double th_full) {
   __shared__ float red[32];
   const int row = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  if (row == 0) {
+    for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
+    if (rope) {
+      const int p = *n_ctx;
+      for (int id = threadIdx.x; id < 2 * half; id += blockDim.x) {
+        const int type = id / half, i = id - type * half;
+        const double inv = pow(type ? th_full : th_swa, -2.0 * i / (2.0 * half));
+        double sn, c;
+        sincos((double)p * inv, &sn, &c);
+        rope[2 * id] = (float)c;
+        rope[2 * id + 1] = (float)sn;
+      }
+    }
+  }
   int tok = tokens[row];
   if (tok < 0 || tok >= vocab) {
     if (threadIdx.x == 0) atomicOr(err, ERRBIT_BOUNDS);
@@ -59,6 +82,8 @@ constexpr int kPairs = kMaxHeadDim / 64;   // rotate-half pairs per lane
 // heads, [Hq+Hkv, Hq+2Hkv) v heads, [Hq+2Hkv, 2Hq+2Hkv) gate heads.
 __global__ void qkv_post_kernel(const QkvPostArgs a) {
   const Dims& dm = a.dm;
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int n_items = 2 * dm.Hq + 2 * dm.Hkv;
@@ -147,6 +172,8 @@ __global__ void update_rows_kernel(const float* s_in, const float* h,
                                    int d) {
   extern __shared__ float tmp[];
   __shared__ float red[32];
+  pdl_wait();
+  pdl_trigger();
   const size_t o = (size_t)blockIdx.x * d;
   ngpt_update_row(s_in + o, h + o, 1, 0, alpha, d, reinject,
                   reinject == RJ_NONE ? nullptr : x_buf + o, s_out + o,
@@ -154,6 +181,8 @@ __global__ void update_rows_kernel(const float* s_in, const float* h,
 }
 
 __global__ void swiglu_kernel(const float* gu, bf16* m, int M, int F) {
+  pdl_wait();
+  pdl_trigger();
   const size_t total = (size_t)M * F;
   for (size_t id = blockIdx.x * (size_t)blockDim.x + threadIdx.x; id < total;
        id += (size_t)gridDim.x * blockDim.x) {
@@ -187,9 +216,14 @@ __device__ void block_argmax(float v, int i, int* out) {
   }
 }
 
+// Also advances the cache length by T (block 0) when n_ctx != null: the
+// attention of every layer of this call has finished reading it.
 __global__ void argmax_partials_kernel(const float* val, const int* idx,
-                                       int n, int* out) {
+                                       int n, int* out, int* n_ctx, int T) {
   const int b = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  if (n_ctx && b == 0 && threadIdx.x == 0) *n_ctx += T;
   float v = -INFINITY;
   int i = 0x7fffffff;
   for (int k = threadIdx.x; k < n; k += blockDim.x)
@@ -198,6 +232,8 @@ __global__ void argmax_partials_kernel(const float* val, const int* idx,
 }
 
 __global__ void argmax_rows_kernel(const float* z, int V, int* out) {
+  pdl_wait();
+  pdl_trigger();
   const size_t r = blockIdx.x;
   float v = -INFINITY;
   int i = 0x7fffffff;
@@ -205,7 +241,11 @@ __global__ void argmax_rows_kernel(const float* z, int V, int* out) {
   block_argmax(v, i, out + r);
 }
 
-__global__ void advance_kernel(int* n_ctx, int T) { *n_ctx += T; }
+__global__ void advance_kernel(int* n_ctx, int T) {
+  pdl_wait();
+  pdl_trigger();
+  *n_ctx += T;
+}
 
 __global__ void cache_init_kernel(int* n_ctx, int* bt, int total) {
   const int id = blockIdx.x * blockDim.x + threadIdx.x;
@@ -219,47 +259,52 @@ void launch_rope_table(float* table, const CacheGeo& g, int T, int hd,
                        double theta_swa, double theta_full, cudaStream_t st) {
   const int total = 2 * T * (hd / 2);
   const int blocks = (total + 255) / 256;
-  rope_table_kernel<<<blocks < 1184 ? blocks : 1184, 256, 0, st>>>(
-      table, g.n_ctx, T, hd / 2, theta_swa, theta_full);
+  launch_k(rope_table_kernel, dim3(blocks < 1184 ? blocks : 1184), dim3(256), 0,
+           st, table, (const int*)g.n_ctx, T, hd / 2, theta_swa, theta_full);
 }
 
 void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
-                  bf16* s_bf, int* err, int vocab, cudaStream_t st) {
-  embed_kernel<<<M, 256, 0, st>>>(tokens, E, d, vocab, s, s_bf, err);
+                  bf16* s_bf, int* err, int vocab, int* counters,
+                  int n_counters, float* rope, const int* n_ctx, int hd,
+                  double theta_swa, double theta_full, cudaStream_t st) {
+  launch_k(embed_kernel, dim3(M), dim3(256), 0, st, tokens, E, d, vocab, s,
+           s_bf, err, counters, n_counters, rope, n_ctx, hd / 2, theta_swa,
+           theta_full);
 }
 
 void launch_qkv_post(const QkvPostArgs& a, cudaStream_t st) {
   const int items = 2 * a.dm.Hq + 2 * a.dm.Hkv;
   dim3 grid((items + 7) / 8, a.M);
-  qkv_post_kernel<<<grid, 256, 0, st>>>(a);
+  launch_k(qkv_post_kernel, grid, dim3(256), 0, st, a);
 }
 
 void launch_update_rows(const float* s_in, const float* h, const float* alpha,
                         float* s_out, bf16* s_bf, float* x_buf, int reinject,
                         int M, int d, cudaStream_t st) {
-  update_rows_kernel<<<M, 256, d * sizeof(float), st>>>(
-      s_in, h, alpha, s_out, s_bf, x_buf, reinject, d);
+  launch_k(update_rows_kernel, dim3(M), dim3(256), d * sizeof(float), st, s_in,
+           h, alpha, s_out, s_bf, x_buf, reinject, d);
 }
 
 void launch_swiglu(const float* gu, bf16* m, int M, int F, cudaStream_t st) {
   const size_t total = (size_t)M * F;
   size_t blocks = (total + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  swiglu_kernel<<<(int)blocks, 256, 0, st>>>(gu, m, M, F);
+  launch_k(swiglu_kernel, dim3((int)blocks), dim3(256), 0, st, gu, m, M, F);
 }
 
 void launch_argmax_partials(const float* val, const int* idx, int B, int n,
-                            int* out, cudaStream_t st) {
-  argmax_partials_kernel<<<B, 256, 0, st>>>(val, idx, n, out);
+                            int* out, int* n_ctx, int T, cudaStream_t st) {
+  launch_k(argmax_partials_kernel, dim3(B), dim3(256), 0, st, val, idx, n, out,
+           n_ctx, T);
 }
 
 void launch_argmax_rows(const float* logits, int rows, int V, int* out,
                         cudaStream_t st) {
-  argmax_rows_kernel<<<rows, 256, 0, st>>>(logits, V, out);
+  launch_k(argmax_rows_kernel, dim3(rows), dim3(256), 0, st, logits, V, out);
 }
 
 void launch_advance(int* n_ctx, int T, cudaStream_t st) {
-  advance_kernel<<<1, 1, 0, st>>>(n_ctx, T);
+  launch_k(advance_kernel, dim3(1), dim3(1), 0, st, n_ctx, T);
 }
 
 void launch_cache_init(int* n_ctx, int* block_table, int B, int pages_per_seq,

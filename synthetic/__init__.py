@@ -20,10 +20,10 @@ Each tensor is drawn from its own PCG64 stream ``default_rng([seed, idx])``
 (idx = the tensor's position in ``tensor_names``), so any subset of tensors
 can be generated alone and the draw does not depend on the order of calls.
 """
-from .shapes import ModelShape, TINY, DORY, tiny_with_blocks
+from .shapes import ModelShape, TINY, DORY, tiny_with_blocks, dory_with_blocks
 from .gen import (tensor_names, tensor_spec, make_tensor, make_weights,
                   make_prompt, bf16_bits_to_f32, f32_to_bf16_bits)
 
-__all__ = ["ModelShape", "TINY", "DORY", "tiny_with_blocks", "tensor_names",
+__all__ = ["ModelShape", "TINY", "DORY", "tiny_with_blocks", "dory_with_blocks", "tensor_names",
            "tensor_spec", "make_tensor", "make_weights", "make_prompt",
            "bf16_bits_to_f32", "f32_to_bf16_bits"]

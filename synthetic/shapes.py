@@ -84,3 +84,12 @@ def tiny_with_blocks(n_in, n_rec, n_out, **kw):
                 n_rec=n_rec, n_out=n_out, swa_window=8)
     base.update(kw)
     return ModelShape(**base)
+
+
+def dory_with_blocks(n_in, n_rec, n_out):
+    """Dory widths (every kernel shape unchanged) with fewer blocks: a small
+    case for profilers that must keep the device footprint to a few GB."""
+    return ModelShape(name=f"dory-{n_in}-{n_rec}-{n_out}", d=2560,
+                      n_q_heads=16, n_kv_heads=4, head_dim=160, ffn=10240,
+                      vocab=131072, n_in=n_in, n_rec=n_rec, n_out=n_out,
+                      swa_window=1024)
