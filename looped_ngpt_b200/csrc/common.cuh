@@ -74,63 +74,120 @@ __device__ __forceinline__ float sigmoidf_(float x) {
   return 1.f / (1.f + __expf(-x));
 }
 
+// Sum of NV values over the whole block; every thread gets the results.
+// `red` needs NV * (blockDim.x / 32) floats.  Contains __syncthreads().
+template <int NV>
+__device__ __forceinline__ void block_sum_n(float (&v)[NV], float* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) v[i] = warp_sum(v[i]);
+  __syncthreads();
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) red[w * NV + i] = v[i];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    float t = 0.f;
+    for (int k = 0; k < nw; ++k) t += red[k * NV + i];
+    v[i] = t;
+  }
+}
+
 // nGPT residual update of one row held by the whole block:
-//   s_new = N(s + alpha (N(h) - s)),  h = sum of h_S partials.
-// Optional loop re-injection: RJ_FIRST stores x := s_new and returns
-// N(s_new + x); RJ_NEXT returns N(s_new + x) with the stored x.
-// dst receives the row (f32) when non-null; dst_bf (bf16) likewise.
-// `red` needs blockDim/32 floats.  All threads must call it.
+//   s_new = N(s + alpha (N(h) - s)) = N((1 - alpha) s + alpha h / |h|),
+//   h = sum of hS partials (stride h_stride).
+// Both norms come from one block reduction: with a = 1 - alpha,
+//   |t|^2 = sum (a s)^2 + 2 sum a alpha s h / |h| + sum (alpha h)^2 / |h|^2.
+// Loop re-injection: RJ_FIRST stores x := s_new (x_row, if given) and
+// returns N(s_new + x) = N(2 s_new) = s_new; RJ_NEXT returns
+// N(s_new + x) using |s_new + x|^2 = 1 + 2 s_new.x + |x|^2, whose terms are
+// reduced in the same pass.  Writes the result to dst (f32) and/or dst_bf
+// (bf16) when non-null.  tmp holds d floats; red needs 7 * blockDim/32
+// floats.  All threads must call it; it ends with __syncthreads().
 __device__ inline void ngpt_update_row(const float* s, const float* h, int hS,
                                        size_t h_stride, const float* alpha,
                                        int d, int reinject, float* x_row,
                                        float* dst, bf16* dst_bf, float* tmp,
                                        float* red) {
-  float ss = 0.f;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    float v = 0.f;
-    for (int k = 0; k < hS; ++k) v += h[k * h_stride + i];
-    tmp[i] = v;
-    ss += v * v;
-  }
-  const float inv_h = 1.f / fmaxf(sqrtf(block_sum(ss, red)), 1e-12f);
-  float tt = 0.f;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    float sv = s[i];
-    float t = sv + alpha[i] * (tmp[i] * inv_h - sv);
-    tmp[i] = t;
-    tt += t * t;
-  }
-  const float inv_t = 1.f / fmaxf(sqrtf(block_sum(tt, red)), 1e-12f);
-  if (reinject == RJ_NONE) {
-    for (int i = threadIdx.x; i < d; i += blockDim.x) {
-      float v = tmp[i] * inv_t;
-      tmp[i] = v;
-      if (dst) dst[i] = v;
-      if (dst_bf) dst_bf[i] = __float2bfloat16_rn(v);
+  constexpr int U = 8;               // elements per thread in flight
+  const int nt = blockDim.x;
+  float r[7] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const bool next = reinject == RJ_NEXT;
+  for (int i0 = threadIdx.x; i0 < d; i0 += U * nt) {
+    float hv[U], sv[U], av[U], xv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * nt;
+      hv[u] = sv[u] = av[u] = xv[u] = 0.f;
+      if (i < d) {
+        sv[u] = s[i];
+        av[u] = alpha[i];
+        if (next) xv[u] = x_row[i];
+      }
     }
-    __syncthreads();
-    return;
-  }
-  float uu = 0.f;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    float v = tmp[i] * inv_t;
-    float xv;
-    if (reinject == RJ_FIRST) {
-      xv = v;
-      if (x_row) x_row[i] = v;
-    } else {
-      xv = x_row[i];
+    for (int k = 0; k < hS; ++k) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = i0 + u * nt;
+        if (i < d) hv[u] += h[k * h_stride + i];
+      }
     }
-    float u = v + xv;
-    tmp[i] = u;
-    uu += u * u;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * nt;
+      if (i < d) {
+        tmp[i] = hv[u];
+        const float as = (1.f - av[u]) * sv[u], ah = av[u] * hv[u];
+        r[0] += hv[u] * hv[u];
+        r[1] += as * as;
+        r[2] += as * ah;
+        r[3] += ah * ah;
+        r[4] += as * xv[u];
+        r[5] += ah * xv[u];
+        r[6] += xv[u] * xv[u];
+      }
+    }
   }
-  const float inv_u = 1.f / fmaxf(sqrtf(block_sum(uu, red)), 1e-12f);
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    float v = tmp[i] * inv_u;
-    tmp[i] = v;
-    if (dst) dst[i] = v;
-    if (dst_bf) dst_bf[i] = __float2bfloat16_rn(v);
+  if (next) block_sum_n<7>(r, red);
+  else {
+    float q[4] = {r[0], r[1], r[2], r[3]};
+    block_sum_n<4>(q, red);
+    r[0] = q[0]; r[1] = q[1]; r[2] = q[2]; r[3] = q[3];
+  }
+  const float inv_h = 1.f / fmaxf(sqrtf(r[0]), 1e-12f);
+  const float tt = r[1] + 2.f * r[2] * inv_h + r[3] * inv_h * inv_h;
+  const float inv_t = 1.f / fmaxf(sqrtf(fmaxf(tt, 0.f)), 1e-12f);
+  float inv_u = 1.f;
+  if (next) {
+    const float dot = (r[4] + r[5] * inv_h) * inv_t;
+    inv_u = 1.f / fmaxf(sqrtf(fmaxf(1.f + 2.f * dot + r[6], 0.f)), 1e-12f);
+  }
+  for (int i0 = threadIdx.x; i0 < d; i0 += U * nt) {
+    float sv[U], av[U], xv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * nt;
+      sv[u] = av[u] = xv[u] = 0.f;
+      if (i < d) {
+        sv[u] = s[i];
+        av[u] = alpha[i];
+        if (next) xv[u] = x_row[i];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * nt;
+      if (i < d) {
+        float v = ((1.f - av[u]) * sv[u] + av[u] * tmp[i] * inv_h) * inv_t;
+        if (reinject == RJ_FIRST && x_row) x_row[i] = v;
+        if (next) v = (v + xv[u]) * inv_u;
+        if (dst) dst[i] = v;
+        if (dst_bf) dst_bf[i] = __float2bfloat16_rn(v);
+      }
+    }
   }
   __syncthreads();
 }

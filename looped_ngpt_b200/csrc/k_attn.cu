@@ -179,6 +179,13 @@ __global__ void __launch_bounds__(2 * HD) attn_decode_fused_kernel(const DecAttn
   constexpr int NQ = HD / 32;          // score parts per key
   constexpr int RP = HD + KPAD;
   constexpr int HP = HD / 2;           // dim pairs
+  // P.V partials, later the merge's weights and gates
+  constexpr int PVS = (4 * G * HD > G * (2 * kMaxSplits + HD))
+                          ? 4 * G * HD : G * (2 * kMaxSplits + HD);
+  // splits staged per merge round trip: as many as fit in the K/V tiles
+  constexpr int CHF = (2 * TK * (HD + KPAD) * 2) / (G * HD * 4);
+  constexpr int CH = CHF < 16 ? CHF : 16;
+  static_assert(CH >= 1, "merge staging buffer must fit in the K/V tiles");
   extern __shared__ float sm[];
   const Dims& dm = a.dm;
   const int b = blockIdx.z, kvh = blockIdx.y, split = blockIdx.x;
@@ -190,7 +197,7 @@ __global__ void __launch_bounds__(2 * HD) attn_decode_fused_kernel(const DecAttn
   float* sc_s = vn_s + HD;                           // [NQ][G][TK] scores / [G][TK] probs
   float* st = sc_s + NQ * G * TK;                    // m, l, corr: [3][G] (+pad)
   float* pv_s = st + 32;                             // [4][G][HD] P.V partials
-  bf16* K_s = reinterpret_cast<bf16*>(pv_s + 4 * G * HD);   // [TK][RP]
+  bf16* K_s = reinterpret_cast<bf16*>(pv_s + PVS);   // [TK][RP]
   bf16* V_s = K_s + TK * RP;
   __shared__ int s_last;
 
@@ -370,13 +377,22 @@ __global__ void __launch_bounds__(2 * HD) attn_decode_fused_kernel(const DecAttn
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  float* mlw = reinterpret_cast<float*>(K_s);        // [G][n][2] (n <= 64)
+  // merge: stage (m, l) of every split and the gate sums in one round trip
+  float* mlw = pv_s;                                 // [G][n][2] (n <= 64)
+  float* gate_s = pv_s + G * kMaxSplits * 2;         // [G][HD]
   for (int id = tid; id < G * sp.n; id += NT) {
     const int g = id / sp.n, s2 = id - g * sp.n;
     const float2 v = __ldcg(reinterpret_cast<const float2*>(
         a.part_ml + ((hb + g) * kMaxSplits + s2) * 2));
     mlw[2 * id] = v.x;
     mlw[2 * id + 1] = v.y;
+  }
+  for (int idx = tid; idx < G * HD; idx += NT) {
+    const int g = idx / HD, c = idx - g * HD;
+    float gs = 0.f;
+    for (int s3 = 0; s3 < a.S; ++s3)
+      gs += src[s3 * pstride + dm.qdim + 2 * dm.kvdim + (kvh * G + g) * HD + c];
+    gate_s[idx] = sigmoidf_(gs);
   }
   __syncthreads();
   if (w < G) {
@@ -393,28 +409,46 @@ __global__ void __launch_bounds__(2 * HD) attn_decode_fused_kernel(const DecAttn
     L = warp_sum(L);
     if (lane == 0) st[w] = 1.f / L;
   }
-  __syncthreads();
-  for (int idx = tid; idx < G * HD; idx += NT) {
-    const int g = idx / HD, c = idx - g * HD;
-    const float* po = a.part_o + (hb + g) * kMaxSplits * HD + c;
-    const float* f = mlw + 2 * g * sp.n;
-    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-    int s2 = 0;
-    for (; s2 + 3 < sp.n; s2 += 4) {
-      const float v0 = __ldcg(po + (s2 + 0) * HD), v1 = __ldcg(po + (s2 + 1) * HD);
-      const float v2 = __ldcg(po + (s2 + 2) * HD), v3 = __ldcg(po + (s2 + 3) * HD);
-      o0 = fmaf(f[2 * (s2 + 0)], v0, o0);
-      o1 = fmaf(f[2 * (s2 + 1)], v1, o1);
-      o2 = fmaf(f[2 * (s2 + 2)], v2, o2);
-      o3 = fmaf(f[2 * (s2 + 3)], v3, o3);
+  // partial outputs, CH splits per round trip, staged with cp.async
+  constexpr int NO = (G * HD + NT - 1) / NT;         // outputs per thread
+  float* buf = reinterpret_cast<float*>(K_s);        // [G][CH][HD]
+  float o[NO];
+#pragma unroll
+  for (int k = 0; k < NO; ++k) o[k] = 0.f;
+  for (int s0 = 0; s0 < sp.n; s0 += CH) {
+    const int cnt = min(CH, sp.n - s0);
+    __syncthreads();                                 // buf free, weights ready
+    constexpr int V4 = HD / 4;                       // 16-byte pieces per row
+    for (int id = tid; id < G * cnt * V4; id += NT) {
+      const int row = id / V4, c = id - row * V4;
+      const int g = row / cnt, s2 = row - g * cnt;
+      cp_async16(buf + (g * CH + s2) * HD + c * 4,
+                 a.part_o + ((hb + g) * kMaxSplits + s0 + s2) * HD + c * 4);
     }
-    for (; s2 < sp.n; ++s2) o0 = fmaf(f[2 * s2], __ldcg(po + s2 * HD), o0);
-    const int h = kvh * G + g;
-    float gsum = 0.f;
-    for (int s3 = 0; s3 < a.S; ++s3)
-      gsum += src[s3 * pstride + dm.qdim + 2 * dm.kvdim + h * HD + c];
-    a.a_out[(size_t)b * dm.qdim + h * HD + c] =
-        __float2bfloat16_rn(sigmoidf_(gsum) * ((o0 + o1) + (o2 + o3)) * st[g]);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < NO; ++k) {
+      const int idx = tid + k * NT;
+      if (idx < G * HD) {
+        const int g = idx / HD, c = idx - g * HD;
+        const float* f = mlw + 2 * (g * sp.n + s0);
+        float t = o[k];
+        for (int s2 = 0; s2 < cnt; ++s2)
+          t = fmaf(f[2 * s2], buf[(g * CH + s2) * HD + c], t);
+        o[k] = t;
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < NO; ++k) {
+    const int idx = tid + k * NT;
+    if (idx < G * HD) {
+      const int g = idx / HD, c = idx - g * HD;
+      a.a_out[(size_t)b * dm.qdim + (kvh * G + g) * HD + c] =
+          __float2bfloat16_rn(gate_s[idx] * o[k] * st[g]);
+    }
   }
   if (tid == 0) a.counters[b * dm.Hkv + kvh] = 0;
 }
@@ -556,7 +590,9 @@ void launch_prefill_t(const AttnArgs& a, cudaStream_t st) {
 template <int HD, int G>
 void launch_dec_t(const DecAttnArgs& a, cudaStream_t st) {
   constexpr int NQ = HD / 32;
-  const size_t smem = (G * HD + 2 * HD + NQ * G * TK + 32 + 4 * G * HD) *
+  constexpr int PVS = (4 * G * HD > G * (2 * kMaxSplits + HD))
+                          ? 4 * G * HD : G * (2 * kMaxSplits + HD);
+  const size_t smem = (G * HD + 2 * HD + NQ * G * TK + 32 + PVS) *
                           sizeof(float) +
                       2 * TK * (HD + KPAD) * sizeof(bf16);
   static bool configured = false;

@@ -132,6 +132,31 @@ __device__ __forceinline__ void row_slice_dot(const bf16* wrow, const bf16* xk,
   for (int b = 0; b < NB; ++b) acc[b] = warp_sum(acc[b]);
 }
 
+// One staged row segment times the register-resident x slice (batch 1):
+// lane covers elements c * 256 + lane * 8 + [0, 8) for c < nc.  Two
+// accumulators break the FMA dependency chain.
+template <int MAXC>
+__device__ __forceinline__ float row_dot_reg(const bf16* wrow, const float* xr,
+                                             int nc, int lane) {
+  float a0 = 0.f, a1 = 0.f;
+  const bf16* wp = wrow + lane * 8;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    if (c < nc) {
+      const uint4 wv = *reinterpret_cast<const uint4*>(wp + c * 256);
+      a0 = fmaf(bf_lo(wv.x), xr[c * 8 + 0], a0);
+      a1 = fmaf(bf_hi(wv.x), xr[c * 8 + 1], a1);
+      a0 = fmaf(bf_lo(wv.y), xr[c * 8 + 2], a0);
+      a1 = fmaf(bf_hi(wv.y), xr[c * 8 + 3], a1);
+      a0 = fmaf(bf_lo(wv.z), xr[c * 8 + 4], a0);
+      a1 = fmaf(bf_hi(wv.z), xr[c * 8 + 5], a1);
+      a0 = fmaf(bf_lo(wv.w), xr[c * 8 + 6], a0);
+      a1 = fmaf(bf_hi(wv.w), xr[c * 8 + 7], a1);
+    }
+  }
+  return warp_sum(a0 + a1);
+}
+
 // Activation vector(s) for the GEMV -> shared memory as bf16: a copy of the
 // caller's bf16 rows (PRO_BF16) or the fused nGPT update (PRO_UPDATE).
 template <int NB>
@@ -185,15 +210,16 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
   uint64_t* full = reinterpret_cast<uint64_t*>(
       tmp + (a.pro == PRO_UPDATE ? K : 0));
   uint64_t* empty = full + NS;
-  __shared__ float red[kWarps + 1];
+  __shared__ float red[7 * (kWarps + 1)];
   __shared__ float bestv[kWarps][NB];
   __shared__ int besti[kWarps][NB];
   __shared__ int s_fail, s_issued;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long total = (long)a.n_items * S;
-  const long j0 = total * blockIdx.x / gridDim.x;
-  const long j1 = total * (blockIdx.x + 1) / gridDim.x;
+  // row-aligned item range: a stage of 8 items starts at a multiple of S,
+  // so warp w always works on K segment w % S
+  const long j0 = (long)a.n_items * blockIdx.x / gridDim.x * S;
+  const long j1 = (long)a.n_items * (blockIdx.x + 1) / gridDim.x * S;
   const int n_stages = (int)((j1 - j0 + kWarps - 1) / kWarps);
   const bool producer = tid == kWarps * 32;
 
@@ -248,6 +274,24 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
     }
   } else {
     // ---- consumers: warp w owns item w of every stage ------------------
+    // NB == 1: this warp's slice of x (segment w % S, lane's 8-element
+    // chunks) stays in registers as f32 for the whole kernel.
+    constexpr int kMaxC = kSeg / 256;
+    const int nc = seg >> 8;
+    float xr[NB == 1 ? kMaxC * 8 : 1];
+    if (NB == 1) {
+      const bf16* xk = xs + (warp % S) * seg + lane * 8;
+#pragma unroll
+      for (int c = 0; c < kMaxC; ++c) {
+        if (c < nc) {
+          const uint4 xv = *reinterpret_cast<const uint4*>(xk + c * 256);
+          xr[c * 8 + 0] = bf_lo(xv.x); xr[c * 8 + 1] = bf_hi(xv.x);
+          xr[c * 8 + 2] = bf_lo(xv.y); xr[c * 8 + 3] = bf_hi(xv.y);
+          xr[c * 8 + 4] = bf_lo(xv.z); xr[c * 8 + 5] = bf_hi(xv.z);
+          xr[c * 8 + 6] = bf_lo(xv.w); xr[c * 8 + 7] = bf_hi(xv.w);
+        }
+      }
+    }
     for (int s = 0; s < n_stages; ++s) {
       const int slot = s % NS;
       if (!mbar_wait(full + slot, (uint32_t)((s / NS) & 1))) {
@@ -262,9 +306,14 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
         const bf16* wrow = reinterpret_cast<const bf16*>(
             ring + slot * stage_bytes + warp * item_bytes);
         float acc[NB], acc2[NB];
-        row_slice_dot<NB>(wrow, xs + sidx * seg, K, seg, lane, acc);
-        if (R == 2)
-          row_slice_dot<NB>(wrow + kWarps * seg, xs, K, seg, lane, acc2);
+        if (NB == 1) {
+          acc[0] = row_dot_reg<kMaxC>(wrow, xr, nc, lane);
+          if (R == 2) acc2[0] = row_dot_reg<kMaxC>(wrow + kWarps * seg, xr, nc, lane);
+        } else {
+          row_slice_dot<NB>(wrow, xs + sidx * seg, K, seg, lane, acc);
+          if (R == 2)
+            row_slice_dot<NB>(wrow + kWarps * seg, xs, K, seg, lane, acc2);
+        }
         if (lane == 0) {
 #pragma unroll
           for (int b = 0; b < NB; ++b) {
@@ -391,8 +440,7 @@ void launch_nb(const GemvArgs& a, int grid, cudaStream_t st) {
 int gemv_splits(const GemvArgs& a) { return make_plan(a, nb_of(a.B)).S; }
 
 int gemv_grid(const GemvArgs& a, int num_sms) {
-  const long items = (long)a.n_items * gemv_splits(a);
-  return items < num_sms ? (int)items : num_sms;
+  return a.n_items < num_sms ? a.n_items : num_sms;
 }
 
 void launch_gemv(const GemvArgs& a, int grid, cudaStream_t st) {

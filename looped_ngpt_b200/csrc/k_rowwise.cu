@@ -171,7 +171,7 @@ __global__ void update_rows_kernel(const float* s_in, const float* h,
                                    bf16* s_bf, float* x_buf, int reinject,
                                    int d) {
   extern __shared__ float tmp[];
-  __shared__ float red[32];
+  __shared__ float red[7 * 32];
   pdl_wait();
   pdl_trigger();
   const size_t o = (size_t)blockIdx.x * d;
