@@ -112,7 +112,7 @@ __device__ inline void ngpt_update_row(const float* s, const float* h, int hS,
                                        int d, int reinject, float* x_row,
                                        float* dst, bf16* dst_bf, float* tmp,
                                        float* red) {
-  constexpr int U = 8;               // elements per thread in flight
+  constexpr int U = 10;              // elements per thread in flight
   const int nt = blockDim.x;
   float r[7] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   const bool next = reinject == RJ_NEXT;
@@ -128,6 +128,7 @@ __device__ inline void ngpt_update_row(const float* s, const float* h, int hS,
         if (next) xv[u] = x_row[i];
       }
     }
+#pragma unroll 4
     for (int k = 0; k < hS; ++k) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
