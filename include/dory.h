@@ -184,6 +184,15 @@ int dory_decode_step_static(dory_model* m, dory_cache* c,
                             int kv_mode, float* d_logits, int32_t* d_argmax,
                             void* stream);
 
+/* Test and benchmark access to the projection GEMM used by prefill:
+ * d_C f32 [M, N] (row-major) = d_A bf16 [M, K] (row stride lda >= K, a
+ * multiple of 8) times d_W bf16 [N, K]^T, on the tcgen05 tensor cores.
+ * K must be a multiple of 64; device pointers 16-byte aligned.  Enqueued on
+ * `stream`; errors: DORY_ERR_ARG, DORY_ERR_CUDA (timeouts of its bounded
+ * waits are reported by dory_sync_status of any model). */
+int dory_debug_gemm_bf16(const void* d_A, int lda, const void* d_W,
+                         float* d_C, int M, int N, int K, void* stream);
+
 /* Per-kernel timing (tracing aid).  While enabled, every call launches its
  * kernels eagerly (no graph replay), each bracketed by CUDA events on the
  * call's stream, and records the kernel's algorithmic bytes (weights, KV

@@ -55,6 +55,8 @@ SIGNATURES = {
                                  c_int64, _P]),
     "dory_decode_step_static": (c_int, [_P, _P, _P, c_int, c_int, c_int, _P,
                                         _P, _P]),
+    "dory_debug_gemm_bf16": (c_int, [_P, c_int, _P, _P, c_int, c_int, c_int,
+                                     _P]),
     "dory_copy_state": (c_int, [_P, _P, c_int, c_int, c_int, _P, _P]),
     "dory_sync_status": (c_int, [_P, _P]),
     "dory_profile_enable": (c_int, [_P, c_int]),

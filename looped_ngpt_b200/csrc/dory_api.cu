@@ -140,7 +140,7 @@ CacheLayout cache_layout(const dory_model* m, int B, int max_ctx,
 
 
 struct WS {
-  float *s0, *s1, *sfin, *x, *qkvg, *q, *gate, *h, *gu, *part_o, *part_ml,
+  float *s0, *s1, *sfin, *x, *qkvg, *q, *gate, *h, *part_o, *part_ml,
       *rope, *amax_val;
   bf16 *s_bf, *a, *mact;
   int* amax_idx;
@@ -171,7 +171,6 @@ WS ws_layout(const dory_model* m, int B, int T, char* base) {
   w.gate = (float*)take(M * dm.qdim * 4);
   w.a = (bf16*)take(M * dm.qdim * 2);
   w.h = (float*)take(kMaxS * M * dm.d * 4);
-  w.gu = (float*)take(M > 8 || T > 1 ? M * 2 * (size_t)dm.F * 4 : 0);
   w.mact = (bf16*)take(M * dm.F * 2);
   w.part_o = (float*)take((size_t)B * dm.Hq * kMaxSplits * dm.hd * 4);
   w.part_ml = (float*)take((size_t)B * dm.Hq * kMaxSplits * 2 * 4);
@@ -321,6 +320,7 @@ int dory_init_weights(const dory_config* cfg, const dory_tensor* tensors,
     delete m;
     return DORY_ERR_CUDA;
   }
+  set_tc_error_word(m->d_status);
   const char* ng = getenv("DORY_NO_GRAPH");
   m->use_graphs = !(ng && ng[0] == '1');
   *out = m;
@@ -650,11 +650,13 @@ void enqueue_forward(const CallCtx& x) {
                            x.M, dm.d, x.st);
       }
       std::swap(cur, other);
-      gemm_run(m, w.s_bf, dm.d, bw.w_gu, w.gu, 2 * dm.F, x.M, 2 * dm.F, dm.d,
-               nullptr, x.st, "gemm_gateup");
       {
-        Prof p(m, x.st, "swiglu", (double)x.M * dm.F * 10, 0);
-        launch_swiglu(w.gu, w.mact, x.M, dm.F, x.st);
+        Prof p(m, x.st, "gemm_gateup",
+               (double)x.M * dm.d * 2 + 2.0 * dm.F * dm.d * 2 +
+                   (double)x.M * dm.F * 2,
+               2.0 * x.M * 2.0 * dm.F * dm.d);
+        launch_gemm_swiglu(w.s_bf, dm.d, bw.w_gu, w.mact, dm.F, x.M, dm.F, dm.d,
+                           x.st);
       }
       gemm_run(m, w.mact, dm.F, bw.w_down, w.h, dm.d, x.M, dm.d, dm.F, nullptr,
                x.st, "gemm_down");
@@ -882,4 +884,16 @@ extern "C" int dory_decode_step_static(dory_model* m, dory_cache* c,
   // decode = false: the kernels are launched directly, never via a graph.
   return run_call(m, c, d_tokens, B, 1, n_loops, kv_mode, 0, d_logits,
                   d_argmax, ws, (int64_t)DORY_STATIC_WS_BYTES, stream, false);
+}
+
+extern "C" int dory_debug_gemm_bf16(const void* d_A, int lda, const void* d_W,
+                                    float* d_C, int M, int N, int K,
+                                    void* stream) {
+  if (!d_A || !d_W || !d_C || M < 1 || N < 1 || K < 64 || K % 64 ||
+      lda < K || lda % 8)
+    return DORY_ERR_ARG;
+  cudaGetLastError();
+  launch_gemm_bf16((const bf16*)d_A, lda, (const bf16*)d_W, d_C, N, M, N, K,
+                   nullptr, (cudaStream_t)stream);
+  return cudaGetLastError() == cudaSuccess ? DORY_OK : DORY_ERR_CUDA;
 }

@@ -140,8 +140,6 @@ void launch_qkv_post(const QkvPostArgs& a, cudaStream_t st);
 void launch_update_rows(const float* s_in, const float* h, const float* alpha,
                         float* s_out, bf16* s_bf, float* x_buf, int reinject,
                         int M, int d, cudaStream_t st);
-// m = silu(gu[:, :F]) * gu[:, F:] (bf16), rows M.
-void launch_swiglu(const float* gu, bf16* m, int M, int F, cudaStream_t st);
 // Final greedy argmax over [B][n] partials or full logits rows.
 void launch_argmax_partials(const float* val, const int* idx, int B, int n,
                             int* out, int* n_ctx, int T, cudaStream_t st);
@@ -187,9 +185,14 @@ void launch_attn_decode_fused(const DecAttnArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- GEMM ----
 // C[M, N] (f32, row stride ldc) = A[M, K] (bf16, row stride lda) * W[N, K]^T
-// optionally times col_scale[n].  M any, N % 128 == 0, K % 32 == 0.
+// optionally times col_scale[n], on tcgen05.  M, N any; K % 64 == 0.
 void launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
                       int M, int N, int K, const float* col_scale,
                       cudaStream_t st);
+// m[M, F] = silu(A W_g^T) * (A W_u^T) as bf16, W = [W_g; W_u] (2F rows).
+void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
+                        int ldm, int M, int F, int K, cudaStream_t st);
+// Device status word the tensor-core GEMM reports timeouts to.
+void set_tc_error_word(int* err);
 
 }  // namespace dory

@@ -96,32 +96,6 @@ __device__ __forceinline__ void head_rope_norm(const float* src, size_t pstride,
   }
 }
 
-// Copy keys [j0, j0 + nk) of (b, kvh) into shared rows; position p (the
-// token of this call) comes from `fresh` (already BF16-exact floats).
-__device__ __forceinline__ void load_tile_fresh(bf16* dst, const bf16* base,
-                                                const KVSlot& kv,
-                                                const CacheGeo& g, int Hkv,
-                                                int hd, int b, int kvh, int j0,
-                                                int nk, int p,
-                                                const float* fresh) {
-  const int vec = hd / 8;
-  for (int id = threadIdx.x; id < nk * vec; id += blockDim.x) {
-    const int r = id / vec, c = id - r * vec;
-    uint4 v;
-    if (j0 + r == p) {
-      __nv_bfloat162 t[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        t[e] = __floats2bfloat162_rn(fresh[c * 8 + 2 * e], fresh[c * 8 + 2 * e + 1]);
-      v = *reinterpret_cast<uint4*>(t);
-    } else {
-      const size_t off = kv_index(kv, g, Hkv, hd, b, kvh, j0 + r);
-      v = *reinterpret_cast<const uint4*>(base + off + c * 8);
-    }
-    *reinterpret_cast<uint4*>(dst + r * (hd + KPAD) + c * 8) = v;
-  }
-}
-
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
                    (uint32_t)__cvta_generic_to_shared(dst)),

@@ -1,0 +1,405 @@
+// BF16 GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA) for prefill
+// projections: C[M, N] = A[M, K] * W[N, K]^T (f32 accumulate), A the bf16
+// activations (row stride lda), W the bf16 weights, both K-contiguous.
+//
+// One CTA computes a 128 x 256 output tile:
+//   warp 0 lane 0  streams 128x64 A and 256x64 W tiles with 2-D TMA loads
+//                  (128-byte swizzle) into a ring of STAGES shared-memory
+//                  stages (full/empty mbarriers);
+//   warp 1 lane 0  issues tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256,
+//                  K=16; 4 per stage) into a 256-column f32 TMEM accumulator
+//                  and releases each stage with tcgen05.commit;
+//   warps 0-3      wait for the accumulator, read it with tcgen05.ld
+//                  (warp w owns TMEM lanes 32w..32w+31 = tile rows) and run
+//                  the epilogue (f32 store, optional per-column scale, or the
+//                  SwiGLU pairing of gate/up column halves).
+// Every mbarrier wait is bounded: on timeout the CTA records ERRBIT_TIMEOUT,
+// waits (bounded) for its outstanding copies and MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "common.cuh"
+
+namespace dory {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int kTmemCols = 256;
+constexpr uint32_t kStageA = BM * BK * 2;     // 16 KB
+constexpr uint32_t kStageB = BN * BK * 2;     // 32 KB
+constexpr long kSpin = 1L << 22;    // bounded polls (~1 s)
+
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, int n) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   su32(b)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
+  for (long i = 0; i < kSpin; ++i)
+    if (mbar_try(b, parity)) return true;
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map,
+                                            int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_"
+      "tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(su32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(su32(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile stored by TMA with the
+// 128-byte swizzle: rows of 64 bf16 (128 B), 8-row atoms 1024 B apart.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);        // start address
+  d |= (uint64_t)1 << 16;                        // leading byte offset (unused)
+  d |= (uint64_t)(1024 >> 4) << 32;              // stride byte offset
+  d |= (uint64_t)1 << 46;                        // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                        // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor, kind::f16: f32 accumulator, bf16 A and B, both
+// K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b,
+                                          uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 "
+      "[%0];" ::"r"(su32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive f32 columns of this thread's TMEM lane (load and wait in
+// one asm statement so no use of the registers can precede the wait).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,"
+      "%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,"
+      "%27,%28,%29,%30,%31}, [%32];\n"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
+        "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
+        "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+struct TcArgs {
+  int M, N, K;          // output rows, output columns (SwiGLU: features)
+  int swiglu;           // 1: W rows [n, n + F) gate/up pairs, F = up_off
+  int up_off;           // row offset of the up half (SwiGLU)
+  float* C;             // f32 out [M][ldc] (plain)
+  bf16* Cb;             // bf16 out [M][ldc] (SwiGLU)
+  int ldc;
+  const float* col_scale;
+  int* err;
+};
+
+__global__ void __launch_bounds__(128, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
+               const __grid_constant__ CUtensorMap tmB, const TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment of the swizzled tiles (shared-window address)
+  const uint32_t raw = su32(smem_raw);
+  uint8_t* base = smem_raw + ((1024 - (raw & 1023)) & 1023);
+  uint8_t* sA = base;
+  uint8_t* sB = base + STAGES * kStageA;
+  __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], accum;
+  __shared__ uint32_t tmem_base;
+  __shared__ int s_fail, s_issued;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * BM;
+  const int ncols = a.swiglu ? BN / 2 : BN;      // output columns of the tile
+  const int n0 = blockIdx.x * ncols;
+  const int KB = a.K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(full + i, 1);
+      mbar_init(empty + i, 1);
+    }
+    mbar_init(&accum, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
+    s_fail = 0;
+    s_issued = 0;
+  }
+  if (warp == 0) {
+    asm volatile(
+        "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+            su32(&tmem_base)),
+        "r"(kTmemCols)
+        : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::
+                     : "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == 0 && lane == 0) {
+    // ---- TMA producer ----------------------------------------------------
+    const int nb0 = a.swiglu ? n0 : n0;
+    const int nb1 = a.swiglu ? a.up_off + n0 : n0 + BN / 2;
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % STAGES, use = kb / STAGES;
+      if (use > 0 && !mbar_wait(empty + s, (uint32_t)((use - 1) & 1))) {
+        atomicOr(&s_fail, 1);
+        break;
+      }
+      mbar_expect_tx(full + s, kStageA + kStageB);
+      tma_load_2d(sA + s * kStageA, &tmA, kb * BK, m0, full + s);
+      tma_load_2d(sB + s * kStageB, &tmB, kb * BK, nb0, full + s);
+      tma_load_2d(sB + s * kStageB + kStageB / 2, &tmB, kb * BK, nb1, full + s);
+      s_issued = kb + 1;
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issuer ------------------------------------------------------
+    const uint32_t idesc = idesc_bf16(BM, BN);
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % STAGES, use = kb / STAGES;
+      if (!mbar_wait(full + s, (uint32_t)(use & 1))) {
+        atomicOr(&s_fail, 1);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a0 = su32(sA + s * kStageA), b0 = su32(sB + s * kStageB);
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk)
+        umma_bf16(tmem, smem_desc(a0 + kk * 32), smem_desc(b0 + kk * 32), idesc,
+                  (kb | kk) != 0);
+      umma_commit(empty + s);                     // stage free once read
+    }
+    // accumulator complete (also after a failed wait: the commit then
+    // tracks the MMAs already issued, so teardown can wait for them)
+    umma_commit(&accum);
+  }
+  __syncwarp();
+
+  // ---- epilogue: TMEM -> registers -> global ------------------------------
+  const bool got = mbar_wait(&accum, 0);
+  if (!got && lane == 0) atomicOr(&s_fail, 1);
+  tc_fence_after();
+  __syncthreads();
+  const bool failed = *(volatile int*)&s_fail != 0;
+  if (!failed) {
+    const int row = m0 + warp * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    if (!a.swiglu) {
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        float v[32];
+        tmem_ld32(trow + c0, v);
+        const int col = n0 + c0;
+        if (row < a.M && col < a.N) {
+          float* dst = a.C + (size_t)row * a.ldc + col;
+          if (a.col_scale) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (col + i < a.N) v[i] *= a.col_scale[col + i];
+          }
+          // 16-byte stores only when every row start stays 16-byte aligned
+          if (col + 32 <= a.N && (a.ldc & 3) == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + i) =
+                  make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          } else {
+            for (int i = 0; i < 32 && col + i < a.N; ++i) dst[i] = v[i];
+          }
+        }
+      }
+    } else {
+      for (int c0 = 0; c0 < BN / 2; c0 += 32) {
+        float g[32], u[32];
+        tmem_ld32(trow + c0, g);
+        tmem_ld32(trow + BN / 2 + c0, u);
+        const int col = n0 + c0;
+        if (row < a.M && col < a.N) {
+          bf16* dst = a.Cb + (size_t)row * a.ldc + col;
+          if (col + 32 <= a.N && (a.ldc & 1) == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float m0v = g[i] * sigmoidf_(g[i]) * u[i];
+              const float m1v = g[i + 1] * sigmoidf_(g[i + 1]) * u[i + 1];
+              *reinterpret_cast<__nv_bfloat162*>(dst + i) =
+                  __floats2bfloat162_rn(m0v, m1v);
+            }
+          } else {
+            for (int i = 0; i < 32 && col + i < a.N; ++i)
+              dst[i] = __float2bfloat16_rn(g[i] * sigmoidf_(g[i]) * u[i]);
+          }
+        }
+      }
+    }
+  } else if (threadIdx.x == 0) {
+    // give in-flight copies and MMAs a bounded chance to land before the
+    // shared memory and TMEM are released
+    atomicOr(a.err, ERRBIT_TIMEOUT);
+    const int hi = s_issued, lo = hi > STAGES ? hi - STAGES : 0;
+    for (int kb = lo; kb < hi; ++kb)
+      if (!mbar_wait(full + kb % STAGES, (uint32_t)((kb / STAGES) & 1))) break;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(
+                     tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host ----
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault,
+                                &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over rows x cols (cols contiguous, row stride ld
+// elements), box 128 rows x 64 columns, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* ptr, long rows, long cols, long ld) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {BK, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor maps of weights are built once per (pointer, shape).
+std::mutex g_map_mu;
+std::map<std::tuple<const void*, long, long, long>, CUtensorMap> g_maps;
+
+bool weight_map(CUtensorMap* m, const void* ptr, long rows, long cols) {
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  auto key = std::make_tuple(ptr, rows, cols, cols);
+  auto it = g_maps.find(key);
+  if (it != g_maps.end()) {
+    *m = it->second;
+    return true;
+  }
+  if (!make_map(m, ptr, rows, cols, cols)) return false;
+  g_maps[key] = *m;
+  return true;
+}
+
+int* g_err_ptr = nullptr;
+
+size_t tc_smem() { return (size_t)STAGES * (kStageA + kStageB) + 1024; }
+
+bool launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const TcArgs& a,
+               dim3 grid, cudaStream_t st) {
+  static bool configured = false;
+  if (!configured) {
+    cudaFuncSetAttribute(gemm_tc_kernel,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)tc_smem());
+    configured = true;
+  }
+  return launch_k(gemm_tc_kernel, grid, dim3(128), tc_smem(), st, ma, mb, a) ==
+         cudaSuccess;
+}
+
+}  // namespace
+
+void set_tc_error_word(int* err) { g_err_ptr = err; }
+
+// C[M, N] = A[M, K] W[N, K]^T (f32, optional column scale) on tcgen05.
+void launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
+                      int M, int N, int K, const float* col_scale,
+                      cudaStream_t st) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, A, M, K, lda) || !weight_map(&mb, W, N, K)) {
+    fprintf(stderr, "dory: tensor map creation failed\n");
+    return;
+  }
+  TcArgs a{M, N, K, 0, 0, C, nullptr, ldc, col_scale, g_err_ptr};
+  launch_tc(ma, mb, a, dim3((N + BN - 1) / BN, (M + BM - 1) / BM), st);
+}
+
+// m[M, F] = silu(A W_g^T) * (A W_u^T) (bf16) with W = [W_g; W_u] of 2F rows.
+void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
+                        int ldm, int M, int F, int K, cudaStream_t st) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, A, M, K, lda) || !weight_map(&mb, W, 2L * F, K)) {
+    fprintf(stderr, "dory: tensor map creation failed\n");
+    return;
+  }
+  TcArgs a{M, F, K, 1, F, nullptr, m, ldm, nullptr, g_err_ptr};
+  launch_tc(ma, mb, a, dim3((F + BN / 2 - 1) / (BN / 2), (M + BM - 1) / BM), st);
+}
+
+}  // namespace dory

@@ -180,18 +180,6 @@ __global__ void update_rows_kernel(const float* s_in, const float* h,
                   s_bf + o, tmp, red);
 }
 
-__global__ void swiglu_kernel(const float* gu, bf16* m, int M, int F) {
-  pdl_wait();
-  pdl_trigger();
-  const size_t total = (size_t)M * F;
-  for (size_t id = blockIdx.x * (size_t)blockDim.x + threadIdx.x; id < total;
-       id += (size_t)gridDim.x * blockDim.x) {
-    const size_t r = id / F, c = id - r * F;
-    const float g = gu[r * 2 * F + c], u = gu[r * 2 * F + F + c];
-    m[id] = __float2bfloat16_rn(g * sigmoidf_(g) * u);
-  }
-}
-
 // Lowest index among the maxima; NaN entries never win.
 __device__ __forceinline__ void better(float& v, int& i, float cv, int ci) {
   if (cv > v || (cv == v && ci < i)) { v = cv; i = ci; }
@@ -283,13 +271,6 @@ void launch_update_rows(const float* s_in, const float* h, const float* alpha,
                         int M, int d, cudaStream_t st) {
   launch_k(update_rows_kernel, dim3(M), dim3(256), d * sizeof(float), st, s_in,
            h, alpha, s_out, s_bf, x_buf, reinject, d);
-}
-
-void launch_swiglu(const float* gu, bf16* m, int M, int F, cudaStream_t st) {
-  const size_t total = (size_t)M * F;
-  size_t blocks = (total + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  launch_k(swiglu_kernel, dim3((int)blocks), dim3(256), 0, st, gu, m, M, F);
 }
 
 void launch_argmax_partials(const float* val, const int* idx, int B, int n,

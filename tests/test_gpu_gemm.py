@@ -1,0 +1,40 @@
+"""The tcgen05 projection GEMM (prefill) against a float64 NumPy matmul of the
+same BF16 operands, through the C ABI, on shapes with ragged M and N tails
+and on the Dory projection shapes."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from looped_ngpt_b200 import _lib
+from synthetic.gen import f32_to_bf16_bits, bf16_bits_to_f32
+
+pytestmark = pytest.mark.gpu
+
+
+def _bf16(rng, shape, scale=1.0):
+    return f32_to_bf16_bits(rng.standard_normal(shape).astype(np.float32) * scale)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 64), (64, 640, 256), (200, 300, 128),
+                                   (129, 257, 192), (512, 6400, 2560),
+                                   (256, 2560, 10240)])
+def test_gemm_matches_numpy(M, N, K):
+    rng = np.random.default_rng(M * 7 + N * 3 + K)
+    A = _bf16(rng, (M, K))
+    W = _bf16(rng, (N, K), 1.0 / np.sqrt(K))
+    dA = torch.from_numpy(A.view(np.int16)).cuda()
+    dW = torch.from_numpy(W.view(np.int16)).cuda()
+    dC = torch.full((M, N), float("nan"), device="cuda")
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    lib = _lib.load()
+    assert lib.dory_debug_gemm_bf16(ctypes.c_void_p(dA.data_ptr()), K,
+                                    ctypes.c_void_p(dW.data_ptr()),
+                                    ctypes.c_void_p(dC.data_ptr()), M, N, K, s) == 0
+    torch.cuda.synchronize()
+    ref = bf16_bits_to_f32(A).astype(np.float64) @ bf16_bits_to_f32(W).astype(np.float64).T
+    got = dC.cpu().numpy()
+    # f32 accumulation of K products of magnitude ~|ref|/sqrt(K)
+    tol = 1e-5 * np.sqrt(K) * (np.abs(ref).max() + 1)
+    assert np.abs(got - ref).max() <= tol, np.abs(got - ref).max()
