@@ -34,20 +34,6 @@ __device__ __forceinline__ Split split_of(int p, int window) {
   return s;
 }
 
-// Copy keys [j0, j0 + nk) of (b, kvh) into shared rows [0, nk).
-__device__ __forceinline__ void load_tile(bf16* dst, const bf16* base,
-                                          const KVSlot& kv, const CacheGeo& g,
-                                          int Hkv, int hd, int b, int kvh,
-                                          int j0, int nk) {
-  const int vec = hd / 8;
-  for (int id = threadIdx.x; id < nk * vec; id += blockDim.x) {
-    const int r = id / vec, c = id - r * vec;
-    const size_t off = kv_index(kv, g, Hkv, hd, b, kvh, j0 + r);
-    *reinterpret_cast<uint4*>(dst + r * (hd + KPAD) + c * 8) =
-        *reinterpret_cast<const uint4*>(base + off + c * 8);
-  }
-}
-
 // ---------------------------------------------------------------- decode --
 // One warp: sum the split-K partials of one head of the fused QKVG output,
 // rotate (rotate-half RoPE), L2-normalise over the head, scale per dim.
@@ -429,126 +415,219 @@ __global__ void __launch_bounds__(2 * HD) attn_decode_fused_kernel(const DecAttn
 
 // --------------------------------------------------------------- prefill --
 // grid (ceil(T/64), Hq, B); block 256 = 64 query rows x 4 threads.
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0,
+                                        uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0,
+                                          uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile(
+      "ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+      : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4],
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Flash attention for prefill (T query tokens per sequence), one query head
+// per block, 64 queries (4 warps x 16 rows) per block, 64-key tiles of the
+// head's KV cache double-buffered in shared memory with cp.async.  S = Q K^T
+// and O += P V on the warp-level tensor-core path (m16n8k16, bf16 operands,
+// f32 accumulation); P stays in registers between the two products; online
+// softmax in exp2 units (q is pre-scaled by sqrt(h) log2 e).  Causal and
+// sliding-window masks per element.  Epilogue: gate * O / l as bf16.
+// grid (ceil(T/64), Hq, B); block 128.
 template <int HD>
-__global__ void __launch_bounds__(256) attn_prefill_kernel(const AttnArgs a) {
-  constexpr int QP = HD + 4;           // padded f32 row of Q
-  constexpr int KP = HD + KPAD;        // padded bf16 row of K / V
-  constexpr int DQ = HD / 4;           // output dims per thread
-  extern __shared__ float sm[];
-  float* Q_s = sm;                                   // [64][QP]
-  float* P_s = Q_s + 64 * QP;                        // [64][TK]
-  bf16* K_s = reinterpret_cast<bf16*>(P_s + 64 * TK);
-  bf16* V_s = K_s + TK * KP;
+__global__ void __launch_bounds__(128) attn_prefill_kernel(const AttnArgs a) {
+  constexpr int RP = HD + KPAD;
+  constexpr int KS = HD / 16;        // k-steps of Q K^T
+  constexpr int NO = HD / 8;         // n-tiles of O
+  extern __shared__ __align__(16) uint8_t smraw[];
+  bf16* Ks = reinterpret_cast<bf16*>(smraw);          // [2][64][RP]
+  bf16* Vs = Ks + 2 * 64 * RP;                        // [2][64][RP]
   const Dims& dm = a.dm;
   const int G = dm.Hq / dm.Hkv;
   const int h = blockIdx.y, b = blockIdx.z, kvh = h / G;
   const int t0 = blockIdx.x * 64;
-  const int r = threadIdx.x >> 2, qc = threadIdx.x & 3;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, tq = lane & 3;
+
+  // finite contents everywhere (partial tiles leave rows unwritten)
+  for (int i = threadIdx.x; i < 4 * 64 * RP / 8; i += 128)
+    reinterpret_cast<uint4*>(smraw)[i] = make_uint4(0, 0, 0, 0);
   pdl_wait();
   pdl_trigger();
   const int n0 = *a.g.n_ctx;
-  const int t = t0 + r;
-  const bool valid = t < a.T;
-  const int p = n0 + t;
-  if (n0 + a.T > a.g.max_ctx) return;   // reported by the K/V writer
+  if (n0 + a.T > a.g.max_ctx) return;                 // reported by the writer
 
-  for (int i = threadIdx.x; i < 64 * HD; i += 256) {
-    const int rr = i / HD, c = i - rr * HD;
-    float v = 0.f;
-    if (t0 + rr < a.T) v = a.q[((size_t)b * a.T + t0 + rr) * dm.qdim + h * HD + c];
-    Q_s[rr * QP + c] = v;
+  const int tr0 = t0 + 16 * warp + g, tr1 = tr0 + 8;  // call-local rows
+  const int p0 = n0 + tr0, p1 = n0 + tr1;             // positions
+  uint32_t qf[KS][4];
+  {
+    const float* q0 = a.q + ((size_t)b * a.T + min(tr0, a.T - 1)) * dm.qdim + h * HD;
+    const float* q1 = a.q + ((size_t)b * a.T + min(tr1, a.T - 1)) * dm.qdim + h * HD;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      const int c = 16 * kk + 2 * tq;
+      const float2 x0 = *reinterpret_cast<const float2*>(q0 + c);
+      const float2 x1 = *reinterpret_cast<const float2*>(q1 + c);
+      const float2 x2 = *reinterpret_cast<const float2*>(q0 + c + 8);
+      const float2 x3 = *reinterpret_cast<const float2*>(q1 + c + 8);
+      qf[kk][0] = pack_bf16(x0.x, x0.y);
+      qf[kk][1] = pack_bf16(x1.x, x1.y);
+      qf[kk][2] = pack_bf16(x2.x, x2.y);
+      qf[kk][3] = pack_bf16(x3.x, x3.y);
+    }
   }
+  float o[NO][4];
+#pragma unroll
+  for (int n = 0; n < NO; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
   const int kmin = a.window ? max(0, n0 + t0 - a.window + 1) : 0;
   const int kmax = n0 + min(a.T, t0 + 64);
-  float m = -INFINITY, l = 0.f;
-  float acc[DQ];
-#pragma unroll
-  for (int i = 0; i < DQ; ++i) acc[i] = 0.f;
+  __syncthreads();                                    // zero fill done
+  issue_kv_tile<HD>(Ks, Vs, a.kv, a.g, dm.Hkv, b, kvh, kmin,
+                    min(64, kmax - kmin), -1, 128);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  const uint32_t ks0 = (uint32_t)__cvta_generic_to_shared(Ks);
+  const uint32_t vs0 = (uint32_t)__cvta_generic_to_shared(Vs);
 
-  for (int j0 = kmin; j0 < kmax; j0 += TK) {
-    const int nk = min(TK, kmax - j0);
-    __syncthreads();
-    load_tile(K_s, a.kv.K, a.kv, a.g, dm.Hkv, HD, b, kvh, j0, nk);
-    load_tile(V_s, a.kv.V, a.kv, a.g, dm.Hkv, HD, b, kvh, j0, nk);
-    __syncthreads();
-    float s[16];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int jj = qc + 4 * i, j = j0 + jj;
-      const bool vis = valid && jj < nk && j <= p && (!a.window || j > p - a.window);
-      float v = -INFINITY;
-      if (vis) {
-        const float* qq = Q_s + r * QP;
-        const bf16* kk = K_s + jj * KP;
-        float d0 = 0.f;
-#pragma unroll 4
-        for (int c = 0; c < HD; c += 8) {
-          const uint4 kv = *reinterpret_cast<const uint4*>(kk + c);
-          const float4 qa = *reinterpret_cast<const float4*>(qq + c);
-          const float4 qb = *reinterpret_cast<const float4*>(qq + c + 4);
-          d0 = fmaf(qa.x, bf_lo(kv.x), d0);
-          d0 = fmaf(qa.y, bf_hi(kv.x), d0);
-          d0 = fmaf(qa.z, bf_lo(kv.y), d0);
-          d0 = fmaf(qa.w, bf_hi(kv.y), d0);
-          d0 = fmaf(qb.x, bf_lo(kv.z), d0);
-          d0 = fmaf(qb.y, bf_hi(kv.z), d0);
-          d0 = fmaf(qb.z, bf_lo(kv.w), d0);
-          d0 = fmaf(qb.w, bf_hi(kv.w), d0);
-        }
-        v = d0;
-      }
-      s[i] = v;
-      mx = fmaxf(mx, v);
-    }
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float m_new = fmaxf(m, mx);
-    float corr = 1.f, sum = 0.f;
-    if (m_new != -INFINITY) {
-      corr = exp2f(m - m_new);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float e = exp2f(s[i] - m_new);
-        P_s[r * TK + qc + 4 * i] = e;
-        sum += e;
-      }
+  int it = 0;
+  for (int j0 = kmin; j0 < kmax; j0 += 64, ++it) {
+    const int buf = it & 1;
+    if (j0 + 64 < kmax) {
+      issue_kv_tile<HD>(Ks + (buf ^ 1) * 64 * RP, Vs + (buf ^ 1) * 64 * RP,
+                        a.kv, a.g, dm.Hkv, b, kvh, j0 + 64,
+                        min(64, kmax - j0 - 64), -1, 128);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
     } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) P_s[r * TK + qc + 4 * i] = 0.f;
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
-    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-    l = l * corr + sum;
-    m = m_new;
-    __syncwarp();
+    __syncthreads();
+    const uint32_t kb = ks0 + buf * 64 * RP * 2, vb = vs0 + buf * 64 * RP * 2;
+
+    // S = Q K^T, 8 n-tiles of 8 keys
+    float sc[8][4];
 #pragma unroll
-    for (int i = 0; i < DQ; ++i) acc[i] *= corr;
-    for (int jj = 0; jj < nk; ++jj) {
-      const float pv = P_s[r * TK + jj];
-      const bf16* vv = V_s + jj * KP + qc * DQ;
+    for (int n = 0; n < 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
 #pragma unroll
-      for (int i = 0; i < DQ; i += 2) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vv + i));
-        acc[i] = fmaf(pv, f.x, acc[i]);
-        acc[i + 1] = fmaf(pv, f.y, acc[i + 1]);
+    for (int kk = 0; kk < KS; ++kk) {
+#pragma unroll
+      for (int nj = 0; nj < 4; ++nj) {
+        const int key = 16 * nj + (lane & 7) + ((lane >> 4) << 3);
+        const int col = 16 * kk + ((lane >> 3) & 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kb + (key * RP + col) * 2, b0, b1, b2, b3);
+        mma16816(sc[2 * nj], qf[kk], b0, b1);
+        mma16816(sc[2 * nj + 1], qf[kk], b2, b3);
       }
     }
-  }
-  if (!valid) return;
-  const float inv = 1.f / l;
-  const size_t row = (size_t)b * a.T + t;
+    // masks and online softmax (rows r0 = g, r1 = g + 8 of this warp)
+    float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < DQ; ++i) {
-    const size_t oi = row * dm.qdim + h * HD + qc * DQ + i;
-    a.a_out[oi] = __float2bfloat16_rn(a.gate[oi] * acc[i] * inv);
+    for (int n = 0; n < 8; ++n) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int j = j0 + 8 * n + 2 * tq + e;
+        const bool in = j < kmax;
+        const bool v0 = in && j <= p0 && (!a.window || j > p0 - a.window);
+        const bool v1 = in && j <= p1 && (!a.window || j > p1 - a.window);
+        if (!v0) sc[n][e] = -INFINITY;
+        if (!v1) sc[n][2 + e] = -INFINITY;
+        mx0 = fmaxf(mx0, sc[n][e]);
+        mx1 = fmaxf(mx1, sc[n][2 + e]);
+      }
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float ref0 = mn0 == -INFINITY ? 0.f : mn0;   // all masked so far
+    const float ref1 = mn1 == -INFINITY ? 0.f : mn1;
+    const float c0 = exp2f(m0 - ref0), c1 = exp2f(m1 - ref1);
+    float s0 = 0.f, s1 = 0.f;
+    uint32_t pf[4][4];                                // P as A fragments
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      const float e0 = exp2f(sc[n][0] - ref0), e1 = exp2f(sc[n][1] - ref0);
+      const float e2 = exp2f(sc[n][2] - ref1), e3 = exp2f(sc[n][3] - ref1);
+      s0 += e0 + e1;
+      s1 += e2 + e3;
+      const int kk2 = n >> 1, hi = n & 1;
+      pf[kk2][hi * 2 + 0] = pack_bf16(e0, e1);
+      pf[kk2][hi * 2 + 1] = pack_bf16(e2, e3);
+    }
+    s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+    s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+    l0 = l0 * c0 + s0;
+    l1 = l1 * c1 + s1;
+    m0 = mn0;
+    m1 = mn1;
+#pragma unroll
+    for (int n = 0; n < NO; ++n) {
+      o[n][0] *= c0; o[n][1] *= c0;
+      o[n][2] *= c1; o[n][3] *= c1;
+    }
+    // O += P V: 4 k-steps of 16 keys, NO/2 pairs of 8-dim n-tiles
+#pragma unroll
+    for (int kk2 = 0; kk2 < 4; ++kk2) {
+      const uint32_t af[4] = {pf[kk2][0], pf[kk2][1], pf[kk2][2], pf[kk2][3]};
+#pragma unroll
+      for (int nn = 0; nn < NO / 2; ++nn) {
+        const int key = 16 * kk2 + (lane & 15);
+        const int col = 16 * nn + ((lane >> 4) << 3);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vb + (key * RP + col) * 2, b0, b1, b2, b3);
+        mma16816(o[2 * nn], af, b0, b1);
+        mma16816(o[2 * nn + 1], af, b2, b3);
+      }
+    }
+    __syncthreads();                                  // buffer free for reuse
+  }
+
+  // epilogue: a = gate * O / l
+  const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+#pragma unroll
+  for (int n = 0; n < NO; ++n) {
+    const int dim = h * HD + 8 * n + 2 * tq;
+    if (tr0 < a.T) {
+      const size_t r = ((size_t)b * a.T + tr0) * dm.qdim + dim;
+      const float2 gv = *reinterpret_cast<const float2*>(a.gate + r);
+      *reinterpret_cast<__nv_bfloat162*>(a.a_out + r) =
+          __floats2bfloat162_rn(gv.x * o[n][0] * i0, gv.y * o[n][1] * i0);
+    }
+    if (tr1 < a.T) {
+      const size_t r = ((size_t)b * a.T + tr1) * dm.qdim + dim;
+      const float2 gv = *reinterpret_cast<const float2*>(a.gate + r);
+      *reinterpret_cast<__nv_bfloat162*>(a.a_out + r) =
+          __floats2bfloat162_rn(gv.x * o[n][2] * i1, gv.y * o[n][3] * i1);
+    }
   }
 }
 
 template <int HD>
 void launch_prefill_t(const AttnArgs& a, cudaStream_t st) {
-  const size_t smem = (64 * (HD + 4) + 64 * TK) * sizeof(float) +
-                      2 * TK * (HD + KPAD) * sizeof(bf16);
+  const size_t smem = 4 * 64 * (HD + KPAD) * sizeof(bf16);
   static bool configured = false;
   if (!configured) {
     cudaFuncSetAttribute(attn_prefill_kernel<HD>,
@@ -556,7 +635,7 @@ void launch_prefill_t(const AttnArgs& a, cudaStream_t st) {
     configured = true;
   }
   dim3 grid((a.T + 63) / 64, a.dm.Hq, a.B);
-  launch_k(attn_prefill_kernel<HD>, grid, dim3(256), smem, st, a);
+  launch_k(attn_prefill_kernel<HD>, grid, dim3(128), smem, st, a);
 }
 
 }  // namespace
