@@ -140,9 +140,9 @@ CacheLayout cache_layout(const dory_model* m, int B, int max_ctx,
 
 
 struct WS {
-  float *s0, *s1, *sfin, *x, *qkvg, *q, *gate, *h, *part_o, *part_ml,
+  float *s0, *s1, *sfin, *x, *qkvg, *gate, *h, *part_o, *part_ml,
       *rope, *amax_val;
-  bf16 *s_bf, *a, *mact;
+  bf16 *s_bf, *a, *mact, *qb;
   int* amax_idx;
   int* counters;
   size_t total;
@@ -167,7 +167,7 @@ WS ws_layout(const dory_model* m, int B, int T, char* base) {
   w.x = (float*)take(M * dm.d * 4);
   w.s_bf = (bf16*)take(M * dm.d * 2);
   w.qkvg = (float*)take(kMaxS * M * dm.rows_qkvg * 4);
-  w.q = (float*)take(M * dm.qdim * 4);
+  w.qb = (bf16*)take(M * dm.qdim * 2);
   w.gate = (float*)take(M * dm.qdim * 4);
   w.a = (bf16*)take(M * dm.qdim * 2);
   w.h = (float*)take(kMaxS * M * dm.d * 4);
@@ -571,8 +571,21 @@ void enqueue_forward(const CallCtx& x) {
                            dm.d, x.st);
         std::swap(cur, other);
       }
-      gemm_run(m, w.s_bf, dm.d, bw.w_qkvg, w.qkvg, dm.rows_qkvg, x.M,
-               dm.rows_qkvg, dm.d, nullptr, x.st, "gemm_qkvg");
+      if (x.T == 1) {
+        gemm_run(m, w.s_bf, dm.d, bw.w_qkvg, w.qkvg, dm.rows_qkvg, x.M,
+                 dm.rows_qkvg, dm.d, nullptr, x.st, "gemm_qkvg");
+      } else {
+        QkvGemmArgs qg{};
+        qg.M = x.M; qg.T = x.T; qg.dm = dm; qg.s_q = bw.s_q; qg.s_k = bw.s_k;
+        qg.rope = w.rope + (full ? (size_t)x.T * half * 2 : 0);
+        qg.q_scale = q_scale; qg.kv = kv; qg.g = geo;
+        qg.q_out = w.qb; qg.gate_out = w.gate;
+        Prof p(m, x.st, "gemm_qkv",
+               (double)x.M * dm.d * 2 + (double)dm.rows_qkvg * dm.d * 2 +
+                   (double)x.M * (dm.qdim * 6.0 + dm.kvdim * 4.0),
+               2.0 * x.M * dm.rows_qkvg * dm.d);
+        launch_gemm_qkv(w.s_bf, dm.d, bw.w_qkvg, qg, x.st);
+      }
     }
     if (x.T == 1) {
       DecAttnArgs da{};
@@ -589,20 +602,8 @@ void enqueue_forward(const CallCtx& x) {
              4.0 * x.B * dm.Hq * nk * dm.hd);
       launch_attn_decode_fused(da, x.st);
     } else {
-      QkvPostArgs qa{};
-      qa.qkvg = w.qkvg; qa.S = S_qkvg; qa.M = x.M; qa.T = x.T; qa.B = x.B;
-      qa.dm = dm; qa.s_q = bw.s_q; qa.s_k = bw.s_k;
-      qa.rope = w.rope + (full ? (size_t)x.T * half * 2 : 0);
-      qa.q_scale = q_scale; qa.q_out = w.q; qa.gate_out = w.gate;
-      qa.kv = kv; qa.g = geo; qa.err = m->d_status;
-      {
-        Prof p(m, x.st, "qkv_post",
-               (double)x.M * (dm.rows_qkvg * 4.0 * S_qkvg + dm.qdim * 8.0 +
-                              dm.kvdim * 4.0), 0);
-        launch_qkv_post(qa, x.st);
-      }
       AttnArgs aa{};
-      aa.q = w.q; aa.gate = w.gate; aa.B = x.B; aa.T = x.T; aa.dm = dm;
+      aa.q = w.qb; aa.gate = w.gate; aa.B = x.B; aa.T = x.T; aa.dm = dm;
       aa.window = full ? 0 : dm.window; aa.kv = kv; aa.g = geo;
       aa.a_out = w.a; aa.err = m->d_status;
       double vis = 0;

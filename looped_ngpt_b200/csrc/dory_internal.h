@@ -123,19 +123,6 @@ void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
                   bf16* s_bf, int* err, int vocab, int* counters,
                   int n_counters, float* rope, const int* n_ctx, int hd,
                   double theta_swa, double theta_full, cudaStream_t st);
-// RoPE + per-head L2 norm + q/k scales + sigmoid gate + K/V cache write.
-struct QkvPostArgs {
-  const float* qkvg; int S; int M; int T; int B;
-  Dims dm;
-  const float* s_q; const float* s_k;
-  const float* rope;   // table of this layer's type [T][hd/2][2]
-  float q_scale;       // extra factor folded into q (softmax temperature)
-  float* q_out;        // [M][qdim]
-  float* gate_out;     // [M][qdim]
-  KVSlot kv; CacheGeo g;
-  int* err;
-};
-void launch_qkv_post(const QkvPostArgs& a, cudaStream_t st);
 // Prefill: s_new = N(s + alpha (N(h) - s)) per row (+ loop re-injection).
 void launch_update_rows(const float* s_in, const float* h, const float* alpha,
                         float* s_out, bf16* s_bf, float* x_buf, int reinject,
@@ -151,7 +138,7 @@ void launch_cache_init(int* n_ctx, int* block_table, int B, int pages_per_seq,
 
 // ----------------------------------------------------------- attention ----
 struct AttnArgs {
-  const float* q;      // [M][qdim], scaled by sqrt(hd) * log2(e)
+  const bf16* q;       // [M][qdim], scaled by sqrt(hd) * log2(e)
   const float* gate;   // [M][qdim] sigmoid(g)
   int B, T;
   Dims dm;
@@ -192,6 +179,21 @@ void launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
 // m[M, F] = silu(A W_g^T) * (A W_u^T) as bf16, W = [W_g; W_u] (2F rows).
 void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
                         int ldm, int M, int F, int K, cudaStream_t st);
+// Prefill q/k/v/gate projection with the RoPE, per-head L2 norm, scales,
+// KV-cache write and gate sigmoid in the GEMM epilogue (one tile column per
+// head).  A: bf16 [M][d] activations.
+struct QkvGemmArgs {
+  int M, T;
+  Dims dm;
+  const float* s_q; const float* s_k;
+  const float* rope;   // this layer type's table [T][hd/2][2]
+  float q_scale;
+  KVSlot kv; CacheGeo g;
+  bf16* q_out;         // [M][qdim]
+  float* gate_out;     // [M][qdim]
+};
+void launch_gemm_qkv(const bf16* A, int lda, const bf16* W,
+                     const QkvGemmArgs& q, cudaStream_t st);
 // Device status word the tensor-core GEMM reports timeouts to.
 void set_tc_error_word(int* err);
 

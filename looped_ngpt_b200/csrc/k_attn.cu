@@ -479,19 +479,15 @@ __global__ void __launch_bounds__(128) attn_prefill_kernel(const AttnArgs a) {
   const int p0 = n0 + tr0, p1 = n0 + tr1;             // positions
   uint32_t qf[KS][4];
   {
-    const float* q0 = a.q + ((size_t)b * a.T + min(tr0, a.T - 1)) * dm.qdim + h * HD;
-    const float* q1 = a.q + ((size_t)b * a.T + min(tr1, a.T - 1)) * dm.qdim + h * HD;
+    const bf16* q0 = a.q + ((size_t)b * a.T + min(tr0, a.T - 1)) * dm.qdim + h * HD;
+    const bf16* q1 = a.q + ((size_t)b * a.T + min(tr1, a.T - 1)) * dm.qdim + h * HD;
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
       const int c = 16 * kk + 2 * tq;
-      const float2 x0 = *reinterpret_cast<const float2*>(q0 + c);
-      const float2 x1 = *reinterpret_cast<const float2*>(q1 + c);
-      const float2 x2 = *reinterpret_cast<const float2*>(q0 + c + 8);
-      const float2 x3 = *reinterpret_cast<const float2*>(q1 + c + 8);
-      qf[kk][0] = pack_bf16(x0.x, x0.y);
-      qf[kk][1] = pack_bf16(x1.x, x1.y);
-      qf[kk][2] = pack_bf16(x2.x, x2.y);
-      qf[kk][3] = pack_bf16(x3.x, x3.y);
+      qf[kk][0] = *reinterpret_cast<const uint32_t*>(q0 + c);
+      qf[kk][1] = *reinterpret_cast<const uint32_t*>(q1 + c);
+      qf[kk][2] = *reinterpret_cast<const uint32_t*>(q0 + c + 8);
+      qf[kk][3] = *reinterpret_cast<const uint32_t*>(q1 + c + 8);
     }
   }
   float o[NO][4];

@@ -117,6 +117,11 @@ __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 // 32 consecutive f32 columns of this thread's TMEM lane (load and wait in
 // one asm statement so no use of the registers can precede the wait).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
@@ -139,17 +144,91 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+enum TcMode : int { TC_PLAIN = 0, TC_SWIGLU = 1, TC_QKV = 2 };
+
 struct TcArgs {
   int M, N, K;          // output rows, output columns (SwiGLU: features)
-  int swiglu;           // 1: W rows [n, n + F) gate/up pairs, F = up_off
-  int up_off;           // row offset of the up half (SwiGLU)
-  float* C;             // f32 out [M][ldc] (plain)
-  bf16* Cb;             // bf16 out [M][ldc] (SwiGLU)
+  int up_off;           // SwiGLU: row offset of the up half of W
+  float* C;             // TC_PLAIN: f32 out [M][ldc]
+  bf16* Cb;             // TC_SWIGLU: bf16 out [M][ldc]
   int ldc;
   const float* col_scale;
   int* err;
+  // TC_QKV: one tile column = one head of the fused q/k/v/gate projection
+  int T;                // tokens per sequence (rows are b * T + t)
+  int Hq, Hkv, qdim, kvdim;
+  const float* s_q; const float* s_k;
+  const float* rope;    // this layer type's table [T][hd/2][2] (cos, sin)
+  float q_scale;
+  KVSlot kv; CacheGeo g;
+  bf16* q_out;          // [M][qdim] bf16, scaled by sqrt(hd) log2 e
+  float* gate_out;      // [M][qdim] sigmoid(gate)
 };
 
+// Epilogue of a TC_QKV tile: this thread holds one row of one head (hd
+// columns).  q/k: rotate-half RoPE at the row's position, L2 norm over the
+// head, per-dim scale; k and v go to the KV cache slot, q to q_out; gate
+// heads get the sigmoid.
+template <int HD>
+__device__ __forceinline__ void qkv_epilogue(const TcArgs& a, int item,
+                                             int row, float (&v)[HD]) {
+  const int b = row / a.T, t = row - b * a.T;
+  int kind, head, col0;
+  if (item < a.Hq) { kind = 0; head = item; col0 = head * HD; }
+  else if (item < a.Hq + a.Hkv) { kind = 1; head = item - a.Hq; col0 = a.qdim + head * HD; }
+  else if (item < a.Hq + 2 * a.Hkv) {
+    kind = 2; head = item - a.Hq - a.Hkv; col0 = a.qdim + a.kvdim + head * HD;
+  } else {
+    kind = 3; head = item - a.Hq - 2 * a.Hkv; col0 = a.qdim + 2 * a.kvdim + head * HD;
+  }
+  (void)col0;
+  if (kind == 3) {
+    float* dst = a.gate_out + (size_t)row * a.qdim + head * HD;
+#pragma unroll
+    for (int i = 0; i < HD; i += 4)
+      *reinterpret_cast<float4*>(dst + i) =
+          make_float4(sigmoidf_(v[i]), sigmoidf_(v[i + 1]), sigmoidf_(v[i + 2]),
+                      sigmoidf_(v[i + 3]));
+    return;
+  }
+  const int p = *a.g.n_ctx + t;
+  if (kind != 0 && p >= a.g.max_ctx) {
+    atomicOr(a.err, ERRBIT_BOUNDS);
+    return;
+  }
+  if (kind != 2) {
+    constexpr int H2 = HD / 2;
+    const float* rt = a.rope + (size_t)t * H2 * 2;
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < H2; ++i) {
+      const float2 cs = *reinterpret_cast<const float2*>(rt + 2 * i);
+      const float x1 = v[i], x2 = v[i + H2];
+      v[i] = x1 * cs.x - x2 * cs.y;
+      v[i + H2] = x2 * cs.x + x1 * cs.y;
+      ss += v[i] * v[i] + v[i + H2] * v[i + H2];
+    }
+    const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+    const float* sc = (kind == 0 ? a.s_q : a.s_k) + head * HD;
+    const float f = kind == 0 ? inv * a.q_scale : inv;
+#pragma unroll
+    for (int i = 0; i < HD; ++i) v[i] *= sc[i] * f;
+  }
+  bf16* dst;
+  if (kind == 0) dst = a.q_out + (size_t)row * a.qdim + head * HD;
+  else dst = (kind == 1 ? a.kv.K : a.kv.V) +
+             kv_index(a.kv, a.g, a.Hkv, HD, b, head, p);
+#pragma unroll
+  for (int i = 0; i < HD; i += 8) {
+    uint4 u;
+    u.x = pack2(v[i], v[i + 1]); u.y = pack2(v[i + 2], v[i + 3]);
+    u.z = pack2(v[i + 4], v[i + 5]); u.w = pack2(v[i + 6], v[i + 7]);
+    *reinterpret_cast<uint4*>(dst + i) = u;
+  }
+}
+
+// TN: tile columns (MMA N): 256 for TC_PLAIN / TC_SWIGLU, hd for TC_QKV.
+template <int MODE, int TN>
 __global__ void __launch_bounds__(128, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                const __grid_constant__ CUtensorMap tmB, const TcArgs a) {
@@ -164,9 +243,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   __shared__ int s_fail, s_issued;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * BM;
-  const int ncols = a.swiglu ? BN / 2 : BN;      // output columns of the tile
-  const int n0 = blockIdx.x * ncols;
+  constexpr int OUTC = MODE == TC_SWIGLU ? TN / 2 : TN;   // output columns
+  const int n0 = blockIdx.x * OUTC;
   const int KB = a.K / BK;
+  constexpr uint32_t kB = (uint32_t)TN * BK * 2;          // B bytes per stage
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -198,23 +278,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
 
   if (warp == 0 && lane == 0) {
     // ---- TMA producer ----------------------------------------------------
-    const int nb0 = a.swiglu ? n0 : n0;
-    const int nb1 = a.swiglu ? a.up_off + n0 : n0 + BN / 2;
     for (int kb = 0; kb < KB; ++kb) {
       const int s = kb % STAGES, use = kb / STAGES;
       if (use > 0 && !mbar_wait(empty + s, (uint32_t)((use - 1) & 1))) {
         atomicOr(&s_fail, 1);
         break;
       }
-      mbar_expect_tx(full + s, kStageA + kStageB);
+      mbar_expect_tx(full + s, kStageA + kB);
       tma_load_2d(sA + s * kStageA, &tmA, kb * BK, m0, full + s);
-      tma_load_2d(sB + s * kStageB, &tmB, kb * BK, nb0, full + s);
-      tma_load_2d(sB + s * kStageB + kStageB / 2, &tmB, kb * BK, nb1, full + s);
+      if (MODE == TC_QKV) {
+        tma_load_2d(sB + s * kStageB, &tmB, kb * BK, blockIdx.x * TN, full + s);
+      } else {
+        const int nb1 = MODE == TC_SWIGLU ? a.up_off + n0 : n0 + TN / 2;
+        tma_load_2d(sB + s * kStageB, &tmB, kb * BK, n0, full + s);
+        tma_load_2d(sB + s * kStageB + kB / 2, &tmB, kb * BK, nb1, full + s);
+      }
       s_issued = kb + 1;
     }
   } else if (warp == 1 && lane == 0) {
     // ---- MMA issuer ------------------------------------------------------
-    const uint32_t idesc = idesc_bf16(BM, BN);
+    constexpr uint32_t idesc = idesc_bf16(BM, TN);
     for (int kb = 0; kb < KB; ++kb) {
       const int s = kb % STAGES, use = kb / STAGES;
       if (!mbar_wait(full + s, (uint32_t)(use & 1))) {
@@ -244,8 +327,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   if (!failed) {
     const int row = m0 + warp * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-    if (!a.swiglu) {
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+    if (MODE == TC_PLAIN) {
+      for (int c0 = 0; c0 < TN; c0 += 32) {
         float v[32];
         tmem_ld32(trow + c0, v);
         const int col = n0 + c0;
@@ -267,28 +350,36 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
       }
-    } else {
-      for (int c0 = 0; c0 < BN / 2; c0 += 32) {
+    } else if (MODE == TC_SWIGLU) {
+      for (int c0 = 0; c0 < TN / 2; c0 += 32) {
         float g[32], u[32];
         tmem_ld32(trow + c0, g);
-        tmem_ld32(trow + BN / 2 + c0, u);
+        tmem_ld32(trow + TN / 2 + c0, u);
         const int col = n0 + c0;
         if (row < a.M && col < a.N) {
           bf16* dst = a.Cb + (size_t)row * a.ldc + col;
           if (col + 32 <= a.N && (a.ldc & 1) == 0) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              const float m0v = g[i] * sigmoidf_(g[i]) * u[i];
-              const float m1v = g[i + 1] * sigmoidf_(g[i + 1]) * u[i + 1];
-              *reinterpret_cast<__nv_bfloat162*>(dst + i) =
-                  __floats2bfloat162_rn(m0v, m1v);
-            }
+            for (int i = 0; i < 32; i += 2)
+              *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(
+                  g[i] * sigmoidf_(g[i]) * u[i],
+                  g[i + 1] * sigmoidf_(g[i + 1]) * u[i + 1]);
           } else {
             for (int i = 0; i < 32 && col + i < a.N; ++i)
               dst[i] = __float2bfloat16_rn(g[i] * sigmoidf_(g[i]) * u[i]);
           }
         }
       }
+    } else {
+      float v[TN];
+#pragma unroll
+      for (int c0 = 0; c0 < TN; c0 += 32) {
+        float t32[32];
+        tmem_ld32(trow + c0, t32);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[c0 + i] = t32[i];
+      }
+      if (row < a.M) qkv_epilogue<TN>(a, blockIdx.x, row, v);
     }
   } else if (threadIdx.x == 0) {
     // give in-flight copies and MMAs a bounded chance to land before the
@@ -325,13 +416,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D bf16 tensor map over rows x cols (cols contiguous, row stride ld
-// elements), box 128 rows x 64 columns, 128-byte swizzle, zero fill.
-bool make_map(CUtensorMap* m, const void* ptr, long rows, long cols, long ld) {
+// elements), box `brows` rows x 64 columns, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* ptr, long rows, long cols, long ld,
+              int brows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-  cuuint32_t box[2] = {BK, 128};
+  cuuint32_t box[2] = {BK, (cuuint32_t)brows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -339,19 +431,20 @@ bool make_map(CUtensorMap* m, const void* ptr, long rows, long cols, long ld) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tensor maps of weights are built once per (pointer, shape).
+// Tensor maps of weights are built once per (pointer, shape, box).
 std::mutex g_map_mu;
-std::map<std::tuple<const void*, long, long, long>, CUtensorMap> g_maps;
+std::map<std::tuple<const void*, long, long, int>, CUtensorMap> g_maps;
 
-bool weight_map(CUtensorMap* m, const void* ptr, long rows, long cols) {
+bool weight_map(CUtensorMap* m, const void* ptr, long rows, long cols,
+                int brows) {
   std::lock_guard<std::mutex> lock(g_map_mu);
-  auto key = std::make_tuple(ptr, rows, cols, cols);
+  auto key = std::make_tuple(ptr, rows, cols, brows);
   auto it = g_maps.find(key);
   if (it != g_maps.end()) {
     *m = it->second;
     return true;
   }
-  if (!make_map(m, ptr, rows, cols, cols)) return false;
+  if (!make_map(m, ptr, rows, cols, cols, brows)) return false;
   g_maps[key] = *m;
   return true;
 }
@@ -360,17 +453,27 @@ int* g_err_ptr = nullptr;
 
 size_t tc_smem() { return (size_t)STAGES * (kStageA + kStageB) + 1024; }
 
+template <int MODE, int TN>
 bool launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const TcArgs& a,
                dim3 grid, cudaStream_t st) {
   static bool configured = false;
   if (!configured) {
-    cudaFuncSetAttribute(gemm_tc_kernel,
+    cudaFuncSetAttribute(gemm_tc_kernel<MODE, TN>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)tc_smem());
     configured = true;
   }
-  return launch_k(gemm_tc_kernel, grid, dim3(128), tc_smem(), st, ma, mb, a) ==
-         cudaSuccess;
+  return launch_k(gemm_tc_kernel<MODE, TN>, grid, dim3(128), tc_smem(), st, ma,
+                  mb, a) == cudaSuccess;
+}
+
+TcArgs base_args(int M, int N, int K) {
+  TcArgs a{};
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.err = g_err_ptr;
+  return a;
 }
 
 }  // namespace
@@ -382,24 +485,66 @@ void launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
                       int M, int N, int K, const float* col_scale,
                       cudaStream_t st) {
   CUtensorMap ma, mb;
-  if (!make_map(&ma, A, M, K, lda) || !weight_map(&mb, W, N, K)) {
+  if (!make_map(&ma, A, M, K, lda, BM) || !weight_map(&mb, W, N, K, 128)) {
     fprintf(stderr, "dory: tensor map creation failed\n");
     return;
   }
-  TcArgs a{M, N, K, 0, 0, C, nullptr, ldc, col_scale, g_err_ptr};
-  launch_tc(ma, mb, a, dim3((N + BN - 1) / BN, (M + BM - 1) / BM), st);
+  TcArgs a = base_args(M, N, K);
+  a.C = C;
+  a.ldc = ldc;
+  a.col_scale = col_scale;
+  launch_tc<TC_PLAIN, BN>(ma, mb, a, dim3((N + BN - 1) / BN, (M + BM - 1) / BM),
+                          st);
 }
 
 // m[M, F] = silu(A W_g^T) * (A W_u^T) (bf16) with W = [W_g; W_u] of 2F rows.
 void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
                         int ldm, int M, int F, int K, cudaStream_t st) {
   CUtensorMap ma, mb;
-  if (!make_map(&ma, A, M, K, lda) || !weight_map(&mb, W, 2L * F, K)) {
+  if (!make_map(&ma, A, M, K, lda, BM) || !weight_map(&mb, W, 2L * F, K, 128)) {
     fprintf(stderr, "dory: tensor map creation failed\n");
     return;
   }
-  TcArgs a{M, F, K, 1, F, nullptr, m, ldm, nullptr, g_err_ptr};
-  launch_tc(ma, mb, a, dim3((F + BN / 2 - 1) / (BN / 2), (M + BM - 1) / BM), st);
+  TcArgs a = base_args(M, F, K);
+  a.up_off = F;
+  a.Cb = m;
+  a.ldc = ldm;
+  launch_tc<TC_SWIGLU, BN>(ma, mb, a,
+                           dim3((F + BN / 2 - 1) / (BN / 2), (M + BM - 1) / BM),
+                           st);
+}
+
+// Fused q/k/v/gate projection with the RoPE / QK-norm / KV-write epilogue.
+void launch_gemm_qkv(const bf16* A, int lda, const bf16* W, const QkvGemmArgs& q,
+                     cudaStream_t st) {
+  const int hd = q.dm.hd;
+  const int rows = q.dm.rows_qkvg;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, A, q.M, q.dm.d, lda, BM) ||
+      !weight_map(&mb, W, rows, q.dm.d, hd)) {
+    fprintf(stderr, "dory: tensor map creation failed\n");
+    return;
+  }
+  TcArgs a = base_args(q.M, rows, q.dm.d);
+  a.T = q.T;
+  a.Hq = q.dm.Hq;
+  a.Hkv = q.dm.Hkv;
+  a.qdim = q.dm.qdim;
+  a.kvdim = q.dm.kvdim;
+  a.s_q = q.s_q;
+  a.s_k = q.s_k;
+  a.rope = q.rope;
+  a.q_scale = q.q_scale;
+  a.kv = q.kv;
+  a.g = q.g;
+  a.q_out = q.q_out;
+  a.gate_out = q.gate_out;
+  const dim3 grid(rows / hd, (q.M + BM - 1) / BM);
+  switch (hd) {
+    case 64: launch_tc<TC_QKV, 64>(ma, mb, a, grid, st); break;
+    case 128: launch_tc<TC_QKV, 128>(ma, mb, a, grid, st); break;
+    default: launch_tc<TC_QKV, 160>(ma, mb, a, grid, st); break;
+  }
 }
 
 }  // namespace dory

@@ -1,6 +1,5 @@
 // Row-wise kernels of the looped nGPT forward pass: embedding, RoPE table,
-// RoPE + per-head QK L2 norm + K/V cache write, the prefill nGPT update,
-// SwiGLU, greedy argmax and cache bookkeeping.  All are HBM/L2-bound and
+// the prefill nGPT update, greedy argmax and cache bookkeeping.  All are HBM/L2-bound and
 // touch each element once.
 #include "common.cuh"
 
@@ -73,96 +72,6 @@ __global__ void embed_kernel(const int* tokens, const bf16* E, int d,
     const float v = __bfloat162float(e[i]) * inv;
     s[(size_t)row * d + i] = v;
     s_bf[(size_t)row * d + i] = __float2bfloat16_rn(v);
-  }
-}
-
-constexpr int kPairs = kMaxHeadDim / 64;   // rotate-half pairs per lane
-
-// One warp per (row, head item).  Items: [0, Hq) q heads, [Hq, Hq+Hkv) k
-// heads, [Hq+Hkv, Hq+2Hkv) v heads, [Hq+2Hkv, 2Hq+2Hkv) gate heads.
-__global__ void qkv_post_kernel(const QkvPostArgs a) {
-  const Dims& dm = a.dm;
-  pdl_wait();
-  pdl_trigger();
-  const int lane = threadIdx.x & 31;
-  const int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int n_items = 2 * dm.Hq + 2 * dm.Hkv;
-  const int row = blockIdx.y;
-  if (item >= n_items) return;
-  const int b = row / a.T, t = row - b * a.T;
-  const int p = *a.g.n_ctx + t;
-  const int hd = dm.hd, half = hd / 2;
-  const size_t part = (size_t)a.M * dm.rows_qkvg;
-  const float* src = a.qkvg + (size_t)row * dm.rows_qkvg;
-
-  int col0, kind, head;
-  if (item < dm.Hq) { kind = 0; head = item; col0 = head * hd; }
-  else if (item < dm.Hq + dm.Hkv) {
-    kind = 1; head = item - dm.Hq; col0 = dm.qdim + head * hd;
-  } else if (item < dm.Hq + 2 * dm.Hkv) {
-    kind = 2; head = item - dm.Hq - dm.Hkv; col0 = dm.qdim + dm.kvdim + head * hd;
-  } else {
-    kind = 3; head = item - dm.Hq - 2 * dm.Hkv;
-    col0 = dm.qdim + 2 * dm.kvdim + head * hd;
-  }
-  auto load = [&](int c) {
-    float v = 0.f;
-    for (int s = 0; s < a.S; ++s) v += src[s * part + col0 + c];
-    return v;
-  };
-
-  if (kind == 3) {
-    for (int c = lane; c < hd; c += 32)
-      a.gate_out[(size_t)row * dm.qdim + head * hd + c] = sigmoidf_(load(c));
-    return;
-  }
-  if (p >= a.g.max_ctx) {
-    if (lane == 0) atomicOr(a.err, ERRBIT_BOUNDS);
-    return;
-  }
-  if (kind == 2) {
-    bf16* dst = a.kv.V + kv_index(a.kv, a.g, dm.Hkv, hd, b, head, p);
-    for (int c = lane; c < hd; c += 32) dst[c] = __float2bfloat16_rn(load(c));
-    return;
-  }
-  // q or k: rotate-half RoPE, then L2 norm over the head, then scale.
-  float r1[kPairs], r2[kPairs];
-  float ss = 0.f;
-#pragma unroll
-  for (int j = 0; j < kPairs; ++j) {
-    const int i = lane + 32 * j;
-    r1[j] = r2[j] = 0.f;
-    if (i < half) {
-      const float x1 = load(i), x2 = load(i + half);
-      const float c = a.rope[(t * half + i) * 2], s = a.rope[(t * half + i) * 2 + 1];
-      r1[j] = x1 * c - x2 * s;
-      r2[j] = x2 * c + x1 * s;
-      ss += r1[j] * r1[j] + r2[j] * r2[j];
-    }
-  }
-  const float inv = 1.f / fmaxf(sqrtf(warp_sum(ss)), 1e-12f);
-  if (kind == 0) {
-    const float* sc = a.s_q + head * hd;
-    float* dst = a.q_out + (size_t)row * dm.qdim + head * hd;
-#pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
-      const int i = lane + 32 * j;
-      if (i < half) {
-        dst[i] = r1[j] * inv * sc[i] * a.q_scale;
-        dst[i + half] = r2[j] * inv * sc[i + half] * a.q_scale;
-      }
-    }
-  } else {
-    const float* sc = a.s_k + head * hd;
-    bf16* dst = a.kv.K + kv_index(a.kv, a.g, dm.Hkv, hd, b, head, p);
-#pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
-      const int i = lane + 32 * j;
-      if (i < half) {
-        dst[i] = __float2bfloat16_rn(r1[j] * inv * sc[i]);
-        dst[i + half] = __float2bfloat16_rn(r2[j] * inv * sc[i + half]);
-      }
-    }
   }
 }
 
@@ -258,12 +167,6 @@ void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
   launch_k(embed_kernel, dim3(M), dim3(256), 0, st, tokens, E, d, vocab, s,
            s_bf, err, counters, n_counters, rope, n_ctx, hd / 2, theta_swa,
            theta_full);
-}
-
-void launch_qkv_post(const QkvPostArgs& a, cudaStream_t st) {
-  const int items = 2 * a.dm.Hq + 2 * a.dm.Hkv;
-  dim3 grid((items + 7) / 8, a.M);
-  launch_k(qkv_post_kernel, grid, dim3(256), 0, st, a);
 }
 
 void launch_update_rows(const float* s_in, const float* h, const float* alpha,
