@@ -120,6 +120,19 @@ int dory_cache_length(const dory_cache* c, int* n_ctx);
 /* Forget all cached tokens (per_loop caches also forget their loop count). */
 int dory_cache_reset(dory_cache* c, void* stream);
 
+/* Input generation for long-context workloads (not a step of the method):
+ * make every sequence of the cache hold n_ctx tokens whose K/V entries are
+ * seeded synthetic values, entry (kind K=0/V=1, block i, slot, b, kv head,
+ * position, dim j) = bf16((2u - 1) * c_kind) with u the 24-bit uniform of
+ * SplitMix64(seed + counter) and c_K = sqrt(3 / head_dim), c_V =
+ * sqrt(3 / d); counter = ((((((kind*64 + i)*8 + slot)*4096 + b)*64 + kvh)
+ * *2^20 + pos)*512 + j), slot = loop t (1-based) for per_loop recurrent
+ * blocks and 0 otherwise.  Sliding-window layers receive only the positions
+ * their ring keeps.  Replaces the cache contents; a per_loop cache forgets
+ * its loop count.  Errors: DORY_ERR_ARG (n_ctx > max_ctx), DORY_ERR_CUDA. */
+int dory_cache_fill_synthetic(dory_model* m, dory_cache* c, int n_ctx,
+                              uint64_t seed, void* stream);
+
 /* Workspace bytes for calls of `batch` sequences x up to `max_chunk`
  * tokens.  The workspace holds activations only; its contents between
  * calls are meaningless except for dory_copy_state(). */

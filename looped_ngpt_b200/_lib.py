@@ -48,6 +48,7 @@ SIGNATURES = {
                                    c_int, _P, POINTER(c_void_p)]),
     "dory_cache_length": (c_int, [_P, POINTER(c_int)]),
     "dory_cache_reset": (c_int, [_P, _P]),
+    "dory_cache_fill_synthetic": (c_int, [_P, _P, c_int, ctypes.c_uint64, _P]),
     "dory_workspace_bytes": (c_int, [_P, c_int, c_int, _I64P]),
     "dory_prefill": (c_int, [_P, _P, _P, c_int, c_int, c_int, c_int, c_int,
                              _P, _P, _P, c_int64, _P]),

@@ -898,3 +898,36 @@ extern "C" int dory_debug_gemm_bf16(const void* d_A, int lda, const void* d_W,
                    nullptr, (cudaStream_t)stream);
   return cudaGetLastError() == cudaSuccess ? DORY_OK : DORY_ERR_CUDA;
 }
+
+extern "C" int dory_cache_fill_synthetic(dory_model* m, dory_cache* c,
+                                         int n_ctx, uint64_t seed,
+                                         void* stream) {
+  if (!m || !c || c->m != m || n_ctx < 0 || n_ctx > c->max_ctx)
+    return DORY_ERR_ARG;
+  const Dims& dm = m->dm;
+  const cudaStream_t st = (cudaStream_t)stream;
+  const CacheGeo geo{c->d_nctx, c->d_block_table, c->pages_per_seq,
+                     c->max_ctx};
+  const float ck = (float)std::sqrt(3.0 / dm.hd);
+  const float cv = (float)std::sqrt(3.0 / dm.d);
+  cudaGetLastError();
+  for (int i = 0; i < m->nblk; ++i) {
+    const int ns = slots_of(m, i, c->kv_mode, c->max_loops);
+    for (int s2 = 0; s2 < ns; ++s2) {
+      const KVSlot& kv = c->slots[c->slot_base[i] + s2];
+      // the generator's slot index: loop t (1-based) of a per_loop
+      // recurrent block, 0 for every single-slot block
+      const int gslot = (ns > 1 || (is_rec(m, i) &&
+                                     c->kv_mode == DORY_KV_PER_LOOP))
+                            ? s2 + 1 : 0;
+      const int lo = kv.ring ? std::max(0, n_ctx - kv.cap) : 0;
+      launch_fill_kv(kv, geo, c->B, dm.Hkv, dm.hd, lo, n_ctx, i, gslot, seed,
+                     ck, cv, st);
+    }
+  }
+  launch_set_nctx(c->d_nctx, n_ctx, st);
+  if (cudaGetLastError() != cudaSuccess) return DORY_ERR_CUDA;
+  c->n_ctx = n_ctx;
+  c->loops_bound = 0;
+  return DORY_OK;
+}

@@ -133,6 +133,11 @@ void launch_argmax_partials(const float* val, const int* idx, int B, int n,
 void launch_argmax_rows(const float* logits, int rows, int V, int* out,
                         cudaStream_t st);
 void launch_advance(int* n_ctx, int T, cudaStream_t st);
+void launch_set_nctx(int* n_ctx, int v, cudaStream_t st);
+// Seeded synthetic K/V entries (SplitMix64 counter generator).
+void launch_fill_kv(const KVSlot& kv, const CacheGeo& g, int B, int Hkv,
+                    int hd, int p_lo, int p_hi, int block, int slot,
+                    uint64_t seed, float ck, float cv, cudaStream_t st);
 void launch_cache_init(int* n_ctx, int* block_table, int B, int pages_per_seq,
                        cudaStream_t st);
 

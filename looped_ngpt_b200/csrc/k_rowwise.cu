@@ -138,6 +138,49 @@ __global__ void argmax_rows_kernel(const float* z, int V, int* out) {
   block_argmax(v, i, out + r);
 }
 
+// SplitMix64 output function (Steele, Lea and Flood, 2014).
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Seeded synthetic cache entries for positions [p_lo, p_hi) of one slot:
+// entry (kind, block, slot, b, kvh, pos, j) is the SplitMix64 counter
+// generator's uniform u scaled to (2u - 1) * c_kind and rounded to bf16.
+__global__ void fill_kv_kernel(KVSlot kv, CacheGeo g, int B, int Hkv, int hd,
+                               int p_lo, int p_hi, int block, int slot,
+                               uint64_t seed, float ck, float cv) {
+  const int np = p_hi - p_lo;
+  const long total = (long)B * Hkv * np * hd;
+  for (long id = blockIdx.x * (long)blockDim.x + threadIdx.x; id < total;
+       id += (long)gridDim.x * blockDim.x) {
+    const int j = (int)(id % hd);
+    long r = id / hd;
+    const int pos = p_lo + (int)(r % np);
+    r /= np;
+    const int kvh = (int)(r % Hkv), b = (int)(r / Hkv);
+    const size_t off = kv_index(kv, g, Hkv, hd, b, kvh, pos) + j;
+#pragma unroll
+    for (int kind = 0; kind < 2; ++kind) {
+      uint64_t c = (uint64_t)kind;
+      c = c * 64 + (uint64_t)block;
+      c = c * 8 + (uint64_t)slot;
+      c = c * 4096 + (uint64_t)b;
+      c = c * 64 + (uint64_t)kvh;
+      c = c * (1ull << 20) + (uint64_t)pos;
+      c = c * 512 + (uint64_t)j;
+      const uint64_t z = splitmix64(seed + c);
+      const float u = __fmul_rn((float)(z >> 40), 0x1p-24f);
+      const float x = __fmul_rn(__fsub_rn(__fmul_rn(2.f, u), 1.f), kind ? cv : ck);
+      (kind ? kv.V : kv.K)[off] = __float2bfloat16_rn(x);
+    }
+  }
+}
+
+__global__ void set_nctx_kernel(int* n_ctx, int v) { *n_ctx = v; }
+
 __global__ void advance_kernel(int* n_ctx, int T) {
   pdl_wait();
   pdl_trigger();
@@ -185,6 +228,18 @@ void launch_argmax_partials(const float* val, const int* idx, int B, int n,
 void launch_argmax_rows(const float* logits, int rows, int V, int* out,
                         cudaStream_t st) {
   launch_k(argmax_rows_kernel, dim3(rows), dim3(256), 0, st, logits, V, out);
+}
+
+void launch_fill_kv(const KVSlot& kv, const CacheGeo& g, int B, int Hkv,
+                    int hd, int p_lo, int p_hi, int block, int slot,
+                    uint64_t seed, float ck, float cv, cudaStream_t st) {
+  if (p_hi <= p_lo) return;
+  fill_kv_kernel<<<148 * 8, 256, 0, st>>>(kv, g, B, Hkv, hd, p_lo, p_hi, block,
+                                          slot, seed, ck, cv);
+}
+
+void launch_set_nctx(int* n_ctx, int v, cudaStream_t st) {
+  set_nctx_kernel<<<1, 1, 0, st>>>(n_ctx, v);
 }
 
 void launch_advance(int* n_ctx, int T, cudaStream_t st) {

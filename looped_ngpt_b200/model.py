@@ -58,6 +58,13 @@ class KVCache:
               _lib.load().dory_cache_length(self.handle, ctypes.byref(n)))
         return n.value
 
+    def fill_synthetic(self, n_ctx, seed=2, stream=None):
+        """dory_cache_fill_synthetic: n_ctx seeded synthetic tokens per row."""
+        check("dory_cache_fill_synthetic",
+              _lib.load().dory_cache_fill_synthetic(
+                  self.model.handle, self.handle, n_ctx, seed,
+                  _stream_ptr(stream)))
+
     def reset(self, stream=None):
         check("dory_cache_reset",
               _lib.load().dory_cache_reset(self.handle, _stream_ptr(stream)))
