@@ -42,6 +42,9 @@ def parse():
     ap.add_argument("--kv-mode", default="last_loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prompt", type=int, default=PROMPT)
+    ap.add_argument("--no-long", action="store_true",
+                    help="skip the long-context batched-decode workloads")
+    ap.add_argument("--long-steps", type=int, default=8)
     ap.add_argument("--profile-decode", type=int, default=0, metavar="K",
                     help="only: prefill, warm up, then one decode step at "
                          "k=K inside the NVTX range 'decode_step' (for ncu)")
@@ -274,8 +277,55 @@ def run_gpu(args, rank, world, local):
         host_tok.copy_(host_out)
     e2e_dt = time.perf_counter() - t0
     barrier(world)
+    if not args.no_long:
+        del cache, headline["cache"]
+        torch.cuda.empty_cache()
+        out["long_context"] = run_long(gm, args, hbm_peak, dev)
     return dict(out=out, headline=headline, e2e_dt=e2e_dt, w=w,
                 hbm_peak=hbm_peak, tc_peak=tc_peak, peak_kind=peak_kind)
+
+
+def run_long(gm, args, hbm_peak, dev):
+    """Decode over seeded synthetic cached context: B=64 x 32768 tokens at
+    k=2 in both KV modes, and B=4 x 131072 tokens at k=2, last_loop."""
+    import torch
+    res = {}
+    K, W = args.long_steps, 2
+    for name, B, ctx, k, mode in (("b64_ctx32k_k2_per_loop", 64, 32768, 2, "per_loop"),
+                                   ("b64_ctx32k_k2_last_loop", 64, 32768, 2, "last_loop"),
+                                   ("b4_ctx131k_k2_last_loop", 4, 131072, 2, "last_loop")):
+        cache = gm.new_cache(B, ctx + K + W + 8, 1, kv_mode=mode, max_loops=k)
+        cache.fill_synthetic(ctx, seed=2)
+        ws = gm.workspace(B, 1)
+        tok = torch.zeros(B, dtype=torch.int32, device=dev)
+        gm.decode_step(cache, tok, k, ws, want_logits=False)
+        tb = cache._dec_bufs[0]
+        for _ in range(W):
+            gm.decode_step(cache, tb, k, ws, argmax=tb, want_logits=False)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            gm.decode_step(cache, tb, k, ws, argmax=tb, want_logits=False)
+        e1.record()
+        torch.cuda.synchronize()
+        dt = e0.elapsed_time(e1) / 1e3
+        gm.profile(True)
+        gm.decode_step(cache, tb, k, ws, argmax=tb, want_logits=False)
+        st = gm.profile_read()
+        gm.profile(False)
+        assert gm.sync_status() == 0, "device-side check failed"
+        step_bytes = sum(v["bytes"] for v in st.values())
+        res[name] = {"tok_s": B * K / dt, "ms_per_step": dt / K * 1e3,
+                     "kv_cache_gb": cache.nbytes / 1e9,
+                     "bytes_per_step_gb": step_bytes / 1e9,
+                     "hbm_frac": step_bytes * K / dt / (hbm_peak * 1e9),
+                     "kernels_us": {n: round(v["ms"] * 1e3, 1)
+                                    for n, v in sorted(st.items(),
+                                                       key=lambda kv: -kv[1]["ms"])}}
+        del cache, ws
+        torch.cuda.empty_cache()
+    return res
 
 
 def profile_run(args):
