@@ -140,7 +140,7 @@ CacheLayout cache_layout(const dory_model* m, int B, int max_ctx,
 
 
 struct WS {
-  float *s0, *s1, *sfin, *x, *qkvg, *gate, *h, *part_o, *part_ml,
+  float *s0, *s1, *sfin, *x, *qkvg, *gate, *h, *part_o, *part_ml, *lg,
       *rope, *amax_val;
   bf16 *s_bf, *a, *mact, *qb;
   int* amax_idx;
@@ -178,6 +178,7 @@ WS ws_layout(const dory_model* m, int B, int T, char* base) {
   w.amax_val = (float*)take((size_t)B * kArgmaxSlots * 4);
   w.amax_idx = (int*)take((size_t)B * kArgmaxSlots * 4);
   w.counters = (int*)take((size_t)B * dm.Hkv * 4);
+  w.lg = (float*)take(B > 8 ? (size_t)B * dm.V * 4 : 0);
   w.total = off;
   return w;
 }
@@ -695,6 +696,16 @@ void enqueue_forward(const CallCtx& x) {
       if (x.argmax) {
         Prof p(m, x.st, "argmax", (double)x.M * dm.V * 4, 0);
         launch_argmax_rows(x.logits, x.M, dm.V, x.argmax, x.st);
+      }
+    } else if (x.B > 8) {
+      // last token of every sequence (rows b*T + T-1, stride T*d) through
+      // the tensor-core GEMM: the 671 MB head is read once, not B/8 times
+      float* lg = x.logits ? x.logits : w.lg;
+      gemm_run(m, w.s_bf + (size_t)(x.T - 1) * dm.d, x.T * dm.d, m->lm_head, lg,
+               dm.V, x.B, dm.V, dm.d, m->s_z, x.st, "gemm_lmhead");
+      if (x.argmax) {
+        Prof p(m, x.st, "argmax", (double)x.B * dm.V * 4, 0);
+        launch_argmax_rows(lg, x.B, dm.V, x.argmax, x.st);
       }
     } else {
       for (int b0 = 0; b0 < x.B; b0 += 8) {

@@ -143,8 +143,8 @@ __global__ void __launch_bounds__(2 * HD) attn_decode_fused_kernel(const DecAttn
   constexpr int PVS = (4 * G * HD > G * (2 * kMaxSplits + HD))
                           ? 4 * G * HD : G * (2 * kMaxSplits + HD);
   // splits staged per merge round trip: as many as fit in the K/V tiles
-  constexpr int CHF = (2 * TK * (HD + KPAD) * 2) / (G * HD * 4);
-  constexpr int CH = CHF < 16 ? CHF : 16;
+  constexpr int CHF = (4 * TK * (HD + KPAD) * 2) / (G * HD * 4);
+  constexpr int CH = CHF < 32 ? CHF : 32;
   static_assert(CH >= 1, "merge staging buffer must fit in the K/V tiles");
   extern __shared__ float sm[];
   const Dims& dm = a.dm;
@@ -157,8 +157,9 @@ __global__ void __launch_bounds__(2 * HD) attn_decode_fused_kernel(const DecAttn
   float* sc_s = vn_s + HD;                           // [NQ][G][TK] scores / [G][TK] probs
   float* st = sc_s + NQ * G * TK;                    // m, l, corr: [3][G] (+pad)
   float* pv_s = st + 32;                             // [4][G][HD] P.V partials
-  bf16* K_s = reinterpret_cast<bf16*>(pv_s + PVS);   // [TK][RP]
-  bf16* V_s = K_s + TK * RP;
+  bf16* Kb = reinterpret_cast<bf16*>(pv_s + PVS);    // [2][TK][RP]
+  bf16* Vb = Kb + 2 * TK * RP;                       // [2][TK][RP]
+  bf16* K_s = Kb;                                    // merge staging base
   __shared__ int s_last;
 
   const int p = *a.g.n_ctx;
@@ -167,7 +168,7 @@ __global__ void __launch_bounds__(2 * HD) attn_decode_fused_kernel(const DecAttn
   const int k_begin = sp.lo + split * sp.chunk;
   const int k_end = min(sp.hi, k_begin + sp.chunk);
   if (active)
-    issue_kv_tile<HD>(K_s, V_s, a.kv, a.g, dm.Hkv, b, kvh, k_begin,
+    issue_kv_tile<HD>(Kb, Vb, a.kv, a.g, dm.Hkv, b, kvh, k_begin,
                       min(TK, k_end - k_begin), p, NT);
   asm volatile("cp.async.commit_group;" ::: "memory");
   pdl_wait();
@@ -215,20 +216,26 @@ __global__ void __launch_bounds__(2 * HD) attn_decode_fused_kernel(const DecAttn
 #pragma unroll
   for (int g = 0; g < G; ++g) acc[g][0] = acc[g][1] = 0.f;
   const int dp = tid % HP, kg = tid / HP;            // P.V: dim pair, key group
-  for (int j0 = k_begin; j0 < k_end; j0 += TK) {
+  // tiles are double-buffered: tile it + 1 is in flight while tile it is
+  // consumed, tile it + 2 is issued once tile it's buffer is free
+  if (k_begin + TK < k_end) {
+    issue_kv_tile<HD>(Kb + TK * RP, Vb + TK * RP, a.kv, a.g, dm.Hkv, b, kvh,
+                      k_begin + TK, min(TK, k_end - k_begin - TK), p, NT);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  int it = 0;
+  for (int j0 = k_begin; j0 < k_end; j0 += TK, ++it) {
     const int nk = min(TK, k_end - j0);
-    if (j0 != k_begin) {
-      __syncthreads();                               // previous tile consumed
-      issue_kv_tile<HD>(K_s, V_s, a.kv, a.g, dm.Hkv, b, kvh, j0, nk, p, NT);
-      asm volatile("cp.async.commit_group;" ::: "memory");
-    }
+    bf16* K_s = Kb + (it & 1) * TK * RP;
+    bf16* V_s = Vb + (it & 1) * TK * RP;
     if (p >= j0 && p < j0 + nk) {                    // current token's row
       for (int c = tid; c < HD; c += NT) {
         K_s[(p - j0) * RP + c] = __float2bfloat16_rn(kn_s[c]);
         V_s[(p - j0) * RP + c] = __float2bfloat16_rn(vn_s[c]);
       }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (j0 + TK < k_end) asm volatile("cp.async.wait_group 1;" ::: "memory");
+    else asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
     {   // scores: thread -> (key j, 32-dim part qp)
       const int j = tid % TK, qp = tid / TK;
@@ -304,6 +311,12 @@ __global__ void __launch_bounds__(2 * HD) attn_decode_fused_kernel(const DecAttn
           acc[g][1] = fmaf(pg, v.y, acc[g][1]);
         }
       }
+    }
+    if (j0 + 2 * TK < k_end) {
+      __syncthreads();                               // tile it's buffer is free
+      issue_kv_tile<HD>(K_s, V_s, a.kv, a.g, dm.Hkv, b, kvh, j0 + 2 * TK,
+                        min(TK, k_end - j0 - 2 * TK), p, NT);
+      asm volatile("cp.async.commit_group;" ::: "memory");
     }
   }
 #pragma unroll
@@ -643,7 +656,7 @@ void launch_dec_t(const DecAttnArgs& a, cudaStream_t st) {
                           ? 4 * G * HD : G * (2 * kMaxSplits + HD);
   const size_t smem = (G * HD + 2 * HD + NQ * G * TK + 32 + PVS) *
                           sizeof(float) +
-                      2 * TK * (HD + KPAD) * sizeof(bf16);
+                      4 * TK * (HD + KPAD) * sizeof(bf16);
   static bool configured = false;
   if (!configured) {
     cudaFuncSetAttribute(attn_decode_fused_kernel<HD, G>,

@@ -7,6 +7,7 @@ import pytest
 import torch
 
 from synthetic import TINY, make_weights, make_prompt
+from oracle.model import Model
 from tests.gpu_util import (oracle_run, gpu_run, compare, NORM_TOL, TOP1_MIN)
 
 pytestmark = pytest.mark.gpu
@@ -120,3 +121,29 @@ def test_pooled_top1_agreement(tiny):
     gp, _, _, _, _, _ = gpu_run(gm, prompt, 2, "last_loop", np.zeros((0, 4), np.int32))
     _, agree, n = compare(gp, zp, "pooled")
     assert agree / n >= TOP1_MIN, f"top-1 agreement {agree}/{n}"
+
+
+@pytest.mark.parametrize("kv_mode", ["per_loop", "last_loop"])
+def test_batch_over_8_uses_gemm_paths(tiny, kv_mode):
+    """B=10: the decode step and the last-token LM head run on the
+    tensor-core GEMM instead of the GEMV; 20-token prompt (last-token
+    logits only), then 3 teacher-forced decode steps at k=2."""
+    w, gm = tiny
+    B = 10
+    prompt = make_prompt(TINY, B, 20, seed=9)
+    ref = Model(TINY, w, batch=B, kv_mode=kv_mode)
+    zr = [ref.forward(prompt, 2)[:, 0]]
+    cache = gm.new_cache(B, 32, 20, kv_mode=kv_mode, max_loops=2)
+    ws = gm.workspace(B, 20)
+    z, a = gm.prefill(cache, torch.from_numpy(prompt).cuda(), 2, ws)
+    zg = [z.cpu().numpy().copy()]
+    assert np.array_equal(a.cpu().numpy(), np.argmax(zg[0], -1))
+    tok = np.argmax(zr[0], -1)
+    for _ in range(3):
+        zr.append(ref.decode_step(tok, 2))
+        g, _ = gm.decode_step(cache, torch.from_numpy(tok.astype(np.int32)).cuda(),
+                              2, ws)
+        zg.append(g.cpu().numpy().copy())
+        tok = np.argmax(zr[-1], -1)
+    assert gm.sync_status() == 0
+    compare(np.array(zg), np.array(zr), f"B=10 {kv_mode}")
