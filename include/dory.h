@@ -68,7 +68,19 @@ typedef struct {
   int wfmt;                   /* dory_wfmt of the block projections      */
 } dory_config;
 
-/* One named weight tensor in device memory (non-owning).  Names and shapes
+/* Quantised checkpoints (wfmt = DORY_W_MXFP8 / DORY_W_NVFP4; MXFP8 explainer
+ * page, deployment section: W8A16, group 32; paper summary, 前置知识: NVFP4 =
+ * E2M1 values with E4M3 scales): each block projection "blk<i>.<w>" is
+ * replaced by
+ *   "blk<i>.<w>.q"  uint8 codes: MXFP8 E4M3 [N, K]; NVFP4 E2M1 pairs
+ *                   [N, K/2] (element 2j in bits 0-3, 2j+1 in bits 4-7)
+ *   "blk<i>.<w>.s"  uint8 scales: MXFP8 E8M0 [N, K/32]; NVFP4 E4M3 [N, K/16]
+ *   "blk<i>.<w>.t"  f32 [1] per-tensor scale (NVFP4 only)
+ * with w = e4m3(q) * 2^(s - 127), or e2m1(q) * e4m3(s) * t.  Embedding and
+ * LM head stay BF16.  Quantised models run decode-style calls (T = 1,
+ * B <= 8); other calls return DORY_ERR_UNSUPPORTED.
+ *
+ * One named weight tensor in device memory (non-owning).  Names and shapes
  * (row-major, K = contraction axis last):
  *   "embed"  bf16 [vocab, d]       "lm_head" bf16 [vocab, d]
  *   "s_z"    f32  [vocab]
@@ -205,6 +217,15 @@ int dory_decode_step_static(dory_model* m, dory_cache* c,
  * waits are reported by dory_sync_status of any model). */
 int dory_debug_gemm_bf16(const void* d_A, int lda, const void* d_W,
                          float* d_C, int M, int N, int K, void* stream);
+
+/* Test access to the in-register weight decode of quantised models: write
+ * rows [row0, row0 + nrows) of block projection `tensor` (e.g.
+ * "blk3.w_gu") as f32 [nrows, K] to d_out: e4m3(q) * 2^(s - 127) (MXFP8) or
+ * e2m1(q) * e4m3(s) (NVFP4, without the tensor scale, which the GEMV applies
+ * to its sums).  Both products are exact in f32.  Errors: DORY_ERR_ARG,
+ * DORY_ERR_UNSUPPORTED (BF16 model). */
+int dory_debug_dequant(const dory_model* m, const char* tensor, int row0,
+                       int nrows, float* d_out, void* stream);
 
 /* Per-kernel timing (tracing aid).  While enabled, every call launches its
  * kernels eagerly (no graph replay), each bracketed by CUDA events on the

@@ -31,8 +31,17 @@ bool pdl_enabled() {
 
 namespace {
 
+// A block projection: BF16 rows, or quantised codes + scales (+ tensor scale).
+struct QMat {
+  const bf16* w = nullptr;
+  const uint8_t* q = nullptr;
+  const uint8_t* s = nullptr;
+  const float* t = nullptr;
+};
+
 struct BlockW {
   const bf16 *w_qkvg, *w_o, *w_gu, *w_down;
+  QMat m_qkvg, m_o, m_gu, m_down;
   const float *s_q, *s_k, *alpha_a, *alpha_m;
 };
 
@@ -50,6 +59,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct dory_model {
   Dims dm;
+  int wfmt = DORY_W_BF16;
   int n_in, n_rec, n_out, nblk;
   std::vector<uint8_t> ltype;
   double th_swa, th_full;
@@ -255,7 +265,9 @@ int dory_init_weights(const dory_config* cfg, const dory_tensor* tensors,
   if (!(cfg->rope_theta_swa > 1.0) || !(cfg->rope_theta_full > 1.0))
     return DORY_ERR_ARG;
   if (Hq % Hkv) return DORY_ERR_ARG;
-  if (cfg->wfmt != DORY_W_BF16) return DORY_ERR_UNSUPPORTED;
+  if (cfg->wfmt != DORY_W_BF16 && cfg->wfmt != DORY_W_MXFP8 &&
+      cfg->wfmt != DORY_W_NVFP4)
+    return DORY_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
   if (!(hd == 64 || hd == 128 || hd == 160) ||
       !(G == 1 || G == 2 || G == 4 || G == 8) || G * hd > 1024)
@@ -277,6 +289,7 @@ int dory_init_weights(const dory_config* cfg, const dory_tensor* tensors,
     if (t > 1) { delete m; return DORY_ERR_ARG; }
   m->th_swa = cfg->rope_theta_swa;
   m->th_full = cfg->rope_theta_full;
+  m->wfmt = cfg->wfmt;
 
   std::map<std::string, std::pair<const void*, int64_t>> tab;
   for (int i = 0; i < n_tensors; ++i) {
@@ -299,17 +312,36 @@ int dory_init_weights(const dory_config* cfg, const dory_tensor* tensors,
   m->embed = (const bf16*)get("embed", (int64_t)V * d * 2);
   m->lm_head = (const bf16*)get("lm_head", (int64_t)V * d * 2);
   m->s_z = (const float*)get("s_z", (int64_t)V * 4);
+  // block projections: BF16 `name`, or `name.q` / `name.s` (/ `name.t`)
+  auto mat = [&](const std::string& n, int64_t N, int64_t K) {
+    QMat q;
+    if (cfg->wfmt == DORY_W_BF16) {
+      q.w = (const bf16*)get(n, N * K * 2);
+    } else if (cfg->wfmt == DORY_W_MXFP8) {
+      q.q = (const uint8_t*)get(n + ".q", N * K);
+      q.s = (const uint8_t*)get(n + ".s", N * K / 32);
+    } else {
+      q.q = (const uint8_t*)get(n + ".q", N * K / 2);
+      q.s = (const uint8_t*)get(n + ".s", N * K / 16);
+      q.t = (const float*)get(n + ".t", 4);
+    }
+    return q;
+  };
   m->blk.resize(m->nblk);
   for (int i = 0; i < m->nblk; ++i) {
     const std::string p = "blk" + std::to_string(i) + ".";
     BlockW& b = m->blk[i];
-    b.w_qkvg = (const bf16*)get(p + "w_qkvg", (int64_t)rows * d * 2);
+    b.m_qkvg = mat(p + "w_qkvg", rows, d);
+    b.m_o = mat(p + "w_o", d, (int64_t)Hq * hd);
+    b.m_gu = mat(p + "w_gu", 2 * (int64_t)F, d);
+    b.m_down = mat(p + "w_down", d, F);
+    b.w_qkvg = b.m_qkvg.w;
+    b.w_o = b.m_o.w;
+    b.w_gu = b.m_gu.w;
+    b.w_down = b.m_down.w;
     b.s_q = (const float*)get(p + "s_q", (int64_t)Hq * hd * 4);
     b.s_k = (const float*)get(p + "s_k", (int64_t)Hkv * hd * 4);
-    b.w_o = (const bf16*)get(p + "w_o", (int64_t)d * Hq * hd * 2);
     b.alpha_a = (const float*)get(p + "alpha_a", (int64_t)d * 4);
-    b.w_gu = (const bf16*)get(p + "w_gu", (int64_t)2 * F * d * 2);
-    b.w_down = (const bf16*)get(p + "w_down", (int64_t)d * F * 2);
     b.alpha_m = (const float*)get(p + "alpha_m", (int64_t)d * 4);
   }
   if (!ok) { delete m; return DORY_ERR_ARG; }
@@ -459,7 +491,10 @@ struct Prof {
 };
 
 double gemv_bytes(const GemvArgs& g, int rows) {
-  const double w = (double)rows * g.K * 2;
+  // weight bytes per element: BF16 2, MXFP8 1 + 1/32, NVFP4 1/2 + 1/16
+  const double per = g.fmt == WF_MXFP8 ? 1.0 + 1.0 / 32
+                     : g.fmt == WF_NVFP4 ? 0.5 + 1.0 / 16 : 2.0;
+  const double w = (double)rows * g.K * per;
   const double in = g.pro == PRO_UPDATE ? (double)g.B * g.K * 4 * (3 + g.h_S)
                                         : (double)g.B * g.K * 2;
   double out;
@@ -471,9 +506,16 @@ double gemv_bytes(const GemvArgs& g, int rows) {
 
 // Launches the GEMV; returns the number of K segments (partials) it writes.
 int gemv_run(dory_model* m, const GemvArgs& g0, cudaStream_t st,
-             const char* name) {
+             const char* name, const QMat* qm = nullptr) {
   GemvArgs g = g0;
   g.err = m->d_status;
+  g.fmt = WF_BF16;
+  if (qm && !qm->w) {
+    g.fmt = m->wfmt == DORY_W_MXFP8 ? WF_MXFP8 : WF_NVFP4;
+    g.Wq = qm->q;
+    g.Ws = qm->s;
+    g.Wt = qm->t;
+  }
   g.S = gemv_splits(g);
   const int grid = gemv_grid(g, m->num_sms);
   const int rows = g.epi == EPI_SWIGLU ? 2 * g.n_items : g.n_items;
@@ -564,7 +606,7 @@ void enqueue_forward(const CallCtx& x) {
         g.alpha = prev_alpha; g.s_out = other; g.reinject = rj; g.x_buf = w.x;
         std::swap(cur, other);
       }
-      S_qkvg = gemv_run(m, g, x.st, "gemv_qkvg");
+      S_qkvg = gemv_run(m, g, x.st, "gemv_qkvg", &bw.m_qkvg);
     } else {
       if (k > 0) {
         Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
@@ -625,7 +667,7 @@ void enqueue_forward(const CallCtx& x) {
       g.W = bw.w_o; g.K = dm.qdim; g.n_items = dm.d; g.B = x.B; g.epi = EPI_F32;
       g.out = w.h;
       g.pro = PRO_BF16; g.xin = w.a; g.xin_stride = dm.qdim;
-      S_o = gemv_run(m, g, x.st, "gemv_o");
+      S_o = gemv_run(m, g, x.st, "gemv_o", &bw.m_o);
     } else {
       gemm_run(m, w.a, dm.qdim, bw.w_o, w.h, dm.d, x.M, dm.d, dm.qdim, nullptr,
                x.st, "gemm_o");
@@ -639,12 +681,12 @@ void enqueue_forward(const CallCtx& x) {
       g.pro = PRO_UPDATE; g.s_in = cur; g.h_in = w.h; g.h_S = S_o;
       g.alpha = bw.alpha_a; g.s_out = other; g.reinject = RJ_NONE; g.x_buf = w.x;
       std::swap(cur, other);
-      gemv_run(m, g, x.st, "gemv_gateup");
+      gemv_run(m, g, x.st, "gemv_gateup", &bw.m_gu);
       GemvArgs g2{};
       g2.W = bw.w_down; g2.K = dm.F; g2.n_items = dm.d; g2.B = x.B;
       g2.epi = EPI_F32; g2.out = w.h;
       g2.pro = PRO_BF16; g2.xin = w.mact; g2.xin_stride = dm.F;
-      prev_S = gemv_run(m, g2, x.st, "gemv_down");
+      prev_S = gemv_run(m, g2, x.st, "gemv_down", &bw.m_down);
     } else {
       {
         Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
@@ -744,6 +786,8 @@ int run_call(dory_model* m, dory_cache* c, const int32_t* tokens, int B,
       (n_loops > c->max_loops || (c->loops_bound && c->loops_bound != n_loops)))
     return DORY_ERR_CACHE;
   if ((int64_t)c->n_ctx + T > c->max_ctx) return DORY_ERR_CACHE;
+  // quantised weights: decode-style calls only (one token, B <= 8)
+  if (m->wfmt != DORY_W_BF16 && !use_gemv(B, T)) return DORY_ERR_UNSUPPORTED;
   const WS w = ws_layout(m, B, T, (char*)ws);
   if ((int64_t)w.total > ws_bytes) return DORY_ERR_WORKSPACE;
   CallCtx x{m, c, w, B, T, B * T, n_loops, logits_all, c->n_ctx, tokens,
@@ -941,4 +985,33 @@ extern "C" int dory_cache_fill_synthetic(dory_model* m, dory_cache* c,
   c->n_ctx = n_ctx;
   c->loops_bound = 0;
   return DORY_OK;
+}
+
+extern "C" int dory_debug_dequant(const dory_model* m, const char* tensor,
+                                  int row0, int nrows, float* d_out,
+                                  void* stream) {
+  if (!m || !tensor || !d_out || row0 < 0 || nrows < 1) return DORY_ERR_ARG;
+  if (m->wfmt == DORY_W_BF16) return DORY_ERR_UNSUPPORTED;
+  const std::string n = tensor;
+  const std::string pre = "blk";
+  if (n.compare(0, 3, pre) != 0) return DORY_ERR_ARG;
+  const size_t dot = n.find('.');
+  if (dot == std::string::npos) return DORY_ERR_ARG;
+  const int i = atoi(n.substr(3, dot - 3).c_str());
+  if (i < 0 || i >= m->nblk) return DORY_ERR_ARG;
+  const std::string leaf = n.substr(dot + 1);
+  const BlockW& b = m->blk[i];
+  const Dims& dm = m->dm;
+  const QMat* q = nullptr;
+  long N = 0, K = 0;
+  if (leaf == "w_qkvg") { q = &b.m_qkvg; N = dm.rows_qkvg; K = dm.d; }
+  else if (leaf == "w_o") { q = &b.m_o; N = dm.d; K = dm.qdim; }
+  else if (leaf == "w_gu") { q = &b.m_gu; N = 2L * dm.F; K = dm.d; }
+  else if (leaf == "w_down") { q = &b.m_down; N = dm.d; K = dm.F; }
+  else return DORY_ERR_ARG;
+  if ((long)row0 + nrows > N) return DORY_ERR_ARG;
+  cudaGetLastError();
+  launch_dequant_rows(m->wfmt == DORY_W_MXFP8 ? WF_MXFP8 : WF_NVFP4, q->q, q->s,
+                      (int)K, row0, nrows, d_out, (cudaStream_t)stream);
+  return cudaGetLastError() == cudaSuccess ? DORY_OK : DORY_ERR_CUDA;
 }

@@ -77,8 +77,14 @@ enum GemvPro : int { PRO_BF16 = 0, PRO_UPDATE = 1 };
 enum GemvEpi : int { EPI_F32 = 0, EPI_SWIGLU = 1, EPI_LMHEAD = 2 };
 enum Reinject : int { RJ_NONE = 0, RJ_FIRST = 1, RJ_NEXT = 2 };
 
+enum WFmt : int { WF_BF16 = 0, WF_MXFP8 = 1, WF_NVFP4 = 2 };
+
 struct GemvArgs {
-  const bf16* W;       // [N_rows, K] row-major
+  const bf16* W;       // [N_rows, K] row-major (WF_BF16)
+  int fmt;             // WFmt of W
+  const uint8_t* Wq;   // WF_MXFP8: E4M3 [N][K]; WF_NVFP4: E2M1 pairs [N][K/2]
+  const uint8_t* Ws;   // WF_MXFP8: E8M0 [N][K/32]; WF_NVFP4: E4M3 [N][K/16]
+  const float* Wt;     // WF_NVFP4: tensor scale [1]
   int K;               // contraction length (multiple of 256 * S)
   int n_items;         // output rows (EPI_SWIGLU: pairs n, n + pair_off)
   int S;               // split-K factor: set to gemv_splits(*this)
@@ -111,6 +117,12 @@ struct GemvArgs {
 int gemv_splits(const GemvArgs& a);
 int gemv_grid(const GemvArgs& a, int num_sms);
 void launch_gemv(const GemvArgs& a, int grid, cudaStream_t st);
+
+// Decode rows [row0, row0 + nrows) of a quantised matrix to f32 (the values
+// the GEMV multiplies: e4m3 * 2^(e8m0 - 127), or e2m1 * e4m3 without the
+// NVFP4 tensor scale).  out [nrows][K].
+void launch_dequant_rows(int fmt, const uint8_t* Wq, const uint8_t* Ws, int K,
+                         int row0, int nrows, float* out, cudaStream_t st);
 
 // ------------------------------------------------------------- rowwise ----
 // RoPE cos/sin for positions n_ctx + t, t < T; table [2][T][hd/2][2].

@@ -31,6 +31,8 @@
 // store, per-block greedy argmax partials).
 #include <cstdlib>
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace dory {
@@ -99,62 +101,124 @@ struct Plan {
   int NS;       // stages in the ring (8 items each)
 };
 
-// Dot products of one staged row segment (kl elements) with the NB
-// activation rows; returns the warp-reduced sums in every lane.
-template <int NB>
-__device__ __forceinline__ void row_slice_dot(const bf16* wrow, const bf16* xk,
-                                              int K, int kl, int lane,
-                                              float (&acc)[NB]) {
+// ---- quantised weights (MXFP8 / NVFP4): decode 8 weights of one lane ----
+__device__ __forceinline__ float2 half2_to_float2(uint32_t h) {
+  __half2 v = *reinterpret_cast<__half2*>(&h);
+  return __half22float2(v);
+}
+// E4M3 pair (low byte first) -> two floats, exact (via f16).
+__device__ __forceinline__ float2 e4m3x2_f2(uint16_t v) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
+  return half2_to_float2(h);
+}
+// E2M1 pair (low nibble first) -> two floats, exact (via f16).
+__device__ __forceinline__ float2 e2m1x2_f2(uint32_t byte) {
+  uint32_t h;
+  asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }"
+      : "=r"(h)
+      : "r"(byte));
+  return half2_to_float2(h);
+}
+// E8M0 scale 2^(e - 127); code 0 is 2^-127 (an f32 subnormal), 0xFF NaN.
+__device__ __forceinline__ float e8m0_f(uint32_t e) {
+  return e == 0 ? __uint_as_float(0x00400000u)
+                : (e == 255 ? __uint_as_float(0x7fc00000u) : __uint_as_float(e << 23));
+}
+__device__ __forceinline__ float e4m3_f(uint32_t b) {
+  return e4m3x2_f2((uint16_t)(b & 0xFF)).x;
+}
+
+// Bytes of one lane's 8 weights, and weights per scale.
+template <int FMT> struct FmtInfo;
+template <> struct FmtInfo<WF_BF16> { static constexpr int LB = 16, GROUP = 0; };
+template <> struct FmtInfo<WF_MXFP8> { static constexpr int LB = 8, GROUP = 32; };
+template <> struct FmtInfo<WF_NVFP4> { static constexpr int LB = 4, GROUP = 16; };
+
+template <int FMT>
+__device__ __forceinline__ void decode8(const uint8_t* p, float (&w)[8]) {
+  if (FMT == WF_BF16) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    w[0] = bf_lo(v.x); w[1] = bf_hi(v.x); w[2] = bf_lo(v.y); w[3] = bf_hi(v.y);
+    w[4] = bf_lo(v.z); w[5] = bf_hi(v.z); w[6] = bf_lo(v.w); w[7] = bf_hi(v.w);
+  } else if (FMT == WF_MXFP8) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    float2 f;
+    f = e4m3x2_f2((uint16_t)(v.x & 0xFFFF)); w[0] = f.x; w[1] = f.y;
+    f = e4m3x2_f2((uint16_t)(v.x >> 16)); w[2] = f.x; w[3] = f.y;
+    f = e4m3x2_f2((uint16_t)(v.y & 0xFFFF)); w[4] = f.x; w[5] = f.y;
+    f = e4m3x2_f2((uint16_t)(v.y >> 16)); w[6] = f.x; w[7] = f.y;
+  } else {
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
+    float2 f;
+    f = e2m1x2_f2(v & 0xFF); w[0] = f.x; w[1] = f.y;
+    f = e2m1x2_f2((v >> 8) & 0xFF); w[2] = f.x; w[3] = f.y;
+    f = e2m1x2_f2((v >> 16) & 0xFF); w[4] = f.x; w[5] = f.y;
+    f = e2m1x2_f2(v >> 24); w[6] = f.x; w[7] = f.y;
+  }
+}
+
+// Scale of the group holding element k of row `row` (1.f for BF16).
+template <int FMT>
+__device__ __forceinline__ float group_scale(const uint8_t* Ws, int K, long row,
+                                             int k) {
+  if (FMT == WF_MXFP8) return e8m0_f(__ldg(Ws + row * (K / 32) + k / 32));
+  if (FMT == WF_NVFP4) return e4m3_f(__ldg(Ws + row * (K / 16) + k / 16));
+  return 1.f;
+}
+
+// One staged row segment (item) times the register-resident x slice
+// (batch 1).  Lane covers elements c * 256 + lane * 8 + [0, 8), c < nc; its
+// 8 weights share one group scale (groups of 32 / 16 elements).
+template <int FMT, int MAXC>
+__device__ __forceinline__ float row_dot_reg_q(const uint8_t* wb, const float* xr,
+                                               const float* scl, int nc,
+                                               int lane) {
+  constexpr int LB = FmtInfo<FMT>::LB;
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    if (c < nc) {
+      float w[8];
+      decode8<FMT>(wb + (c * 32 + lane) * LB, w);
+      float t0 = w[0] * xr[c * 8 + 0], t1 = w[1] * xr[c * 8 + 1];
+      t0 = fmaf(w[2], xr[c * 8 + 2], t0); t1 = fmaf(w[3], xr[c * 8 + 3], t1);
+      t0 = fmaf(w[4], xr[c * 8 + 4], t0); t1 = fmaf(w[5], xr[c * 8 + 5], t1);
+      t0 = fmaf(w[6], xr[c * 8 + 6], t0); t1 = fmaf(w[7], xr[c * 8 + 7], t1);
+      if (FMT == WF_BF16) { a0 += t0; a1 += t1; }
+      else { a0 = fmaf(t0, scl[c], a0); a1 = fmaf(t1, scl[c], a1); }
+    }
+  }
+  return warp_sum(a0 + a1);
+}
+
+// Batched variant: x from shared memory (bf16 [NB][K], slice at xk).
+template <int FMT, int NB, int MAXC>
+__device__ __forceinline__ void row_dot_smem_q(const uint8_t* wb, const bf16* xk,
+                                               int K, const float* scl, int nc,
+                                               int lane, float (&acc)[NB]) {
+  constexpr int LB = FmtInfo<FMT>::LB;
 #pragma unroll
   for (int b = 0; b < NB; ++b) acc[b] = 0.f;
-#pragma unroll 5
-  for (int k = lane * 8; k < kl; k += 256) {
-    const uint4 wv = *reinterpret_cast<const uint4*>(wrow + k);
-    const float w0 = bf_lo(wv.x), w1 = bf_hi(wv.x), w2 = bf_lo(wv.y),
-                w3 = bf_hi(wv.y), w4 = bf_lo(wv.z), w5 = bf_hi(wv.z),
-                w6 = bf_lo(wv.w), w7 = bf_hi(wv.w);
 #pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      const uint4 xv = *reinterpret_cast<const uint4*>(xk + b * K + k);
-      float t = acc[b];
-      t = fmaf(w0, bf_lo(xv.x), t);
-      t = fmaf(w1, bf_hi(xv.x), t);
-      t = fmaf(w2, bf_lo(xv.y), t);
-      t = fmaf(w3, bf_hi(xv.y), t);
-      t = fmaf(w4, bf_lo(xv.z), t);
-      t = fmaf(w5, bf_hi(xv.z), t);
-      t = fmaf(w6, bf_lo(xv.w), t);
-      t = fmaf(w7, bf_hi(xv.w), t);
-      acc[b] = t;
+  for (int c = 0; c < MAXC; ++c) {
+    if (c < nc) {
+      float w[8];
+      decode8<FMT>(wb + (c * 32 + lane) * LB, w);
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const uint4 xv = *reinterpret_cast<const uint4*>(xk + b * K + c * 256 + lane * 8);
+        float t = w[0] * bf_lo(xv.x);
+        t = fmaf(w[1], bf_hi(xv.x), t); t = fmaf(w[2], bf_lo(xv.y), t);
+        t = fmaf(w[3], bf_hi(xv.y), t); t = fmaf(w[4], bf_lo(xv.z), t);
+        t = fmaf(w[5], bf_hi(xv.z), t); t = fmaf(w[6], bf_lo(xv.w), t);
+        t = fmaf(w[7], bf_hi(xv.w), t);
+        acc[b] = FMT == WF_BF16 ? acc[b] + t : fmaf(t, scl[c], acc[b]);
+      }
     }
   }
 #pragma unroll
   for (int b = 0; b < NB; ++b) acc[b] = warp_sum(acc[b]);
-}
-
-// One staged row segment times the register-resident x slice (batch 1):
-// lane covers elements c * 256 + lane * 8 + [0, 8) for c < nc.  Two
-// accumulators break the FMA dependency chain.
-template <int MAXC>
-__device__ __forceinline__ float row_dot_reg(const bf16* wrow, const float* xr,
-                                             int nc, int lane) {
-  float a0 = 0.f, a1 = 0.f;
-  const bf16* wp = wrow + lane * 8;
-#pragma unroll
-  for (int c = 0; c < MAXC; ++c) {
-    if (c < nc) {
-      const uint4 wv = *reinterpret_cast<const uint4*>(wp + c * 256);
-      a0 = fmaf(bf_lo(wv.x), xr[c * 8 + 0], a0);
-      a1 = fmaf(bf_hi(wv.x), xr[c * 8 + 1], a1);
-      a0 = fmaf(bf_lo(wv.y), xr[c * 8 + 2], a0);
-      a1 = fmaf(bf_hi(wv.y), xr[c * 8 + 3], a1);
-      a0 = fmaf(bf_lo(wv.z), xr[c * 8 + 4], a0);
-      a1 = fmaf(bf_hi(wv.z), xr[c * 8 + 5], a1);
-      a0 = fmaf(bf_lo(wv.w), xr[c * 8 + 6], a0);
-      a1 = fmaf(bf_hi(wv.w), xr[c * 8 + 7], a1);
-    }
-  }
-  return warp_sum(a0 + a1);
 }
 
 // Activation vector(s) for the GEMV -> shared memory as bf16: a copy of the
@@ -195,14 +259,15 @@ __device__ __forceinline__ void gemv_prologue(const GemvArgs& a, bf16* xs,
 }
 
 
-template <int NB, int EPI>
+template <int NB, int EPI, int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemv_kernel(const GemvArgs a, const Plan pl) {
   constexpr int R = (EPI == EPI_SWIGLU) ? 2 : 1;
+  constexpr int LB = FmtInfo<FMT>::LB;       // bytes per 8 weights
   extern __shared__ __align__(128) uint8_t smem[];
   const int K = a.K, S = pl.S, NS = pl.NS;
   const int seg = K / S;
-  const size_t item_bytes = (size_t)seg * sizeof(bf16);
+  const size_t item_bytes = (size_t)seg / 8 * LB;
   const size_t stage_bytes = (size_t)kWarps * R * item_bytes;
   uint8_t* ring = smem;                                         // NS stages
   bf16* xs = reinterpret_cast<bf16*>(ring + NS * stage_bytes);  // [NB][K]
@@ -230,7 +295,8 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
     const uint32_t bytes = (uint32_t)(cnt * item_bytes);
     uint64_t* bar = full + (s % NS);
     uint8_t* dst = ring + (s % NS) * stage_bytes;
-    const char* w = reinterpret_cast<const char*>(a.W);
+    const char* w = FMT == WF_BF16 ? reinterpret_cast<const char*>(a.W)
+                                   : reinterpret_cast<const char*>(a.Wq);
     mbar_expect_tx(bar, bytes * R);
     tma_load_1d(dst, w + it * item_bytes, bytes, bar);
     if (R == 2)
@@ -294,25 +360,49 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
     }
     for (int s = 0; s < n_stages; ++s) {
       const int slot = s % NS;
+      const long it = j0 + (long)s * kWarps + warp;
+      const bool has = it < j1;
+      const int n = has ? (int)(it / S) : 0;
+      const int sidx = has ? (int)(it - (long)n * S) : 0;
+      // group scales of this lane's chunks, fetched before the stage lands
+      float sc1[FMT == WF_BF16 ? 1 : kMaxC], sc2[FMT == WF_BF16 ? 1 : kMaxC];
+      if (FMT != WF_BF16 && has) {
+#pragma unroll
+        for (int c = 0; c < kMaxC; ++c) {
+          if (c < nc) {
+            const int k = sidx * seg + c * 256 + lane * 8;
+            sc1[c] = group_scale<FMT>(a.Ws, K, n, k);
+            if (R == 2) sc2[c] = group_scale<FMT>(a.Ws, K, (long)n + a.pair_off, k);
+          }
+        }
+      }
       if (!mbar_wait(full + slot, (uint32_t)((s / NS) & 1))) {
         if (lane == 0) atomicOr(&s_fail, 1);
         break;
       }
-      const long it = j0 + (long)s * kWarps + warp;
-      if (it < j1) {
-        const int n = (int)(it / S), sidx = (int)(it - (long)n * S);
+      if (has) {
         float scl = 0.f;
         if (EPI == EPI_LMHEAD && lane == 0) scl = a.col_scale[n];
-        const bf16* wrow = reinterpret_cast<const bf16*>(
-            ring + slot * stage_bytes + warp * item_bytes);
+        const uint8_t* wb = ring + slot * stage_bytes + warp * item_bytes;
         float acc[NB], acc2[NB];
         if (NB == 1) {
-          acc[0] = row_dot_reg<kMaxC>(wrow, xr, nc, lane);
-          if (R == 2) acc2[0] = row_dot_reg<kMaxC>(wrow + kWarps * seg, xr, nc, lane);
-        } else {
-          row_slice_dot<NB>(wrow, xs + sidx * seg, K, seg, lane, acc);
+          acc[0] = row_dot_reg_q<FMT, kMaxC>(wb, xr, sc1, nc, lane);
           if (R == 2)
-            row_slice_dot<NB>(wrow + kWarps * seg, xs, K, seg, lane, acc2);
+            acc2[0] = row_dot_reg_q<FMT, kMaxC>(wb + kWarps * item_bytes, xr, sc2,
+                                                nc, lane);
+        } else {
+          row_dot_smem_q<FMT, NB, kMaxC>(wb, xs + sidx * seg, K, sc1, nc, lane, acc);
+          if (R == 2)
+            row_dot_smem_q<FMT, NB, kMaxC>(wb + kWarps * item_bytes, xs, K, sc2,
+                                           nc, lane, acc2);
+        }
+        if (FMT == WF_NVFP4) {            // per-tensor second-level scale
+          const float ts = __ldg(a.Wt);
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            acc[b] *= ts;
+            if (R == 2) acc2[b] *= ts;
+          }
         }
         if (lane == 0) {
 #pragma unroll
@@ -390,48 +480,85 @@ size_t fixed_smem(const GemvArgs& a, int nb) {
 // Segments per row S (F32 only: SwiGLU and LM head need whole rows) and
 // ring depth: the largest segment <= kSeg whose 8-item stages still fit at
 // least 3 deep (2 as a last resort).
+int lane_bytes(int fmt) { return fmt == WF_BF16 ? 16 : fmt == WF_MXFP8 ? 8 : 4; }
+
+// Segments per row S (F32 only: SwiGLU and LM head need whole rows) and
+// ring depth: the largest segment <= kSeg whose 8-item stages still fit at
+// least 3 deep (2 as a last resort).
 Plan make_plan(const GemvArgs& a, int nb) {
   const int R = a.epi == EPI_SWIGLU ? 2 : 1;
   const size_t fixed = fixed_smem(a, nb);
+  const int lb = lane_bytes(a.fmt);
   int S = 1;
   if (a.epi == EPI_F32) {
     while (a.K / S > kSeg && (a.K / (2 * S)) % 256 == 0) S *= 2;
     while ((a.K / (2 * S)) % 256 == 0 &&
-           fixed + 3 * (size_t)kWarps * R * (a.K / S) * 2 > kSmemBudget)
+           fixed + 3 * (size_t)kWarps * R * (a.K / S) / 8 * lb > kSmemBudget)
       S *= 2;
   }
-  const size_t stage = (size_t)kWarps * R * (a.K / S) * 2;
+  const size_t stage = (size_t)kWarps * R * (a.K / S) / 8 * lb;
   int NS = stages_default();
+  if (a.fmt != WF_BF16) NS = kMaxStages;          // smaller items: go deeper
   while (NS > 2 && fixed + NS * stage > kSmemBudget) --NS;
   return Plan{S, NS};
 }
 
 size_t smem_bytes(const GemvArgs& a, const Plan& p, int nb) {
   const int R = a.epi == EPI_SWIGLU ? 2 : 1;
-  return (size_t)p.NS * kWarps * R * (a.K / p.S) * 2 + fixed_smem(a, nb);
+  return (size_t)p.NS * kWarps * R * (a.K / p.S) / 8 * lane_bytes(a.fmt) +
+         fixed_smem(a, nb);
 }
 
 int nb_of(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : 8; }
 
-template <int NB, int EPI>
+template <int NB, int EPI, int FMT>
 void launch_t(const GemvArgs& a, int grid, cudaStream_t st) {
   const Plan pl = make_plan(a, NB);
   const size_t smem = smem_bytes(a, pl, NB);
   static size_t configured = 0;
   if (smem > configured) {
-    cudaFuncSetAttribute(gemv_kernel<NB, EPI>,
+    cudaFuncSetAttribute(gemv_kernel<NB, EPI, FMT>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     configured = smem;
   }
-  launch_k(gemv_kernel<NB, EPI>, dim3(grid), dim3(kThreads), smem, st, a, pl);
+  launch_k(gemv_kernel<NB, EPI, FMT>, dim3(grid), dim3(kThreads), smem, st, a,
+           pl);
+}
+
+template <int NB, int EPI>
+void launch_f(const GemvArgs& a, int grid, cudaStream_t st) {
+  switch (a.fmt) {
+    case WF_MXFP8: launch_t<NB, EPI, WF_MXFP8>(a, grid, st); break;
+    case WF_NVFP4: launch_t<NB, EPI, WF_NVFP4>(a, grid, st); break;
+    default: launch_t<NB, EPI, WF_BF16>(a, grid, st); break;
+  }
 }
 
 template <int NB>
 void launch_nb(const GemvArgs& a, int grid, cudaStream_t st) {
   switch (a.epi) {
-    case EPI_F32: launch_t<NB, EPI_F32>(a, grid, st); break;
-    case EPI_SWIGLU: launch_t<NB, EPI_SWIGLU>(a, grid, st); break;
-    default: launch_t<NB, EPI_LMHEAD>(a, grid, st); break;
+    case EPI_F32: launch_f<NB, EPI_F32>(a, grid, st); break;
+    case EPI_SWIGLU: launch_f<NB, EPI_SWIGLU>(a, grid, st); break;
+    default: launch_t<NB, EPI_LMHEAD, WF_BF16>(a, grid, st); break;
+  }
+}
+
+// Decode rows of a quantised matrix to f32 (tests: bit-exact against the
+// format definitions); one thread per 8 consecutive weights.
+template <int FMT>
+__global__ void dequant_rows_kernel(const uint8_t* Wq, const uint8_t* Ws, int K,
+                                    int row0, int nrows, float* out) {
+  const long total = (long)nrows * K / 8;
+  for (long id = blockIdx.x * (long)blockDim.x + threadIdx.x; id < total;
+       id += (long)gridDim.x * blockDim.x) {
+    const long r = id / (K / 8);
+    const int k = (int)(id - r * (K / 8)) * 8;
+    const long row = row0 + r;
+    float w[8];
+    decode8<FMT>(Wq + (row * K + k) / 8 * FmtInfo<FMT>::LB, w);
+    const float sc = group_scale<FMT>(Ws, K, row, k);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[r * K + k + e] = w[e] * sc;
   }
 }
 
@@ -441,6 +568,14 @@ int gemv_splits(const GemvArgs& a) { return make_plan(a, nb_of(a.B)).S; }
 
 int gemv_grid(const GemvArgs& a, int num_sms) {
   return a.n_items < num_sms ? a.n_items : num_sms;
+}
+
+void launch_dequant_rows(int fmt, const uint8_t* Wq, const uint8_t* Ws, int K,
+                         int row0, int nrows, float* out, cudaStream_t st) {
+  if (fmt == WF_MXFP8)
+    dequant_rows_kernel<WF_MXFP8><<<592, 256, 0, st>>>(Wq, Ws, K, row0, nrows, out);
+  else
+    dequant_rows_kernel<WF_NVFP4><<<592, 256, 0, st>>>(Wq, Ws, K, row0, nrows, out);
 }
 
 void launch_gemv(const GemvArgs& a, int grid, cudaStream_t st) {

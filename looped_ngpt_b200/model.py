@@ -90,11 +90,18 @@ class DoryModel:
         for i, (n, t) in enumerate(self.tensors.items()):
             arr[i] = DoryTensor(self._names[i], t.data_ptr(),
                                 t.numel() * t.element_size())
+        # weight format of the block projections, from the tensor names
+        self.wfmt = 0
+        if "blk0.w_qkvg.t" in self.tensors:
+            self.wfmt = 2
+        elif "blk0.w_qkvg.q" in self.tensors:
+            self.wfmt = 1
         lt = (ctypes.c_uint8 * shape.n_blocks)(*shape.layer_types)
         cfg = DoryConfig(shape.d, shape.n_q_heads, shape.n_kv_heads,
                          shape.head_dim, shape.ffn, shape.vocab, shape.n_in,
                          shape.n_rec, shape.n_out, lt, shape.swa_window,
-                         shape.rope_theta_swa, shape.rope_theta_full, 0)
+                         shape.rope_theta_swa, shape.rope_theta_full,
+                         self.wfmt)
         h = ctypes.c_void_p()
         check("dory_init_weights", lib.dory_init_weights(
             ctypes.byref(cfg), arr, len(self.tensors), ctypes.byref(h)))
@@ -190,6 +197,14 @@ class DoryModel:
                                            bytes=arr[i].bytes,
                                            flops=arr[i].flops)
                 for i in range(n.value)}
+
+    def debug_dequant(self, tensor, row0, nrows, K, stream=None):
+        """dory_debug_dequant: f32 [nrows, K] decoded weights."""
+        out = torch.empty((nrows, K), dtype=torch.float32, device=self.device)
+        check("dory_debug_dequant", _lib.load().dory_debug_dequant(
+            self.handle, tensor.encode(), row0, nrows,
+            ctypes.c_void_p(out.data_ptr()), _stream_ptr(stream)))
+        return out
 
     def sync_status(self, stream=None):
         return _lib.load().dory_sync_status(self.handle, _stream_ptr(stream))

@@ -156,8 +156,23 @@ class Model:
 
     # ---- weights -------------------------------------------------------
     def W(self, name):
+        """Weight `name` in float64: BF16 bits widened exactly, or a quantised
+        matrix (name.q / name.s [/ name.t]) decoded by oracle.quant: MXFP8
+        when there is no tensor scale, NVFP4 (with its f32 tensor scale)
+        otherwise."""
         if name in self._dec:
             return self._dec[name]
+        if name not in self.w and name + ".q" in self.w:
+            from . import quant
+            q, sc = self.w[name + ".q"], self.w[name + ".s"]
+            if name + ".t" in self.w:
+                out = quant.dequant_nvfp4(q, sc, float(self.w[name + ".t"][0]))
+            else:
+                out = quant.dequant_mxfp8(q, sc)
+            out = np.asarray(out, dtype=DT)
+            if self._keep:
+                self._dec[name] = out
+            return out
         t = self.w[name]
         if isinstance(t, np.ndarray) and t.dtype == np.uint16:
             out = (t.astype(np.uint32) << 16).view(np.float32).astype(DT)

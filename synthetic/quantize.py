@@ -1,0 +1,90 @@
+"""Weight-format encoding of the seeded BF16 weights into the quantised
+checkpoint formats the Dory pages name: MXFP8 W8A16 (E4M3 values, E8M0 scale
+per 32 weights; MXFP8 explainer page, deployment section) and NVFP4 W4A16
+(E2M1 values, E4M3 scale per 16 weights, f32 tensor scale; paper summary,
+前置知识 / NVFP4).  Maximum scaling (paperlayer §5.2).  This is input
+preparation only; a test checks that it produces exactly the bytes of the
+oracle's own quantiser.
+
+Only the block projections are quantised; embeddings and the LM head stay
+BF16 (paperlayer §5.2).  A quantised matrix `name` becomes
+  name.q  uint8 codes  (MXFP8 [N, K]; NVFP4 [N, K/2], element 2j in the low
+                        nibble)
+  name.s  uint8 scales (MXFP8 E8M0 [N, K/32]; NVFP4 E4M3 [N, K/16])
+  name.t  float32 [1]  (NVFP4 tensor scale)
+"""
+import numpy as np
+
+from .gen import bf16_bits_to_f32
+
+QUANT_LEAVES = ("w_qkvg", "w_o", "w_gu", "w_down")
+
+
+def _e4m3_values():
+    c = np.arange(0x7F)
+    e, m = (c >> 3) & 0xF, c & 7
+    return np.where(e == 0, m * 2.0 ** -9, (1 + m / 8.0) * 2.0 ** (e - 7.0))
+
+
+def _e2m1_values():
+    return np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def _nearest(x, vals):
+    """Code of the nearest value (ties to the even code), with sign bit as
+    the top bit of the format; magnitudes beyond the table saturate."""
+    a = np.abs(x)
+    hi = np.clip(np.searchsorted(vals, a), 1, len(vals) - 1)
+    lo = hi - 1
+    up = (vals[hi] - a < a - vals[lo]) | ((vals[hi] - a == a - vals[lo]) &
+                                          (hi % 2 == 0))
+    return np.where(a >= vals[-1], len(vals) - 1, np.where(up, hi, lo))
+
+
+def encode_mxfp8(w):
+    w = np.asarray(w, dtype=np.float64)
+    N, K = w.shape
+    g = w.reshape(N, K // 32, 32)
+    amax = np.abs(g).max(-1)
+    _, ex = np.frexp(amax)
+    e = np.clip(ex - 9, -127, 127)
+    ecode = np.where(amax > 0, e + 127, 0).astype(np.uint8)
+    scale = np.ldexp(1.0, ecode.astype(np.int64) - 127)
+    y = g / scale[..., None]
+    code = _nearest(y, _e4m3_values()) | np.where(np.signbit(y), 0x80, 0)
+    return code.reshape(N, K).astype(np.uint8), ecode
+
+
+def encode_nvfp4(w):
+    w = np.asarray(w, dtype=np.float64)
+    N, K = w.shape
+    amax = float(np.abs(w).max())
+    S = np.float32(amax / (6.0 * 448.0)) if amax > 0 else np.float32(1.0)
+    g = w.reshape(N, K // 16, 16)
+    e4 = _e4m3_values()
+    sb = _nearest(np.abs(g).max(-1) / (6.0 * float(S)), e4).astype(np.uint8)
+    den = e4[sb] * float(S)
+    y = g / np.where(den > 0, den, 1.0)[..., None]
+    c = _nearest(y, _e2m1_values()) | np.where(np.signbit(y), 0x8, 0)
+    c = np.where(den[..., None] > 0, c, 0).reshape(N, K).astype(np.uint8)
+    packed = (c[:, 0::2] & 0xF) | ((c[:, 1::2] & 0xF) << 4)
+    return packed.astype(np.uint8), sb, np.array([S], dtype=np.float32)
+
+
+def quantize_weights(weights, fmt):
+    """Copy of `weights` with the block projections in `fmt` ('mxfp8' or
+    'nvfp4'); embeddings, LM head and vectors unchanged."""
+    out = {}
+    for name, t in weights.items():
+        leaf = name.split(".", 1)[-1]
+        if leaf in QUANT_LEAVES:
+            w = bf16_bits_to_f32(t)
+            if fmt == "mxfp8":
+                out[name + ".q"], out[name + ".s"] = encode_mxfp8(w)
+            elif fmt == "nvfp4":
+                out[name + ".q"], out[name + ".s"], out[name + ".t"] = encode_nvfp4(w)
+            else:
+                raise ValueError(fmt)
+        else:
+            out[name] = t
+    return out

@@ -51,7 +51,7 @@ def _cfg(shape, **over):
 @pytest.mark.parametrize("over,code", [
     (dict(n_q_heads=3, n_kv_heads=2), -1),   # Hq % Hkv != 0
     (dict(head_dim=96), -2),
-    (dict(wfmt=1), -2),
+    (dict(wfmt=7), -2),                      # unknown weight format
     (dict(d=300), -2),
     (dict(n_rec_blocks=0), -1),
     (dict(swa_window=0), -1),
