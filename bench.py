@@ -45,12 +45,19 @@ def parse():
     ap.add_argument("--no-long", action="store_true",
                     help="skip the long-context batched-decode workloads")
     ap.add_argument("--long-steps", type=int, default=8)
+    ap.add_argument("--quant", action="store_true",
+                    help="also time MXFP8 / NVFP4 weight-only models (B=1 at "
+                         "2048 context and B=4 at 131072 context, k=2)")
     ap.add_argument("--profile-decode", type=int, default=0, metavar="K",
                     help="only: prefill, warm up, then one decode step at "
                          "k=K inside the NVTX range 'decode_step' (for ncu)")
     ap.add_argument("--profile-blocks", default="",
                     help="profile runs only: input,recurrent,output block "
                          "counts of a reduced-depth Dory-width model")
+    ap.add_argument("--profile-quant", default="", choices=["", "mxfp8", "nvfp4"],
+                    help="profile decode runs only: weight format of the "
+                         "block projections (context from the synthetic "
+                         "cache fill)")
     ap.add_argument("--profile-prefill", type=int, default=0, metavar="K",
                     help="only: one prefill at k=K inside the NVTX range "
                          "'prefill' (for ncu)")
@@ -277,12 +284,82 @@ def run_gpu(args, rank, world, local):
         host_tok.copy_(host_out)
     e2e_dt = time.perf_counter() - t0
     barrier(world)
-    if not args.no_long:
+    if not args.no_long or args.quant:
         del cache, headline["cache"]
         torch.cuda.empty_cache()
+    if not args.no_long:
         out["long_context"] = run_long(gm, args, hbm_peak, dev)
+    if args.quant:
+        del gm
+        torch.cuda.empty_cache()
+        out["quantized"] = run_quant(w, args, hbm_peak, dev)
     return dict(out=out, headline=headline, e2e_dt=e2e_dt, w=w,
                 hbm_peak=hbm_peak, tc_peak=tc_peak, peak_kind=peak_kind)
+
+
+def timed_decode(gm, B, ctx, k, mode, steps, hbm_peak, dev, prompt=None):
+    """Decode `steps` tokens (CUDA-graph replays) after `ctx` tokens of
+    context (prefill of `prompt`, else seeded synthetic cache)."""
+    import torch
+    cache = gm.new_cache(B, ctx + steps + 16, 1 if prompt is None else ctx,
+                         kv_mode=mode, max_loops=k)
+    ws = gm.workspace(B, 1 if prompt is None else ctx)
+    if prompt is None:
+        cache.fill_synthetic(ctx, seed=2)
+    else:
+        for t in range(prompt.shape[1]):      # quantised models: T = 1 calls
+            gm.decode_step(cache, prompt[:, t].contiguous(), k, ws,
+                           want_logits=False)
+    tok = torch.zeros(B, dtype=torch.int32, device=dev)
+    gm.decode_step(cache, tok, k, ws, want_logits=False)
+    tb = cache._dec_bufs[0]
+    for _ in range(2):
+        gm.decode_step(cache, tb, k, ws, argmax=tb, want_logits=False)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        gm.decode_step(cache, tb, k, ws, argmax=tb, want_logits=False)
+    e1.record()
+    torch.cuda.synchronize()
+    dt = e0.elapsed_time(e1) / 1e3
+    gm.profile(True)
+    gm.decode_step(cache, tb, k, ws, argmax=tb, want_logits=False)
+    st = gm.profile_read()
+    gm.profile(False)
+    assert gm.sync_status() == 0, "device-side check failed"
+    step_bytes = sum(v["bytes"] for v in st.values())
+    res = {"tok_s": B * steps / dt, "ms_per_step": dt / steps * 1e3,
+           "kv_cache_gb": cache.nbytes / 1e9, "bytes_per_step_gb": step_bytes / 1e9,
+           "hbm_frac": step_bytes * steps / dt / (hbm_peak * 1e9),
+           "kernels_us": {n: round(v["ms"] * 1e3, 1)
+                          for n, v in sorted(st.items(), key=lambda kv: -kv[1]["ms"])}}
+    del cache, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_quant(w, args, hbm_peak, dev):
+    """MXFP8 / NVFP4 weight-only models (embedding and head BF16)."""
+    import torch
+    import looped_ngpt_b200 as lb
+    from synthetic import DORY, make_prompt
+    from synthetic.quantize import quantize_weights
+    res = {}
+    for fmt in ("mxfp8", "nvfp4"):
+        t0 = time.time()
+        qw = quantize_weights(w, fmt)
+        gm = lb.DoryModel(DORY, qw, device=dev)
+        del qw
+        r = {"encode_s": time.time() - t0}
+        r["b1_ctx2k_k2_last_loop"] = timed_decode(gm, 1, 2048, 2, "last_loop",
+                                                  32, hbm_peak, dev)
+        r["b4_ctx131k_k2_last_loop"] = timed_decode(gm, 4, 131072, 2,
+                                                    "last_loop", 8, hbm_peak, dev)
+        res[fmt] = r
+        del gm
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_long(gm, args, hbm_peak, dev):
@@ -337,12 +414,29 @@ def profile_run(args):
     if args.profile_blocks:
         shape = dory_with_blocks(*[int(x) for x in args.profile_blocks.split(",")])
     w = make_weights(shape, seed=0)
+    if args.profile_quant:
+        from synthetic.quantize import quantize_weights
+        w = quantize_weights(w, args.profile_quant)
     gm = lb.DoryModel(shape, w, device="cuda:0")
     prompt = torch.from_numpy(make_prompt(shape, 1, args.prompt)).to("cuda:0")
     k = args.profile_decode or args.profile_prefill
-    cache = gm.new_cache(1, args.prompt + 64, args.prompt, kv_mode=args.kv_mode,
-                         max_loops=k)
+    cache = gm.new_cache(1, args.prompt + 64, 1 if args.profile_quant else args.prompt,
+                         kv_mode=args.kv_mode, max_loops=k)
     ws = gm.workspace(1, args.prompt)
+    if args.profile_quant:
+        # block projections are quantised: T = 1 calls only, so the context
+        # comes from the seeded cache fill
+        cache.fill_synthetic(args.prompt, seed=3)
+        tok = torch.zeros(1, dtype=torch.int32, device="cuda:0")
+        for _ in range(4):
+            gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_push("decode_step")
+        gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
+        assert gm.sync_status() == 0
+        return 0
     if args.profile_prefill:
         torch.cuda.synchronize()
         torch.cuda.nvtx.range_push("prefill")

@@ -10,7 +10,10 @@
 // flight without spending registers.  Each of the 8 consumer warps owns one
 // item of every stage, reduces it with shuffles, writes its output and
 // releases the stage on an "empty" mbarrier: there is no block-wide barrier
-// in the streaming loop.  The first stages are issued before
+// in the streaming loop.  The activations sit in shared memory and the
+// per-lane K loop stays rolled, which keeps the loop body inside the
+// instruction cache (a fully unrolled body with register-resident x was
+// measured 2-3x slower per stage: its code was re-fetched every stage).  The first stages are issued before
 // the programmatic-dependent-launch wait: the weights do not depend on the
 // previous kernel, so HBM starts streaming while the predecessor finishes and
 // while this kernel's prologue runs.  Every mbarrier wait is bounded; on
@@ -22,7 +25,9 @@
 // and the loop-boundary re-injection u_t = N(s_{t-1} + x) (paper summary,
 // 核心方法): every block recomputes the d-length update from L2-resident
 // vectors and block 0 writes the new state, so no separate launch or
-// grid-wide synchronisation is needed.
+// grid-wide synchronisation is needed.  Each thread holds its elements in
+// registers across the block reduction (one L2 round trip; alpha is read
+// before the dependent-launch wait).
 //
 // Epilogues: EPI_F32 (plain), EPI_SWIGLU (rows n and n + F of the fused
 // gate/up matrix -> silu(gate) * up as bf16; the L2 norm that precedes the
@@ -97,8 +102,10 @@ __device__ __forceinline__ void tma_load_1d(void* dst, const void* src,
 }
 
 struct Plan {
-  int S;        // K segments per row (items per row)
+  int S;        // K segments per row (items per row), a power of two
+  int sh;       // log2(S)
   int NS;       // stages in the ring (8 items each)
+  int tmp;      // PRO_UPDATE needs the two-pass prologue (K > kU * kThreads)
 };
 
 // ---- quantised weights (MXFP8 / NVFP4): decode 8 weights of one lane ----
@@ -129,11 +136,11 @@ __device__ __forceinline__ float e4m3_f(uint32_t b) {
   return e4m3x2_f2((uint16_t)(b & 0xFF)).x;
 }
 
-// Bytes of one lane's 8 weights, and weights per scale.
+// Bytes of one lane's 8 weights (scales cover 32 / 16 weights).
 template <int FMT> struct FmtInfo;
-template <> struct FmtInfo<WF_BF16> { static constexpr int LB = 16, GROUP = 0; };
-template <> struct FmtInfo<WF_MXFP8> { static constexpr int LB = 8, GROUP = 32; };
-template <> struct FmtInfo<WF_NVFP4> { static constexpr int LB = 4, GROUP = 16; };
+template <> struct FmtInfo<WF_BF16> { static constexpr int LB = 16; };
+template <> struct FmtInfo<WF_MXFP8> { static constexpr int LB = 8; };
+template <> struct FmtInfo<WF_NVFP4> { static constexpr int LB = 4; };
 
 template <int FMT>
 __device__ __forceinline__ void decode8(const uint8_t* p, float (&w)[8]) {
@@ -167,113 +174,307 @@ __device__ __forceinline__ float group_scale(const uint8_t* Ws, int K, long row,
   return 1.f;
 }
 
-// One staged row segment (item) times the register-resident x slice
-// (batch 1).  Lane covers elements c * 256 + lane * 8 + [0, 8), c < nc; its
-// 8 weights share one group scale (groups of 32 / 16 elements).
-template <int FMT, int MAXC>
-__device__ __forceinline__ float row_dot_reg_q(const uint8_t* wb, const float* xr,
-                                               const float* scl, int nc,
-                                               int lane) {
-  constexpr int LB = FmtInfo<FMT>::LB;
-  float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-  for (int c = 0; c < MAXC; ++c) {
-    if (c < nc) {
-      float w[8];
-      decode8<FMT>(wb + (c * 32 + lane) * LB, w);
-      float t0 = w[0] * xr[c * 8 + 0], t1 = w[1] * xr[c * 8 + 1];
-      t0 = fmaf(w[2], xr[c * 8 + 2], t0); t1 = fmaf(w[3], xr[c * 8 + 3], t1);
-      t0 = fmaf(w[4], xr[c * 8 + 4], t0); t1 = fmaf(w[5], xr[c * 8 + 5], t1);
-      t0 = fmaf(w[6], xr[c * 8 + 6], t0); t1 = fmaf(w[7], xr[c * 8 + 7], t1);
-      if (FMT == WF_BF16) { a0 += t0; a1 += t1; }
-      else { a0 = fmaf(t0, scl[c], a0); a1 = fmaf(t1, scl[c], a1); }
-    }
-  }
-  return warp_sum(a0 + a1);
-}
+// ---- consumer arithmetic ------------------------------------------------
+// The streaming loop is kept compact on purpose: a fully unrolled K loop
+// (x held in registers) made the loop body larger than the instruction cache
+// and every stage re-fetched its code.  Here x lives in shared memory in the
+// multiply format (bf16 for BF16 weights, f16 for the quantised formats) and
+// a lane walks its 8-weight chunks c = lane, lane + 32, ... in a short
+// rolled loop (two chunks per trip for ILP).
 
-// Batched variant: x from shared memory (bf16 [NB][K], slice at xk).
-template <int FMT, int NB, int MAXC>
-__device__ __forceinline__ void row_dot_smem_q(const uint8_t* wb, const bf16* xk,
-                                               int K, const float* scl, int nc,
-                                               int lane, float (&acc)[NB]) {
-  constexpr int LB = FmtInfo<FMT>::LB;
+// Quantised codes of one lane chunk -> four exact f16 pairs (hardware cvt).
+template <int FMT>
+__device__ __forceinline__ void decode8_h2(const uint8_t* p, __half2 (&w)[4]) {
+  if (FMT == WF_MXFP8) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    const uint16_t c[4] = {(uint16_t)(v.x & 0xFFFF), (uint16_t)(v.x >> 16),
+                           (uint16_t)(v.y & 0xFFFF), (uint16_t)(v.y >> 16)};
 #pragma unroll
-  for (int b = 0; b < NB; ++b) acc[b] = 0.f;
-#pragma unroll
-  for (int c = 0; c < MAXC; ++c) {
-    if (c < nc) {
-      float w[8];
-      decode8<FMT>(wb + (c * 32 + lane) * LB, w);
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(xk + b * K + c * 256 + lane * 8);
-        float t = w[0] * bf_lo(xv.x);
-        t = fmaf(w[1], bf_hi(xv.x), t); t = fmaf(w[2], bf_lo(xv.y), t);
-        t = fmaf(w[3], bf_hi(xv.y), t); t = fmaf(w[4], bf_lo(xv.z), t);
-        t = fmaf(w[5], bf_hi(xv.z), t); t = fmaf(w[6], bf_lo(xv.w), t);
-        t = fmaf(w[7], bf_hi(xv.w), t);
-        acc[b] = FMT == WF_BF16 ? acc[b] + t : fmaf(t, scl[c], acc[b]);
-      }
-    }
-  }
-#pragma unroll
-  for (int b = 0; b < NB; ++b) acc[b] = warp_sum(acc[b]);
-}
-
-// Activation vector(s) for the GEMV -> shared memory as bf16: a copy of the
-// caller's bf16 rows (PRO_BF16) or the fused nGPT update (PRO_UPDATE).
-template <int NB>
-__device__ __forceinline__ void gemv_prologue(const GemvArgs& a, bf16* xs,
-                                              float* tmp, float* red) {
-  const int K = a.K, tid = threadIdx.x;
-  if (a.pro == PRO_BF16) {
-    const int vec = K / 8;
-    for (int b = 0; b < NB; ++b) {
-      uint4* dst = reinterpret_cast<uint4*>(xs + b * K);
-      if (b < a.B) {
-        const uint4* src =
-            reinterpret_cast<const uint4*>(a.xin + (size_t)b * a.xin_stride);
-        for (int i = tid; i < vec; i += kThreads) dst[i] = src[i];
-      } else {
-        for (int i = tid; i < vec; i += kThreads) dst[i] = make_uint4(0, 0, 0, 0);
-      }
+    for (int i = 0; i < 4; ++i) {
+      uint32_t h;
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(c[i]));
+      w[i] = *reinterpret_cast<__half2*>(&h);
     }
   } else {
-    for (int b = 0; b < NB; ++b) {
-      if (b < a.B) {
-        float* xrow = nullptr;
-        if (a.reinject == RJ_FIRST && blockIdx.x == 0) xrow = a.x_buf + b * K;
-        if (a.reinject == RJ_NEXT) xrow = a.x_buf + b * K;
-        ngpt_update_row(a.s_in + (size_t)b * K, a.h_in + (size_t)b * K,
-                        a.h_S, (size_t)a.B * K, a.alpha, K, a.reinject, xrow,
-                        blockIdx.x == 0 ? a.s_out + (size_t)b * K : nullptr,
-                        xs + b * K, tmp, red);
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t h;
+      asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }"
+          : "=r"(h)
+          : "r"((v >> (8 * i)) & 0xFF));
+      w[i] = *reinterpret_cast<__half2*>(&h);
+    }
+  }
+}
+
+// 8-term dot product of decoded f16 weights with 8 f16 activations: packed
+// f16 multiply-adds, the pair sum widened to f32.
+__device__ __forceinline__ float dot8_h2(const __half2 (&w)[4], const uint4 xv) {
+  const __half2* x = reinterpret_cast<const __half2*>(&xv);
+  __half2 s = __hmul2(w[0], x[0]);
+  s = __hfma2(w[1], x[1], s);
+  s = __hfma2(w[2], x[2], s);
+  s = __hfma2(w[3], x[3], s);
+  return __low2float(s) + __high2float(s);
+}
+
+// 8-term dot product of bf16 weights with bf16 activations in f32.
+__device__ __forceinline__ float dot8_bf(const uint4 w, const uint4 x) {
+  float t0 = bf_lo(w.x) * bf_lo(x.x), t1 = bf_hi(w.x) * bf_hi(x.x);
+  t0 = fmaf(bf_lo(w.y), bf_lo(x.y), t0); t1 = fmaf(bf_hi(w.y), bf_hi(x.y), t1);
+  t0 = fmaf(bf_lo(w.z), bf_lo(x.z), t0); t1 = fmaf(bf_hi(w.z), bf_hi(x.z), t1);
+  t0 = fmaf(bf_lo(w.w), bf_lo(x.w), t0); t1 = fmaf(bf_hi(w.w), bf_hi(x.w), t1);
+  return t0 + t1;
+}
+
+// Group scale byte -> f32 (E8M0 for MXFP8, E4M3 for NVFP4).
+template <int FMT>
+__device__ __forceinline__ float scale_f(uint32_t b) {
+  return FMT == WF_MXFP8 ? e8m0_f(b) : e4m3_f(b);
+}
+
+// Lane-partial dot products of R staged rows (an item each: wr[r], seg
+// weights) with NB activation segments (x, row stride K elements).  Group
+// scales come from the stage (sr[r], shared memory) or, when they could not
+// be staged, from global memory (gr[r], already offset to the segment).
+template <int FMT, int NB, int R>
+__device__ __forceinline__ void item_dot(const uint8_t* const (&wr)[R],
+                                         const uint8_t* const (&sr)[R],
+                                         const uint8_t* const (&gr)[R],
+                                         const void* x, int K, int nch,
+                                         int lane, float (&acc)[R][NB]) {
+  constexpr int LB = FmtInfo<FMT>::LB;
+  constexpr int GSH = FMT == WF_MXFP8 ? 2 : 1;   // chunk -> group index
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[r][b] = 0.f;
+#pragma unroll 2
+  for (int c = lane; c < nch; c += 32) {
+    uint4 xv[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+      xv[b] = *reinterpret_cast<const uint4*>(
+          reinterpret_cast<const uint16_t*>(x) + (size_t)b * K + c * 8);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (FMT == WF_BF16) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(wr[r] + c * LB);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) acc[r][b] += dot8_bf(wv, xv[b]);
       } else {
-        for (int i = tid; i < K; i += kThreads)
-          xs[b * K + i] = __float2bfloat16_rn(0.f);
+        const uint32_t sb = sr[r] ? (uint32_t)sr[r][c >> GSH]
+                                  : (uint32_t)__ldg(gr[r] + (c >> GSH));
+        const float sc = scale_f<FMT>(sb);
+        __half2 w[4];
+        decode8_h2<FMT>(wr[r] + c * LB, w);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+          acc[r][b] = fmaf(dot8_h2(w, xv[b]), sc, acc[r][b]);
       }
     }
   }
-  __syncthreads();
 }
 
+// ---- prologue: activation rows -> shared memory ---------------------------
+constexpr int kU = 9;        // PRO_UPDATE: elements per thread, K <= kU * kThreads
+constexpr int kCopyU = 5;    // PRO_BF16: 16-byte loads per thread in flight
 
+template <int FMT>
+__device__ __forceinline__ void put_x(void* xs, int i, float v) {
+  if (FMT == WF_BF16) reinterpret_cast<bf16*>(xs)[i] = __float2bfloat16_rn(v);
+  else reinterpret_cast<__half*>(xs)[i] = __float2half_rn(v);
+}
+
+// 8 bf16 -> 8 f16 (exact for the magnitudes of normalised activations).
+__device__ __forceinline__ uint4 bf8_to_h8(uint4 v) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 h = __floats2half2_rn(bf_lo(w[i]), bf_hi(w[i]));
+    w[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// PRO_BF16: copy the caller's bf16 rows (zero rows past B), all loads of a
+// thread in flight together.
+template <int FMT, int NB>
+__device__ __forceinline__ void stage_x_copy(const GemvArgs& a, void* xs) {
+  const int vec = a.K / 8, tid = threadIdx.x;
+#pragma unroll 1
+  for (int b = 0; b < NB; ++b) {
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(xs) +
+                                          (size_t)b * a.K);
+    const uint4* src = reinterpret_cast<const uint4*>(
+        a.xin + (size_t)(b < a.B ? b : 0) * a.xin_stride);
+#pragma unroll 1
+    for (int i0 = tid; i0 < vec; i0 += kCopyU * kThreads) {
+      uint4 v[kCopyU];
+#pragma unroll
+      for (int u = 0; u < kCopyU; ++u) {
+        const int i = i0 + u * kThreads;
+        v[u] = (b < a.B && i < vec) ? src[i] : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kCopyU; ++u) {
+        const int i = i0 + u * kThreads;
+        if (i < vec) dst[i] = FMT == WF_BF16 ? v[u] : bf8_to_h8(v[u]);
+      }
+    }
+  }
+}
+
+struct UpdScal { float inv_h, inv_t, inv_u; };
+
+// Norm reciprocals from the block-reduced sums r = [|h|^2, sum (a s)^2,
+// sum (a s)(alpha h), sum (alpha h)^2, sum (a s) x, sum (alpha h) x, |x|^2],
+// a = 1 - alpha.
+__device__ __forceinline__ UpdScal upd_scalars(const float (&r)[7], bool next) {
+  UpdScal q;
+  q.inv_h = 1.f / fmaxf(sqrtf(r[0]), 1e-12f);
+  const float tt = r[1] + 2.f * r[2] * q.inv_h + r[3] * q.inv_h * q.inv_h;
+  q.inv_t = 1.f / fmaxf(sqrtf(fmaxf(tt, 0.f)), 1e-12f);
+  q.inv_u = 1.f;
+  if (next) {
+    const float dot = (r[4] + r[5] * q.inv_h) * q.inv_t;
+    q.inv_u = 1.f / fmaxf(sqrtf(fmaxf(1.f + 2.f * dot + r[6], 0.f)), 1e-12f);
+  }
+  return q;
+}
+
+// Element i of the updated row: new state (block 0 stores it, and x for
+// RJ_FIRST), re-injected value to the activation row in shared memory.
+template <int FMT>
+__device__ __forceinline__ void upd_store(const GemvArgs& a, const UpdScal& q,
+                                          size_t row, int i, float al, float sv,
+                                          float hv, float xv, void* xs) {
+  const bool lead = blockIdx.x == 0;
+  float v = ((1.f - al) * sv + al * hv * q.inv_h) * q.inv_t;
+  if (a.reinject == RJ_FIRST && lead && a.x_buf) a.x_buf[row + i] = v;
+  if (a.reinject == RJ_NEXT) v = (v + xv) * q.inv_u;
+  if (lead) a.s_out[row + i] = v;
+  put_x<FMT>(xs, (int)(row + i), v);
+}
+
+// PRO_UPDATE for batch row b: the previous sublayer's nGPT update
+//   s <- N((1 - alpha) s + alpha h / |h|),  h = sum of h_S partials,
+// and the loop re-injection (RJ_FIRST: x := s, result s; RJ_NEXT: result
+// N(s + x)), with both norms from one block reduction
+//   |t|^2 = sum ((1-alpha) s)^2 + 2 sum (1-alpha) alpha s h / |h|
+//           + sum (alpha h)^2 / |h|^2,
+//   |t + x|^2 = 1 + 2 t.x + |x|^2   (t of unit norm).
+// Every thread keeps its kU elements in registers across the reduction, so
+// the whole update costs one round trip to L2.  `al` holds this thread's
+// alpha values (loaded before the programmatic-dependent-launch wait).
+template <int FMT>
+__device__ __forceinline__ void stage_x_update(const GemvArgs& a, int b,
+                                               const float (&al)[kU], void* xs,
+                                               float* red) {
+  const int K = a.K, tid = threadIdx.x;
+  const bool next = a.reinject == RJ_NEXT;
+  const size_t row = (size_t)b * K, hs = (size_t)a.B * K;
+  float sv[kU], hv[kU], xv[kU];
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+    const int i = tid + u * kThreads;
+    sv[u] = hv[u] = xv[u] = 0.f;
+    if (i < K) {
+      sv[u] = a.s_in[row + i];
+      hv[u] = a.h_in[row + i];
+      if (next) xv[u] = a.x_buf[row + i];
+    }
+  }
+#pragma unroll 1
+  for (int k0 = 1; k0 < a.h_S; k0 += 3) {
+    float t[3][kU];
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int i = tid + u * kThreads;
+        t[j][u] = (k0 + j < a.h_S && i < K) ? a.h_in[(k0 + j) * hs + row + i] : 0.f;
+      }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) hv[u] += t[0][u] + t[1][u] + t[2][u];
+  }
+  float r[7] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+    const float as = (1.f - al[u]) * sv[u], ah = al[u] * hv[u];
+    r[0] = fmaf(hv[u], hv[u], r[0]);
+    r[1] = fmaf(as, as, r[1]);
+    r[2] = fmaf(as, ah, r[2]);
+    r[3] = fmaf(ah, ah, r[3]);
+    r[4] = fmaf(as, xv[u], r[4]);
+    r[5] = fmaf(ah, xv[u], r[5]);
+    r[6] = fmaf(xv[u], xv[u], r[6]);
+  }
+  block_sum_n<7>(r, red);
+  const UpdScal q = upd_scalars(r, next);
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+    const int i = tid + u * kThreads;
+    if (i < K) upd_store<FMT>(a, q, row, i, al[u], sv[u], hv[u], xv[u], xs);
+  }
+}
+
+// PRO_UPDATE for K > kU * kThreads: the same update in two passes, the
+// summed h kept in shared memory (tmp [K]) in between.
+template <int FMT>
+__device__ void stage_x_update_2pass(const GemvArgs& a, int b, void* xs,
+                                     float* tmp, float* red) {
+  const int K = a.K, tid = threadIdx.x;
+  const bool next = a.reinject == RJ_NEXT;
+  const size_t row = (size_t)b * K, hs = (size_t)a.B * K;
+  float r[7] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int i = tid; i < K; i += kThreads) {
+    float h = 0.f;
+    for (int k = 0; k < a.h_S; ++k) h += a.h_in[k * hs + row + i];
+    const float al = a.alpha[i], sv = a.s_in[row + i];
+    const float xv = next ? a.x_buf[row + i] : 0.f;
+    tmp[i] = h;
+    const float as = (1.f - al) * sv, ah = al * h;
+    r[0] = fmaf(h, h, r[0]);
+    r[1] = fmaf(as, as, r[1]);
+    r[2] = fmaf(as, ah, r[2]);
+    r[3] = fmaf(ah, ah, r[3]);
+    r[4] = fmaf(as, xv, r[4]);
+    r[5] = fmaf(ah, xv, r[5]);
+    r[6] = fmaf(xv, xv, r[6]);
+  }
+  block_sum_n<7>(r, red);
+  const UpdScal q = upd_scalars(r, next);
+  for (int i = tid; i < K; i += kThreads)
+    upd_store<FMT>(a, q, row, i, a.alpha[i], a.s_in[row + i], tmp[i],
+                   next ? a.x_buf[row + i] : 0.f, xs);
+}
+
+// ---- the kernel -----------------------------------------------------------
 template <int NB, int EPI, int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemv_kernel(const GemvArgs a, const Plan pl) {
   constexpr int R = (EPI == EPI_SWIGLU) ? 2 : 1;
   constexpr int LB = FmtInfo<FMT>::LB;       // bytes per 8 weights
+  constexpr int GROUP = FMT == WF_MXFP8 ? 32 : 16;
   extern __shared__ __align__(128) uint8_t smem[];
   const int K = a.K, S = pl.S, NS = pl.NS;
-  const int seg = K / S;
-  const size_t item_bytes = (size_t)seg / 8 * LB;
-  const size_t stage_bytes = (size_t)kWarps * R * item_bytes;
-  uint8_t* ring = smem;                                         // NS stages
-  bf16* xs = reinterpret_cast<bf16*>(ring + NS * stage_bytes);  // [NB][K]
-  float* tmp = reinterpret_cast<float*>(xs + NB * K);           // [K] if UPDATE
-  uint64_t* full = reinterpret_cast<uint64_t*>(
-      tmp + (a.pro == PRO_UPDATE ? K : 0));
+  const int seg = K >> pl.sh, nch = seg / 8;
+  const uint32_t item_bytes = (uint32_t)nch * LB;
+  // quantised formats: each item's group scales (sb bytes) ride in the same
+  // stage as its codes when they keep the 16-byte rules of bulk copies,
+  // else the consumers read them from global memory
+  const int sb = FMT == WF_BF16 ? 0 : seg / GROUP;
+  const bool sc_tma = FMT != WF_BF16 && (sb % 16) == 0;
+  const uint32_t codes_bytes = (uint32_t)kWarps * R * item_bytes;
+  const uint32_t stage_bytes =
+      codes_bytes + (sc_tma ? (uint32_t)(kWarps * R * sb) : 0u);
+  uint8_t* ring = smem;                                   // NS stages
+  void* xs = ring + (size_t)NS * stage_bytes;             // [NB][K] 16-bit
+  float* tmp = reinterpret_cast<float*>(reinterpret_cast<uint16_t*>(xs) +
+                                        (size_t)NB * K);  // [K] if 2-pass
+  uint64_t* full = reinterpret_cast<uint64_t*>(tmp + (pl.tmp ? K : 0));
   uint64_t* empty = full + NS;
   __shared__ float red[7 * (kWarps + 1)];
   __shared__ float bestv[kWarps][NB];
@@ -283,27 +484,45 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // row-aligned item range: a stage of 8 items starts at a multiple of S,
   // so warp w always works on K segment w % S
-  const long j0 = (long)a.n_items * blockIdx.x / gridDim.x * S;
-  const long j1 = (long)a.n_items * (blockIdx.x + 1) / gridDim.x * S;
-  const int n_stages = (int)((j1 - j0 + kWarps - 1) / kWarps);
+  const int j0 = (int)((long)a.n_items * blockIdx.x / gridDim.x) * S;
+  const int j1 = (int)((long)a.n_items * (blockIdx.x + 1) / gridDim.x) * S;
+  const int n_stages = (j1 - j0 + kWarps - 1) / kWarps;
   const bool producer = tid == kWarps * 32;
 
-  // items j0.. are contiguous in W: item it = (row it / S, segment it % S)
+  // items j0.. are contiguous in W: item it = (row it >> sh, segment it & (S-1))
   auto issue = [&](int s) {
-    const long it = j0 + (long)s * kWarps;
-    const long cnt = j1 - it < kWarps ? j1 - it : kWarps;
-    const uint32_t bytes = (uint32_t)(cnt * item_bytes);
+    const int it = j0 + s * kWarps;
+    const int cnt = j1 - it < kWarps ? j1 - it : kWarps;
+    const uint32_t bytes = (uint32_t)cnt * item_bytes;
     uint64_t* bar = full + (s % NS);
-    uint8_t* dst = ring + (s % NS) * stage_bytes;
+    uint8_t* dst = ring + (size_t)(s % NS) * stage_bytes;
     const char* w = FMT == WF_BF16 ? reinterpret_cast<const char*>(a.W)
                                    : reinterpret_cast<const char*>(a.Wq);
-    mbar_expect_tx(bar, bytes * R);
-    tma_load_1d(dst, w + it * item_bytes, bytes, bar);
+    const uint32_t sbytes = sc_tma ? (uint32_t)(cnt * sb) : 0u;
+    mbar_expect_tx(bar, (bytes + sbytes) * R);
+    tma_load_1d(dst, w + (size_t)it * item_bytes, bytes, bar);
     if (R == 2)
       tma_load_1d(dst + kWarps * item_bytes,
-                  w + (it + (long)a.pair_off * S) * item_bytes, bytes, bar);
+                  w + ((size_t)it + (size_t)a.pair_off * S) * item_bytes, bytes,
+                  bar);
+    if (sc_tma) {
+      // scales of item it start at byte it * sb (rows are K / GROUP bytes)
+      const char* ws = reinterpret_cast<const char*>(a.Ws);
+      tma_load_1d(dst + codes_bytes, ws + (size_t)it * sb, sbytes, bar);
+      if (R == 2)
+        tma_load_1d(dst + codes_bytes + kWarps * sb,
+                    ws + ((size_t)it + (size_t)a.pair_off * S) * sb, sbytes, bar);
+    }
   };
 
+  // alpha is a weight: read it before the wait, like the first stages
+  float al[kU];
+  const bool upd_reg = a.pro == PRO_UPDATE && !pl.tmp;
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+    const int i = tid + u * kThreads;
+    al[u] = (upd_reg && i < K) ? __ldg(a.alpha + i) : 0.f;
+  }
   if (producer) {
     for (int i = 0; i < NS; ++i) {
       mbar_init(full + i, 1);
@@ -317,7 +536,20 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
   }
   pdl_wait();
   pdl_trigger();
-  gemv_prologue<NB>(a, xs, tmp, red);           // ends with __syncthreads()
+  if (a.pro == PRO_UPDATE) {
+#pragma unroll 1
+    for (int b = 0; b < NB; ++b) {
+      if (b < a.B) {
+        if (upd_reg) stage_x_update<FMT>(a, b, al, xs, red);
+        else stage_x_update_2pass<FMT>(a, b, xs, tmp, red);
+      } else {
+        for (int i = tid; i < K; i += kThreads) put_x<FMT>(xs, b * K + i, 0.f);
+      }
+    }
+  } else {
+    stage_x_copy<FMT, NB>(a, xs);
+  }
+  __syncthreads();
 
   volatile int* fail = &s_fail;
   float bv[NB];
@@ -340,82 +572,58 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
     }
   } else {
     // ---- consumers: warp w owns item w of every stage ------------------
-    // NB == 1: this warp's slice of x (segment w % S, lane's 8-element
-    // chunks) stays in registers as f32 for the whole kernel.
-    constexpr int kMaxC = kSeg / 256;
-    const int nc = seg >> 8;
-    float xr[NB == 1 ? kMaxC * 8 : 1];
-    if (NB == 1) {
-      const bf16* xk = xs + (warp % S) * seg + lane * 8;
-#pragma unroll
-      for (int c = 0; c < kMaxC; ++c) {
-        if (c < nc) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(xk + c * 256);
-          xr[c * 8 + 0] = bf_lo(xv.x); xr[c * 8 + 1] = bf_hi(xv.x);
-          xr[c * 8 + 2] = bf_lo(xv.y); xr[c * 8 + 3] = bf_hi(xv.y);
-          xr[c * 8 + 4] = bf_lo(xv.z); xr[c * 8 + 5] = bf_hi(xv.z);
-          xr[c * 8 + 6] = bf_lo(xv.w); xr[c * 8 + 7] = bf_hi(xv.w);
-        }
-      }
-    }
+    const int sbrow = FMT == WF_BF16 ? 0 : K / GROUP;
+    int slot = 0;
+    uint32_t phase = 0;
     for (int s = 0; s < n_stages; ++s) {
-      const int slot = s % NS;
-      const long it = j0 + (long)s * kWarps + warp;
+      const int it = j0 + s * kWarps + warp;
       const bool has = it < j1;
-      const int n = has ? (int)(it / S) : 0;
-      const int sidx = has ? (int)(it - (long)n * S) : 0;
-      // group scales of this lane's chunks, fetched before the stage lands
-      float sc1[FMT == WF_BF16 ? 1 : kMaxC], sc2[FMT == WF_BF16 ? 1 : kMaxC];
-      if (FMT != WF_BF16 && has) {
-#pragma unroll
-        for (int c = 0; c < kMaxC; ++c) {
-          if (c < nc) {
-            const int k = sidx * seg + c * 256 + lane * 8;
-            sc1[c] = group_scale<FMT>(a.Ws, K, n, k);
-            if (R == 2) sc2[c] = group_scale<FMT>(a.Ws, K, (long)n + a.pair_off, k);
-          }
-        }
-      }
-      if (!mbar_wait(full + slot, (uint32_t)((s / NS) & 1))) {
+      const int n = it >> pl.sh, sidx = it & (S - 1);
+      if (!mbar_wait(full + slot, phase)) {
         if (lane == 0) atomicOr(&s_fail, 1);
         break;
       }
       if (has) {
-        float scl = 0.f;
-        if (EPI == EPI_LMHEAD && lane == 0) scl = a.col_scale[n];
-        const uint8_t* wb = ring + slot * stage_bytes + warp * item_bytes;
-        float acc[NB], acc2[NB];
-        if (NB == 1) {
-          acc[0] = row_dot_reg_q<FMT, kMaxC>(wb, xr, sc1, nc, lane);
-          if (R == 2)
-            acc2[0] = row_dot_reg_q<FMT, kMaxC>(wb + kWarps * item_bytes, xr, sc2,
-                                                nc, lane);
-        } else {
-          row_dot_smem_q<FMT, NB, kMaxC>(wb, xs + sidx * seg, K, sc1, nc, lane, acc);
-          if (R == 2)
-            row_dot_smem_q<FMT, NB, kMaxC>(wb + kWarps * item_bytes, xs, K, sc2,
-                                           nc, lane, acc2);
+        const uint8_t* stg = ring + (size_t)slot * stage_bytes;
+        const uint8_t* wr[R];
+        const uint8_t* sr[R];
+        const uint8_t* gr[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          wr[r] = stg + (r * kWarps + warp) * item_bytes;
+          sr[r] = sc_tma ? stg + codes_bytes + (r * kWarps + warp) * sb : nullptr;
+          gr[r] = (FMT != WF_BF16 && !sc_tma)
+                      ? a.Ws + (size_t)(n + r * a.pair_off) * sbrow + sidx * sb
+                      : nullptr;
         }
+        float acc[R][NB];
+        item_dot<FMT, NB, R>(wr, sr, gr,
+                             reinterpret_cast<const uint16_t*>(xs) + sidx * seg,
+                             K, nch, lane, acc);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int b = 0; b < NB; ++b) acc[r][b] = warp_sum(acc[r][b]);
         if (FMT == WF_NVFP4) {            // per-tensor second-level scale
           const float ts = __ldg(a.Wt);
 #pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            acc[b] *= ts;
-            if (R == 2) acc2[b] *= ts;
-          }
+          for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int b = 0; b < NB; ++b) acc[r][b] *= ts;
         }
         if (lane == 0) {
+          const float scl = EPI == EPI_LMHEAD ? a.col_scale[n] : 0.f;
 #pragma unroll
           for (int b = 0; b < NB; ++b) {
             if (b >= a.B) break;
             if (EPI == EPI_F32) {
-              a.out[((size_t)sidx * a.B + b) * a.n_items + n] = acc[b];
+              a.out[((size_t)sidx * a.B + b) * a.n_items + n] = acc[0][b];
             } else if (EPI == EPI_SWIGLU) {
-              const float g = acc[b];
+              const float g = acc[0][b];
               a.out_bf[(size_t)b * a.pair_off + n] =
-                  __float2bfloat16_rn(g * sigmoidf_(g) * acc2[b]);
+                  __float2bfloat16_rn(g * sigmoidf_(g) * acc[R - 1][b]);
             } else {
-              const float z = scl * acc[b];
+              const float z = scl * acc[0][b];
               if (a.out) a.out[(size_t)b * a.out_stride + n] = z;
               if (z > bv[b]) { bv[b] = z; bi[b] = n; }
             }
@@ -424,6 +632,7 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + slot);
+      if (++slot == NS) { slot = 0; phase ^= 1u; }
       if (*fail) break;
     }
   }
@@ -472,14 +681,16 @@ int stages_default() {
 
 constexpr size_t kSmemBudget = 220 * 1024;
 
+bool needs_tmp(const GemvArgs& a) {
+  return a.pro == PRO_UPDATE && a.K > kU * kThreads;
+}
+
 size_t fixed_smem(const GemvArgs& a, int nb) {
-  return (size_t)nb * a.K * 2 + (a.pro == PRO_UPDATE ? (size_t)a.K * 4 : 0) +
+  return (size_t)nb * a.K * 2 + (needs_tmp(a) ? (size_t)a.K * 4 : 0) +
          2 * kMaxStages * 8;
 }
 
-// Segments per row S (F32 only: SwiGLU and LM head need whole rows) and
-// ring depth: the largest segment <= kSeg whose 8-item stages still fit at
-// least 3 deep (2 as a last resort).
+// Bytes of one lane chunk (8 weights) of a format.
 int lane_bytes(int fmt) { return fmt == WF_BF16 ? 16 : fmt == WF_MXFP8 ? 8 : 4; }
 
 // Segments per row S (F32 only: SwiGLU and LM head need whole rows) and
@@ -496,16 +707,25 @@ Plan make_plan(const GemvArgs& a, int nb) {
            fixed + 3 * (size_t)kWarps * R * (a.K / S) / 8 * lb > kSmemBudget)
       S *= 2;
   }
-  const size_t stage = (size_t)kWarps * R * (a.K / S) / 8 * lb;
+  const int sbytes = a.fmt == WF_BF16 ? 0
+                     : (a.K / S) / (a.fmt == WF_MXFP8 ? 32 : 16);
+  const size_t stage = (size_t)kWarps * R * ((a.K / S) / 8 * lb +
+                                             (sbytes % 16 == 0 ? sbytes : 0));
   int NS = stages_default();
   if (a.fmt != WF_BF16) NS = kMaxStages;          // smaller items: go deeper
   while (NS > 2 && fixed + NS * stage > kSmemBudget) --NS;
-  return Plan{S, NS};
+  int sh = 0;
+  while ((1 << sh) < S) ++sh;
+  return Plan{S, sh, NS, needs_tmp(a) ? 1 : 0};
 }
 
 size_t smem_bytes(const GemvArgs& a, const Plan& p, int nb) {
   const int R = a.epi == EPI_SWIGLU ? 2 : 1;
-  return (size_t)p.NS * kWarps * R * (a.K / p.S) / 8 * lane_bytes(a.fmt) +
+  const int sbytes = a.fmt == WF_BF16 ? 0
+                     : (a.K / p.S) / (a.fmt == WF_MXFP8 ? 32 : 16);
+  return (size_t)p.NS * kWarps * R *
+             ((a.K / p.S) / 8 * lane_bytes(a.fmt) +
+              (sbytes % 16 == 0 ? sbytes : 0)) +
          fixed_smem(a, nb);
 }
 

@@ -71,20 +71,47 @@ def encode_nvfp4(w):
     return packed.astype(np.uint8), sb, np.array([S], dtype=np.float32)
 
 
-def quantize_weights(weights, fmt):
+def _encode_rows(w, fmt, rows=2048):
+    """Encode in row chunks (bounded float64 temporaries).  The NVFP4 tensor
+    scale needs the whole-matrix maximum first."""
+    N = w.shape[0]
+    if fmt == "mxfp8":
+        qs, ss = zip(*(encode_mxfp8(w[r:r + rows]) for r in range(0, N, rows)))
+        return np.concatenate(qs), np.concatenate(ss)
+    amax = float(np.abs(w).max())
+    S = np.float32(amax / (6.0 * 448.0)) if amax > 0 else np.float32(1.0)
+    e4, out_q, out_s = _e4m3_values(), [], []
+    for r in range(0, N, rows):
+        g = np.asarray(w[r:r + rows], dtype=np.float64)
+        n, K = g.shape
+        g = g.reshape(n, K // 16, 16)
+        sb = _nearest(np.abs(g).max(-1) / (6.0 * float(S)), e4).astype(np.uint8)
+        den = e4[sb] * float(S)
+        y = g / np.where(den > 0, den, 1.0)[..., None]
+        c = _nearest(y, _e2m1_values()) | np.where(np.signbit(y), 0x8, 0)
+        c = np.where(den[..., None] > 0, c, 0).reshape(n, K).astype(np.uint8)
+        out_q.append(((c[:, 0::2] & 0xF) | ((c[:, 1::2] & 0xF) << 4)).astype(np.uint8))
+        out_s.append(sb)
+    return (np.concatenate(out_q), np.concatenate(out_s),
+            np.array([S], dtype=np.float32))
+
+
+def quantize_weights(weights, fmt, workers=None):
     """Copy of `weights` with the block projections in `fmt` ('mxfp8' or
-    'nvfp4'); embeddings, LM head and vectors unchanged."""
-    out = {}
-    for name, t in weights.items():
-        leaf = name.split(".", 1)[-1]
-        if leaf in QUANT_LEAVES:
-            w = bf16_bits_to_f32(t)
-            if fmt == "mxfp8":
-                out[name + ".q"], out[name + ".s"] = encode_mxfp8(w)
-            elif fmt == "nvfp4":
-                out[name + ".q"], out[name + ".s"], out[name + ".t"] = encode_nvfp4(w)
-            else:
-                raise ValueError(fmt)
-        else:
-            out[name] = t
+    'nvfp4'); embeddings, LM head and vectors unchanged.  Matrices are
+    encoded on a thread pool (NumPy releases the GIL in the bulk work)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    if fmt not in ("mxfp8", "nvfp4"):
+        raise ValueError(fmt)
+    names = [n for n in weights if n.split(".", 1)[-1] in QUANT_LEAVES]
+    out = {n: t for n, t in weights.items() if n not in names}
+    workers = workers or min(32, os.cpu_count() or 1)
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        res = list(ex.map(lambda n: _encode_rows(bf16_bits_to_f32(weights[n]),
+                                                 fmt), names))
+    for n, r in zip(names, res):
+        out[n + ".q"], out[n + ".s"] = r[0], r[1]
+        if fmt == "nvfp4":
+            out[n + ".t"] = r[2]
     return out
