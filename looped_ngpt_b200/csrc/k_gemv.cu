@@ -101,6 +101,26 @@ __device__ __forceinline__ void tma_load_1d(void* dst, const void* src,
       : "memory");
 }
 
+// The same copy with an L2 eviction-priority hint: streamed weights are read
+// once per call, and evict-first keeps them from displacing the small
+// vectors (states, partial outputs, per-layer scales, KV tiles) that the
+// dependent kernels read next.
+__device__ __forceinline__ void tma_load_1d_hint(void* dst, const void* src,
+                                                 uint32_t bytes, uint64_t* bar,
+                                                 uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 struct Plan {
   int S;        // K segments per row (items per row), a power of two
   int sh;       // log2(S)
@@ -451,6 +471,81 @@ __device__ void stage_x_update_2pass(const GemvArgs& a, int b, void* xs,
                    next ? a.x_buf[row + i] : 0.f, xs);
 }
 
+// ---- batch-1 BF16 rows on the tensor cores ---------------------------------
+// One row segment w[0..seg) (seg = 256 * nks, in shared memory) dotted with
+// x on the warp-level MMA: the segment is read as a 16 x (seg/16) matrix A
+// whose row i holds the 8-element chunks i, i+16, i+32, ... of w, and B
+// holds the matching chunks of x in its column i, so that
+// sum_i (A B)[i][i] = w . x.  The off-diagonal products are discarded: the
+// tensor cores have far more throughput than this needs, and in exchange x
+// stays in registers (B fragments, loaded once per launch) and the weights
+// are read from shared memory once, by ldmatrix (k-step s covers chunks
+// 32 s .. 32 s + 31, 512 contiguous bytes).  Per row: nks ldmatrix.x4 and
+// 2 nks MMAs instead of ~27 instructions per 8 weights and lane.
+constexpr int kKS = kSeg / 256;           // k-steps of a full segment
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// B fragments of x segment xseg (bf16) for k-steps s < nks.  Fragment layout
+// of m16n8k16 (col-major B): lane (g = lane / 4, t = lane % 4) holds k rows
+// 2t, 2t+1 (reg 0) and 2t+8, 2t+9 (reg 1) of column g.  Columns 0-7 of the
+// first MMA take chunks g and g+16 of k-step s, columns 8-15 of the second
+// chunks g+8 and g+24.
+__device__ __forceinline__ void load_xfrag(const bf16* xseg, int nks, int lane,
+                                           uint32_t (&xb)[kKS][4]) {
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t* xw = reinterpret_cast<const uint32_t*>(xseg);
+#pragma unroll
+  for (int s = 0; s < kKS; ++s) {
+    if (s < nks) {
+      const int c0 = 32 * s + g;
+      xb[s][0] = xw[(c0 + 0) * 4 + t];
+      xb[s][1] = xw[(c0 + 16) * 4 + t];
+      xb[s][2] = xw[(c0 + 8) * 4 + t];
+      xb[s][3] = xw[(c0 + 24) * 4 + t];
+    } else {
+      xb[s][0] = xb[s][1] = xb[s][2] = xb[s][3] = 0u;
+    }
+  }
+}
+
+// Full dot product (every lane gets it) of the staged row segment at w.
+__device__ __forceinline__ float row_dot_mma(const uint8_t* w,
+                                             const uint32_t (&xb)[kKS][4],
+                                             int nks, int lane) {
+  float d[4][4] = {};                     // two accumulator pairs (ILP)
+  const uint32_t base = smem_addr(w) + lane * 16;
+#pragma unroll
+  for (int s = 0; s < kKS; ++s) {
+    if (s < nks) {
+      uint32_t a[4];
+      asm volatile(
+          "ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+          : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+          : "r"(base + s * 512));
+      mma_bf16_16816(d[(s & 1) * 2 + 0], a, xb[s][0], xb[s][1]);
+      mma_bf16_16816(d[(s & 1) * 2 + 1], a, xb[s][2], xb[s][3]);
+    }
+  }
+  // diagonal: (i, i) of the first MMA sits in lane 4i + i/2 (d[0] / d[1]
+  // for even / odd i), (8+i, 8+i) of the second in the same lane (d[2] /
+  // d[3])
+  const int g = lane >> 2, t = lane & 3;
+  float v = 0.f;
+  if (t == (g >> 1)) {
+    v = (g & 1) ? d[0][1] + d[1][3] + d[2][1] + d[3][3]
+                : d[0][0] + d[1][2] + d[2][0] + d[3][2];
+  }
+  return warp_sum(v);
+}
+
 // ---- the kernel -----------------------------------------------------------
 template <int NB, int EPI, int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -490,6 +585,7 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
   const bool producer = tid == kWarps * 32;
 
   // items j0.. are contiguous in W: item it = (row it >> sh, segment it & (S-1))
+  const uint64_t pol = evict_first_policy();
   auto issue = [&](int s) {
     const int it = j0 + s * kWarps;
     const int cnt = j1 - it < kWarps ? j1 - it : kWarps;
@@ -500,18 +596,19 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
                                    : reinterpret_cast<const char*>(a.Wq);
     const uint32_t sbytes = sc_tma ? (uint32_t)(cnt * sb) : 0u;
     mbar_expect_tx(bar, (bytes + sbytes) * R);
-    tma_load_1d(dst, w + (size_t)it * item_bytes, bytes, bar);
+    tma_load_1d_hint(dst, w + (size_t)it * item_bytes, bytes, bar, pol);
     if (R == 2)
-      tma_load_1d(dst + kWarps * item_bytes,
-                  w + ((size_t)it + (size_t)a.pair_off * S) * item_bytes, bytes,
-                  bar);
+      tma_load_1d_hint(dst + kWarps * item_bytes,
+                       w + ((size_t)it + (size_t)a.pair_off * S) * item_bytes, bytes,
+                       bar, pol);
     if (sc_tma) {
       // scales of item it start at byte it * sb (rows are K / GROUP bytes)
       const char* ws = reinterpret_cast<const char*>(a.Ws);
-      tma_load_1d(dst + codes_bytes, ws + (size_t)it * sb, sbytes, bar);
+      tma_load_1d_hint(dst + codes_bytes, ws + (size_t)it * sb, sbytes, bar, pol);
       if (R == 2)
-        tma_load_1d(dst + codes_bytes + kWarps * sb,
-                    ws + ((size_t)it + (size_t)a.pair_off * S) * sb, sbytes, bar);
+        tma_load_1d_hint(dst + codes_bytes + kWarps * sb,
+                         ws + ((size_t)it + (size_t)a.pair_off * S) * sb, sbytes,
+                         bar, pol);
     }
   };
 
@@ -575,6 +672,13 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
     const int sbrow = FMT == WF_BF16 ? 0 : K / GROUP;
     int slot = 0;
     uint32_t phase = 0;
+    // batch 1, BF16: tensor-core row dots with x (this warp's segment
+    // w % S) held as MMA fragments for the whole launch
+    constexpr bool kMma = FMT == WF_BF16 && NB == 1;
+    uint32_t xb[kMma ? kKS : 1][4];
+    if constexpr (kMma)
+      load_xfrag(reinterpret_cast<const bf16*>(xs) + (warp % S) * seg, seg / 256,
+                 lane, reinterpret_cast<uint32_t (&)[kKS][4]>(xb));
     for (int s = 0; s < n_stages; ++s) {
       const int it = j0 + s * kWarps + warp;
       const bool has = it < j1;
@@ -597,13 +701,20 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
                       : nullptr;
         }
         float acc[R][NB];
-        item_dot<FMT, NB, R>(wr, sr, gr,
-                             reinterpret_cast<const uint16_t*>(xs) + sidx * seg,
-                             K, nch, lane, acc);
+        if constexpr (kMma) {
 #pragma unroll
-        for (int r = 0; r < R; ++r)
+          for (int r = 0; r < R; ++r)
+            acc[r][0] = row_dot_mma(wr[r], reinterpret_cast<const uint32_t (&)[kKS][4]>(xb),
+                                    seg / 256, lane);
+        } else {
+          item_dot<FMT, NB, R>(wr, sr, gr,
+                               reinterpret_cast<const uint16_t*>(xs) + sidx * seg,
+                               K, nch, lane, acc);
 #pragma unroll
-          for (int b = 0; b < NB; ++b) acc[r][b] = warp_sum(acc[r][b]);
+          for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int b = 0; b < NB; ++b) acc[r][b] = warp_sum(acc[r][b]);
+        }
         if (FMT == WF_NVFP4) {            // per-tensor second-level scale
           const float ts = __ldg(a.Wt);
 #pragma unroll
