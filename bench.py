@@ -64,6 +64,29 @@ def parse():
     return ap.parse_args()
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu capture of the named kernel (profiles/gemv_gateup_dory_full.md),
+# valid only for the source it was taken on (sha256 prefix of the file).
+NCU_TRAFFIC = {
+    "gemv_gateup": ("looped_ngpt_b200/csrc/k_gemv.cu", "dbf0351c20ec961b",
+                    (104.955136 + 3.734272) * 1e6),
+}
+
+
+def dram_traffic(kernel):
+    import hashlib
+    entry = NCU_TRAFFIC.get(kernel)
+    if not entry:
+        return None
+    path, sha, nbytes = entry
+    try:
+        with open(os.path.join(ROOT, path), "rb") as f:
+            cur = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return nbytes if cur == sha else None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -505,7 +528,7 @@ def main():
                    "l2": "no flush: 12 GB of weights streamed per token > L2"},
         "roofline": {"bound": bound, "kernel": dom, "achieved": achieved,
                      "peak": peak, "unit": unit, "frac": achieved / peak,
-                     "peak_source": r["peak_kind"], "traffic": None,
+                     "peak_source": r["peak_kind"], "traffic": dram_traffic(dom),
                      "share_of_step": d["ms"] / total_ms},
         "cpu_baseline": cpu,
         "e2e": {"value": world * K / e2e_dt, "unit": "tok/s",
