@@ -2,17 +2,19 @@
 // projections: C[M, N] = A[M, K] * W[N, K]^T (f32 accumulate), A the bf16
 // activations (row stride lda), W the bf16 weights, both K-contiguous.
 //
-// One CTA computes a 128 x 256 output tile:
+// Persistent CTAs (one per SM at most) walk 128 x 256 output tiles:
 //   warp 0 lane 0  streams 128x64 A and 256x64 W tiles with 2-D TMA loads
 //                  (128-byte swizzle) into a ring of STAGES shared-memory
-//                  stages (full/empty mbarriers);
+//                  stages (full/empty mbarriers), across tile boundaries;
 //   warp 1 lane 0  issues tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256,
-//                  K=16; 4 per stage) into a 256-column f32 TMEM accumulator
-//                  and releases each stage with tcgen05.commit;
-//   warps 0-3      wait for the accumulator, read it with tcgen05.ld
-//                  (warp w owns TMEM lanes 32w..32w+31 = tile rows) and run
-//                  the epilogue (f32 store, optional per-column scale, or the
-//                  SwiGLU pairing of gate/up column halves).
+//                  K=16; 4 per stage) into one of two 256-column f32 TMEM
+//                  accumulators and releases each stage with tcgen05.commit;
+//   warps 2-5      wait for a finished accumulator, read it with tcgen05.ld
+//                  (warp w owns TMEM lanes 32 (w % 4) .. + 31 = tile rows),
+//                  run the epilogue (f32 store, optional per-column scale,
+//                  the SwiGLU pairing of gate/up column halves, or the QKV
+//                  head epilogue) and hand the buffer back to the MMA warp,
+//                  so epilogues overlap the next tile's MMAs.
 // Every mbarrier wait is bounded: on timeout the CTA records ERRBIT_TIMEOUT,
 // waits (bounded) for its outstanding copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
@@ -227,33 +229,64 @@ __device__ __forceinline__ void qkv_epilogue(const TcArgs& a, int item,
   }
 }
 
+// Persistent tile loop: a grid of at most one CTA per SM walks the output
+// tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...  Tiles are numbered in
+// groups of kGroupN column tiles: inside a group the column tile varies
+// fastest, then the row tile, so the ~gridDim.x tiles in flight share a few
+// row blocks of A and kGroupN column blocks of W, both of which stay in L2.
+// Six warps: warp 0 (one lane) streams A/W stages with TMA, warp 1 (one
+// lane) issues the MMAs, warps 2-5 run the epilogue.  The accumulator is
+// double-buffered in TMEM (2 x 256 columns), so the epilogue of tile i
+// overlaps the MMAs of tile i + 1.
+constexpr int kGroupN = 8;
+constexpr int kEpiWarps = 4;
+constexpr int kGemmThreads = 32 * (2 + kEpiWarps);
+constexpr int kAccCols = 256;                 // columns per accumulator buffer
+
+struct TileGrid {
+  int mt, nt;                                 // row / column tiles
+  __device__ __forceinline__ int count() const { return mt * nt; }
+  __device__ __forceinline__ void at(int t, int& m, int& n) const {
+    const int per = kGroupN * mt;             // tiles per column group
+    const int g = t / per, r = t - g * per;
+    const int gw = min(kGroupN, nt - g * kGroupN);   // width of this group
+    m = r / gw;
+    n = g * kGroupN + (r - m * gw);
+  }
+};
+
 // TN: tile columns (MMA N): 256 for TC_PLAIN / TC_SWIGLU, hd for TC_QKV.
 template <int MODE, int TN>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
-               const __grid_constant__ CUtensorMap tmB, const TcArgs a) {
+               const __grid_constant__ CUtensorMap tmB, const TcArgs a,
+               const TileGrid tg) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment of the swizzled tiles (shared-window address)
   const uint32_t raw = su32(smem_raw);
   uint8_t* base = smem_raw + ((1024 - (raw & 1023)) & 1023);
   uint8_t* sA = base;
   uint8_t* sB = base + STAGES * kStageA;
-  __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], accum;
+  __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES];
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
   __shared__ uint32_t tmem_base;
   __shared__ int s_fail, s_issued;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM;
   constexpr int OUTC = MODE == TC_SWIGLU ? TN / 2 : TN;   // output columns
-  const int n0 = blockIdx.x * OUTC;
   const int KB = a.K / BK;
   constexpr uint32_t kB = (uint32_t)TN * BK * 2;          // B bytes per stage
+  volatile int* fail = &s_fail;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(full + i, 1);
       mbar_init(empty + i, 1);
     }
-    mbar_init(&accum, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(acc_full + i, 1);
+      mbar_init(acc_empty + i, kEpiWarps);
+    }
+    mbar_init(&mma_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
@@ -264,7 +297,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     asm volatile(
         "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
             su32(&tmem_base)),
-        "r"(kTmemCols)
+        "r"(2 * kAccCols)
         : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::
                      : "memory");
@@ -275,119 +308,162 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   const uint32_t tmem = tmem_base;
   pdl_wait();
   pdl_trigger();
+  const int ntiles = tg.count();
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ---- TMA producer ----------------------------------------------------
-    for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % STAGES, use = kb / STAGES;
-      if (use > 0 && !mbar_wait(empty + s, (uint32_t)((use - 1) & 1))) {
-        atomicOr(&s_fail, 1);
-        break;
+    if (lane == 0) {
+      int g = 0;                                // stage counter over all tiles
+      for (int t = blockIdx.x; t < ntiles && !*fail; t += gridDim.x) {
+        int mi, ni;
+        tg.at(t, mi, ni);
+        const int m0 = mi * BM, n0 = ni * OUTC;
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          const int s = g % STAGES, use = g / STAGES;
+          if (use > 0 && !mbar_wait(empty + s, (uint32_t)((use - 1) & 1))) {
+            atomicOr(&s_fail, 1);
+            break;
+          }
+          mbar_expect_tx(full + s, kStageA + kB);
+          tma_load_2d(sA + s * kStageA, &tmA, kb * BK, m0, full + s);
+          if (MODE == TC_QKV) {
+            tma_load_2d(sB + s * kStageB, &tmB, kb * BK, ni * TN, full + s);
+          } else {
+            const int nb1 = MODE == TC_SWIGLU ? a.up_off + n0 : n0 + TN / 2;
+            tma_load_2d(sB + s * kStageB, &tmB, kb * BK, n0, full + s);
+            tma_load_2d(sB + s * kStageB + kB / 2, &tmB, kb * BK, nb1, full + s);
+          }
+          s_issued = g + 1;
+        }
       }
-      mbar_expect_tx(full + s, kStageA + kB);
-      tma_load_2d(sA + s * kStageA, &tmA, kb * BK, m0, full + s);
-      if (MODE == TC_QKV) {
-        tma_load_2d(sB + s * kStageB, &tmB, kb * BK, blockIdx.x * TN, full + s);
-      } else {
-        const int nb1 = MODE == TC_SWIGLU ? a.up_off + n0 : n0 + TN / 2;
-        tma_load_2d(sB + s * kStageB, &tmB, kb * BK, n0, full + s);
-        tma_load_2d(sB + s * kStageB + kB / 2, &tmB, kb * BK, nb1, full + s);
-      }
-      s_issued = kb + 1;
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---- MMA issuer ------------------------------------------------------
-    constexpr uint32_t idesc = idesc_bf16(BM, TN);
-    for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % STAGES, use = kb / STAGES;
-      if (!mbar_wait(full + s, (uint32_t)(use & 1))) {
-        atomicOr(&s_fail, 1);
+  } else if (warp == 1) {
+    // ---- MMA issuer --------------------------------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(BM, TN);
+      int g = 0, i = 0;
+      for (int t = blockIdx.x; t < ntiles && !*fail; t += gridDim.x, ++i) {
+        const int buf = i & 1, ub = i >> 1;
+        // the epilogue has drained this accumulator buffer (tile i - 2)
+        if (ub > 0 && !mbar_wait(acc_empty + buf, (uint32_t)((ub - 1) & 1))) {
+          atomicOr(&s_fail, 1);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + buf * kAccCols;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          const int s = g % STAGES, use = g / STAGES;
+          if (!mbar_wait(full + s, (uint32_t)(use & 1))) {
+            atomicOr(&s_fail, 1);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = su32(sA + s * kStageA), b0 = su32(sB + s * kStageB);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16(acc, smem_desc(a0 + kk * 32), smem_desc(b0 + kk * 32), idesc,
+                      (kb | kk) != 0);
+          umma_commit(empty + s);                 // stage free once read
+        }
+        umma_commit(acc_full + buf);              // this tile's accumulator
+        if (!ok) break;
+      }
+      // every MMA issued so far has completed once this arrives
+      umma_commit(&mma_done);
+    }
+  } else {
+    // ---- epilogue warps: TMEM -> registers -> global -------------------
+    const int q = warp & 3;                       // TMEM lane quarter
+    int i = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+      const int buf = i & 1, ub = i >> 1;
+      const bool got = !*fail && mbar_wait(acc_full + buf, (uint32_t)(ub & 1));
+      if (!got) {
+        if (lane == 0) atomicOr(&s_fail, 1);
         break;
       }
       tc_fence_after();
-      const uint32_t a0 = su32(sA + s * kStageA), b0 = su32(sB + s * kStageB);
+      int mi, ni;
+      tg.at(t, mi, ni);
+      const int m0 = mi * BM, n0 = ni * OUTC;
+      const int row = m0 + q * 32 + lane;
+      const uint32_t trow = tmem + buf * kAccCols + ((uint32_t)(q * 32) << 16);
+      if (MODE == TC_PLAIN) {
+        for (int c0 = 0; c0 < TN; c0 += 32) {
+          float v[32];
+          tmem_ld32(trow + c0, v);
+          const int col = n0 + c0;
+          if (row < a.M && col < a.N) {
+            float* dst = a.C + (size_t)row * a.ldc + col;
+            if (a.col_scale) {
 #pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk)
-        umma_bf16(tmem, smem_desc(a0 + kk * 32), smem_desc(b0 + kk * 32), idesc,
-                  (kb | kk) != 0);
-      umma_commit(empty + s);                     // stage free once read
+              for (int k = 0; k < 32; ++k)
+                if (col + k < a.N) v[k] *= a.col_scale[col + k];
+            }
+            // 16-byte stores only when every row start stays 16-byte aligned
+            if (col + 32 <= a.N && (a.ldc & 3) == 0) {
+#pragma unroll
+              for (int k = 0; k < 32; k += 4)
+                *reinterpret_cast<float4*>(dst + k) =
+                    make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+            } else {
+              for (int k = 0; k < 32 && col + k < a.N; ++k) dst[k] = v[k];
+            }
+          }
+        }
+      } else if (MODE == TC_SWIGLU) {
+        for (int c0 = 0; c0 < TN / 2; c0 += 32) {
+          float gt[32], u[32];
+          tmem_ld32(trow + c0, gt);
+          tmem_ld32(trow + TN / 2 + c0, u);
+          const int col = n0 + c0;
+          if (row < a.M && col < a.N) {
+            bf16* dst = a.Cb + (size_t)row * a.ldc + col;
+            if (col + 32 <= a.N && (a.ldc & 1) == 0) {
+#pragma unroll
+              for (int k = 0; k < 32; k += 2)
+                *reinterpret_cast<__nv_bfloat162*>(dst + k) = __floats2bfloat162_rn(
+                    gt[k] * sigmoidf_(gt[k]) * u[k],
+                    gt[k + 1] * sigmoidf_(gt[k + 1]) * u[k + 1]);
+            } else {
+              for (int k = 0; k < 32 && col + k < a.N; ++k)
+                dst[k] = __float2bfloat16_rn(gt[k] * sigmoidf_(gt[k]) * u[k]);
+            }
+          }
+        }
+      } else {
+        float v[TN];
+#pragma unroll
+        for (int c0 = 0; c0 < TN; c0 += 32) {
+          float t32[32];
+          tmem_ld32(trow + c0, t32);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[c0 + k] = t32[k];
+        }
+        if (row < a.M) qkv_epilogue<TN>(a, ni, row, v);
+      }
+      // this warp's lanes are read: the buffer may take tile i + 2
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0)
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(
+                         su32(acc_empty + buf))
+                     : "memory");
     }
-    // accumulator complete (also after a failed wait: the commit then
-    // tracks the MMAs already issued, so teardown can wait for them)
-    umma_commit(&accum);
   }
-  __syncwarp();
-
-  // ---- epilogue: TMEM -> registers -> global ------------------------------
-  const bool got = mbar_wait(&accum, 0);
-  if (!got && lane == 0) atomicOr(&s_fail, 1);
-  tc_fence_after();
   __syncthreads();
-  const bool failed = *(volatile int*)&s_fail != 0;
-  if (!failed) {
-    const int row = m0 + warp * 32 + lane;
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-    if (MODE == TC_PLAIN) {
-      for (int c0 = 0; c0 < TN; c0 += 32) {
-        float v[32];
-        tmem_ld32(trow + c0, v);
-        const int col = n0 + c0;
-        if (row < a.M && col < a.N) {
-          float* dst = a.C + (size_t)row * a.ldc + col;
-          if (a.col_scale) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (col + i < a.N) v[i] *= a.col_scale[col + i];
-          }
-          // 16-byte stores only when every row start stays 16-byte aligned
-          if (col + 32 <= a.N && (a.ldc & 3) == 0) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(dst + i) =
-                  make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-          } else {
-            for (int i = 0; i < 32 && col + i < a.N; ++i) dst[i] = v[i];
-          }
-        }
-      }
-    } else if (MODE == TC_SWIGLU) {
-      for (int c0 = 0; c0 < TN / 2; c0 += 32) {
-        float g[32], u[32];
-        tmem_ld32(trow + c0, g);
-        tmem_ld32(trow + TN / 2 + c0, u);
-        const int col = n0 + c0;
-        if (row < a.M && col < a.N) {
-          bf16* dst = a.Cb + (size_t)row * a.ldc + col;
-          if (col + 32 <= a.N && (a.ldc & 1) == 0) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 2)
-              *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(
-                  g[i] * sigmoidf_(g[i]) * u[i],
-                  g[i + 1] * sigmoidf_(g[i + 1]) * u[i + 1]);
-          } else {
-            for (int i = 0; i < 32 && col + i < a.N; ++i)
-              dst[i] = __float2bfloat16_rn(g[i] * sigmoidf_(g[i]) * u[i]);
-          }
-        }
-      }
-    } else {
-      float v[TN];
-#pragma unroll
-      for (int c0 = 0; c0 < TN; c0 += 32) {
-        float t32[32];
-        tmem_ld32(trow + c0, t32);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[c0 + i] = t32[i];
-      }
-      if (row < a.M) qkv_epilogue<TN>(a, blockIdx.x, row, v);
-    }
-  } else if (threadIdx.x == 0) {
-    // give in-flight copies and MMAs a bounded chance to land before the
+  if (threadIdx.x == 0) {
+    // the MMAs (and, after a failure, the copies) must be done before the
     // shared memory and TMEM are released
-    atomicOr(a.err, ERRBIT_TIMEOUT);
-    const int hi = s_issued, lo = hi > STAGES ? hi - STAGES : 0;
-    for (int kb = lo; kb < hi; ++kb)
-      if (!mbar_wait(full + kb % STAGES, (uint32_t)((kb / STAGES) & 1))) break;
+    if (!mbar_wait(&mma_done, 0)) atomicOr(&s_fail, 1);
+    if (*fail) {
+      atomicOr(a.err, ERRBIT_TIMEOUT);
+      const int hi = s_issued, lo = hi > STAGES ? hi - STAGES : 0;
+      for (int g = lo; g < hi; ++g)
+        if (!mbar_wait(full + g % STAGES, (uint32_t)((g / STAGES) & 1))) break;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -395,7 +471,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(
                      tmem),
-                 "r"(kTmemCols)
+                 "r"(2 * kAccCols)
                  : "memory");
   }
 }
@@ -453,9 +529,21 @@ int* g_err_ptr = nullptr;
 
 size_t tc_smem() { return (size_t)STAGES * (kStageA + kStageB) + 1024; }
 
+int num_sms() {
+  static int n = [] {
+    int dev = 0, v = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    return v > 0 ? v : 1;
+  }();
+  return n;
+}
+
+// tiles: row tiles x column tiles of the output; one persistent CTA per SM
+// at most
 template <int MODE, int TN>
 bool launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const TcArgs& a,
-               dim3 grid, cudaStream_t st) {
+               int mt, int nt, cudaStream_t st) {
   static bool configured = false;
   if (!configured) {
     cudaFuncSetAttribute(gemm_tc_kernel<MODE, TN>,
@@ -463,8 +551,11 @@ bool launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const TcArgs& a,
                          (int)tc_smem());
     configured = true;
   }
-  return launch_k(gemm_tc_kernel<MODE, TN>, grid, dim3(128), tc_smem(), st, ma,
-                  mb, a) == cudaSuccess;
+  const TileGrid tg{mt, nt};
+  const int tiles = mt * nt;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  return launch_k(gemm_tc_kernel<MODE, TN>, dim3(grid), dim3(kGemmThreads),
+                  tc_smem(), st, ma, mb, a, tg) == cudaSuccess;
 }
 
 TcArgs base_args(int M, int N, int K) {
@@ -493,8 +584,7 @@ void launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
   a.C = C;
   a.ldc = ldc;
   a.col_scale = col_scale;
-  launch_tc<TC_PLAIN, BN>(ma, mb, a, dim3((N + BN - 1) / BN, (M + BM - 1) / BM),
-                          st);
+  launch_tc<TC_PLAIN, BN>(ma, mb, a, (M + BM - 1) / BM, (N + BN - 1) / BN, st);
 }
 
 // m[M, F] = silu(A W_g^T) * (A W_u^T) (bf16) with W = [W_g; W_u] of 2F rows.
@@ -509,8 +599,7 @@ void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
   a.up_off = F;
   a.Cb = m;
   a.ldc = ldm;
-  launch_tc<TC_SWIGLU, BN>(ma, mb, a,
-                           dim3((F + BN / 2 - 1) / (BN / 2), (M + BM - 1) / BM),
+  launch_tc<TC_SWIGLU, BN>(ma, mb, a, (M + BM - 1) / BM, (F + BN / 2 - 1) / (BN / 2),
                            st);
 }
 
@@ -539,11 +628,11 @@ void launch_gemm_qkv(const bf16* A, int lda, const bf16* W, const QkvGemmArgs& q
   a.g = q.g;
   a.q_out = q.q_out;
   a.gate_out = q.gate_out;
-  const dim3 grid(rows / hd, (q.M + BM - 1) / BM);
+  const int mt = (q.M + BM - 1) / BM, nt = rows / hd;
   switch (hd) {
-    case 64: launch_tc<TC_QKV, 64>(ma, mb, a, grid, st); break;
-    case 128: launch_tc<TC_QKV, 128>(ma, mb, a, grid, st); break;
-    default: launch_tc<TC_QKV, 160>(ma, mb, a, grid, st); break;
+    case 64: launch_tc<TC_QKV, 64>(ma, mb, a, mt, nt, st); break;
+    case 128: launch_tc<TC_QKV, 128>(ma, mb, a, mt, nt, st); break;
+    default: launch_tc<TC_QKV, 160>(ma, mb, a, mt, nt, st); break;
   }
 }
 
