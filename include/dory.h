@@ -218,6 +218,17 @@ int dory_decode_step_static(dory_model* m, dory_cache* c,
 int dory_debug_gemm_bf16(const void* d_A, int lda, const void* d_W,
                          float* d_C, int M, int N, int K, void* stream);
 
+/* The same GEMM with the K split that decode batches use when the output has
+ * fewer 128 x 256 tiles than the GPU has SMs: d_C holds max_splits slabs of
+ * [M, N] f32, split z writes its partial sum over its K range to slab z, and
+ * *n_partials (host) receives the number of slabs written; their sum is
+ * A W^T.  Without a split (*n_partials = 1) slab 0 holds the product.
+ * Errors as dory_debug_gemm_bf16, DORY_ERR_ARG also for max_splits < 1 or a
+ * null n_partials. */
+int dory_debug_gemm_bf16_split(const void* d_A, int lda, const void* d_W,
+                               float* d_C, int M, int N, int K, int max_splits,
+                               int* n_partials, void* stream);
+
 /* Test access to the in-register weight decode of quantised models: write
  * rows [row0, row0 + nrows) of block projection `tensor` (e.g.
  * "blk3.w_gu") as f32 [nrows, K] to d_out: e4m3(q) * 2^(s - 127) (MXFP8) or

@@ -58,6 +58,8 @@ SIGNATURES = {
                                         _P, _P]),
     "dory_debug_gemm_bf16": (c_int, [_P, c_int, _P, _P, c_int, c_int, c_int,
                                      _P]),
+    "dory_debug_gemm_bf16_split": (c_int, [_P, c_int, _P, _P, c_int, c_int,
+                                           c_int, c_int, POINTER(c_int), _P]),
     "dory_debug_dequant": (c_int, [_P, c_char_p, c_int, c_int, _P, _P]),
     "dory_copy_state": (c_int, [_P, _P, c_int, c_int, c_int, _P, _P]),
     "dory_sync_status": (c_int, [_P, _P]),

@@ -97,6 +97,7 @@ struct dory_cache {
   int* d_block_table;
   std::vector<int> slot_base;   // per block: first entry in `slots`
   std::vector<KVSlot> slots;
+  std::vector<CUtensorMap> kv_maps;   // per slot: TMA maps of K, then V
 };
 
 namespace {
@@ -124,7 +125,9 @@ CacheLayout cache_layout(const dory_model* m, int B, int max_ctx,
   CacheLayout L;
   const Dims& dm = m->dm;
   L.pages_per_seq = (max_ctx + kPage - 1) / kPage;
-  L.swa_cap = std::min(max_ctx, dm.window + max_chunk - 1);
+  // a multiple of the decode-attention tile, so that no tile wraps the ring
+  const int tr = kv_tile_rows();
+  L.swa_cap = (std::min(max_ctx, dm.window + max_chunk - 1) + tr - 1) / tr * tr;
   L.header = 256;
   L.table = align256((size_t)B * L.pages_per_seq * sizeof(int));
   size_t off = L.header + L.table;
@@ -159,6 +162,10 @@ struct WS {
 };
 
 constexpr int kMaxS = 8;
+// K-split partial slabs of the f32 projection outputs (qkvg, h): decode
+// batches that go through the tensor-core GEMM (one row tile) split K up
+// to 16 ways; the GEMV splits at most kMaxS ways.
+int slabs_of(size_t M, int T) { return T == 1 && M <= 128 ? 16 : kMaxS; }
 constexpr int kArgmaxSlots = 2048;
 
 WS ws_layout(const dory_model* m, int B, int T, char* base) {
@@ -176,11 +183,11 @@ WS ws_layout(const dory_model* m, int B, int T, char* base) {
   w.sfin = (float*)take(M * dm.d * 4);
   w.x = (float*)take(M * dm.d * 4);
   w.s_bf = (bf16*)take(M * dm.d * 2);
-  w.qkvg = (float*)take(kMaxS * M * dm.rows_qkvg * 4);
+  w.qkvg = (float*)take(slabs_of(M, T) * M * dm.rows_qkvg * 4);
   w.qb = (bf16*)take(M * dm.qdim * 2);
   w.gate = (float*)take(M * dm.qdim * 4);
   w.a = (bf16*)take(M * dm.qdim * 2);
-  w.h = (float*)take(kMaxS * M * dm.d * 4);
+  w.h = (float*)take(slabs_of(M, T) * M * dm.d * 4);
   w.mact = (bf16*)take(M * dm.F * 2);
   w.part_o = (float*)take((size_t)B * dm.Hq * kMaxSplits * dm.hd * 4);
   w.part_ml = (float*)take((size_t)B * dm.Hq * kMaxSplits * 2 * 4);
@@ -408,9 +415,22 @@ int dory_kv_cache_bind(dory_model* m, void* d_buf, int64_t bytes, int batch,
   c->d_nctx = (int*)base;
   c->d_block_table = (int*)(base + L.header);
   c->slot_base = L.base;
-  for (size_t i = 0; i < L.k_off.size(); ++i)
-    c->slots.push_back(KVSlot{(bf16*)(base + L.k_off[i]),
-                              (bf16*)(base + L.v_off[i]), L.ring[i], L.cap[i]});
+  for (size_t i = 0; i < L.k_off.size(); ++i) {
+    const KVSlot kv{(bf16*)(base + L.k_off[i]), (bf16*)(base + L.v_off[i]),
+                    L.ring[i], L.cap[i]};
+    c->slots.push_back(kv);
+    // rows of the [rows][hd] view: ring slots, or every page's rows
+    const long rows = kv.ring ? (long)batch * m->dm.Hkv * kv.cap
+                              : (long)batch * L.pages_per_seq * m->dm.Hkv * kPage;
+    CUtensorMap mk, mv;
+    if (!make_kv_tile_map(&mk, kv.K, rows, m->dm.hd) ||
+        !make_kv_tile_map(&mv, kv.V, rows, m->dm.hd)) {
+      delete c;
+      return DORY_ERR_CUDA;
+    }
+    c->kv_maps.push_back(mk);
+    c->kv_maps.push_back(mv);
+  }
   launch_cache_init(c->d_nctx, c->d_block_table, batch, L.pages_per_seq,
                     (cudaStream_t)stream);
   if (cudaGetLastError() != cudaSuccess) { delete c; return DORY_ERR_CUDA; }
@@ -456,7 +476,9 @@ void dory_cache_free(dory_cache* c) {
 int dory_workspace_bytes(const dory_model* m, int batch, int max_chunk,
                          int64_t* bytes) {
   if (!m || !bytes || batch < 1 || max_chunk < 1) return DORY_ERR_ARG;
-  *bytes = (int64_t)ws_layout(m, batch, max_chunk, nullptr).total;
+  // decode calls (T = 1) lay out more K-split slabs per row
+  *bytes = (int64_t)std::max(ws_layout(m, batch, max_chunk, nullptr).total,
+                             ws_layout(m, batch, 1, nullptr).total);
   return DORY_OK;
 }
 
@@ -524,13 +546,15 @@ int gemv_run(dory_model* m, const GemvArgs& g0, cudaStream_t st,
   return g.S;
 }
 
-void gemm_run(dory_model* m, const bf16* A, int lda, const bf16* W, float* C,
-              int ldc, int M, int N, int K, const float* scale,
-              cudaStream_t st, const char* name) {
+// Returns the number of K-split partials written (C + z * M * ldc).
+int gemm_run(dory_model* m, const bf16* A, int lda, const bf16* W, float* C,
+             int ldc, int M, int N, int K, const float* scale,
+             cudaStream_t st, const char* name, int max_splits = 1) {
   Prof p(m, st, name,
          (double)M * K * 2 + (double)N * K * 2 + (double)M * N * 4,
          2.0 * M * N * K);
-  launch_gemm_bf16(A, lda, W, C, ldc, M, N, K, scale, st);
+  return launch_gemm_bf16(A, lda, W, C, ldc, M, N, K, scale, st, max_splits,
+                          (long)M * ldc);
 }
 
 struct CallCtx {
@@ -544,10 +568,13 @@ struct CallCtx {
   cudaStream_t st;
 };
 
-KVSlot slot_for(const dory_cache* c, int i, int t) {
+int slot_index(const dory_cache* c, int i, int t) {
   int idx = c->slot_base[i];
   if (is_rec(c->m, i) && c->kv_mode == DORY_KV_PER_LOOP) idx += t - 1;
-  return c->slots[idx];
+  return idx;
+}
+KVSlot slot_for(const dory_cache* c, int i, int t) {
+  return c->slots[slot_index(c, i, t)];
 }
 
 bool use_gemv(int B, int T) { return T == 1 && B <= 8; }
@@ -577,6 +604,7 @@ void enqueue_forward(const CallCtx& x) {
   float* other = w.s1;
   const float* prev_alpha = nullptr;
   int prev_S = 1;
+  const int slabs = slabs_of(x.M, x.T);       // K-split partials that fit
 
   std::vector<std::pair<int, int>> order;
   for (int i = 0; i < m->n_in; ++i) order.push_back({i, 0});
@@ -611,10 +639,12 @@ void enqueue_forward(const CallCtx& x) {
       if (k > 0) {
         Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
         launch_update_rows(cur, w.h, prev_alpha, other, w.s_bf, w.x, rj, x.M,
-                           dm.d, x.st);
+                           dm.d, x.st, prev_S);
         std::swap(cur, other);
       }
       if (x.T == 1) {
+        // one partial: every attention block re-reads the q/k/v rows of its
+        // KV head, so K-split partials would multiply that traffic
         gemm_run(m, w.s_bf, dm.d, bw.w_qkvg, w.qkvg, dm.rows_qkvg, x.M,
                  dm.rows_qkvg, dm.d, nullptr, x.st, "gemm_qkvg");
       } else {
@@ -643,7 +673,7 @@ void enqueue_forward(const CallCtx& x) {
       Prof p(m, x.st, "attn_decode",
              x.B * (dm.Hkv * nk * dm.hd * 4.0 + S_qkvg * dm.rows_qkvg * 4.0),
              4.0 * x.B * dm.Hq * nk * dm.hd);
-      launch_attn_decode_fused(da, x.st);
+      launch_attn_decode(da, &x.c->kv_maps[2 * slot_index(x.c, i, t)], x.st);
     } else {
       AttnArgs aa{};
       aa.q = w.qb; aa.gate = w.gate; aa.B = x.B; aa.T = x.T; aa.dm = dm;
@@ -669,8 +699,8 @@ void enqueue_forward(const CallCtx& x) {
       g.pro = PRO_BF16; g.xin = w.a; g.xin_stride = dm.qdim;
       S_o = gemv_run(m, g, x.st, "gemv_o", &bw.m_o);
     } else {
-      gemm_run(m, w.a, dm.qdim, bw.w_o, w.h, dm.d, x.M, dm.d, dm.qdim, nullptr,
-               x.st, "gemm_o");
+      S_o = gemm_run(m, w.a, dm.qdim, bw.w_o, w.h, dm.d, x.M, dm.d, dm.qdim,
+                     nullptr, x.st, "gemm_o", slabs);
     }
 
     // ---- MLP sublayer ---------------------------------------------------
@@ -691,7 +721,7 @@ void enqueue_forward(const CallCtx& x) {
       {
         Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
         launch_update_rows(cur, w.h, bw.alpha_a, other, w.s_bf, w.x, RJ_NONE,
-                           x.M, dm.d, x.st);
+                           x.M, dm.d, x.st, S_o);
       }
       std::swap(cur, other);
       {
@@ -702,9 +732,8 @@ void enqueue_forward(const CallCtx& x) {
         launch_gemm_swiglu(w.s_bf, dm.d, bw.w_gu, w.mact, dm.F, x.M, dm.F, dm.d,
                            x.st);
       }
-      gemm_run(m, w.mact, dm.F, bw.w_down, w.h, dm.d, x.M, dm.d, dm.F, nullptr,
-               x.st, "gemm_down");
-      prev_S = 1;
+      prev_S = gemm_run(m, w.mact, dm.F, bw.w_down, w.h, dm.d, x.M, dm.d, dm.F,
+                        nullptr, x.st, "gemm_down", slabs);
     }
     prev_alpha = bw.alpha_m;
   }
@@ -730,7 +759,7 @@ void enqueue_forward(const CallCtx& x) {
     {
       Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
       launch_update_rows(cur, w.h, prev_alpha, w.sfin, w.s_bf, w.x, RJ_NONE,
-                         x.M, dm.d, x.st);
+                         x.M, dm.d, x.st, prev_S);
     }
     if (x.logits_all) {
       gemm_run(m, w.s_bf, dm.d, m->lm_head, x.logits, dm.V, x.M, dm.V, dm.d,
@@ -951,6 +980,20 @@ extern "C" int dory_debug_gemm_bf16(const void* d_A, int lda, const void* d_W,
   cudaGetLastError();
   launch_gemm_bf16((const bf16*)d_A, lda, (const bf16*)d_W, d_C, N, M, N, K,
                    nullptr, (cudaStream_t)stream);
+  return cudaGetLastError() == cudaSuccess ? DORY_OK : DORY_ERR_CUDA;
+}
+
+extern "C" int dory_debug_gemm_bf16_split(const void* d_A, int lda,
+                                          const void* d_W, float* d_C, int M,
+                                          int N, int K, int max_splits,
+                                          int* n_partials, void* stream) {
+  if (!d_A || !d_W || !d_C || !n_partials || M < 1 || N < 1 || K < 64 ||
+      K % 64 || lda < K || lda % 8 || max_splits < 1)
+    return DORY_ERR_ARG;
+  cudaGetLastError();
+  *n_partials = launch_gemm_bf16((const bf16*)d_A, lda, (const bf16*)d_W, d_C,
+                                 N, M, N, K, nullptr, (cudaStream_t)stream,
+                                 max_splits, (long)M * N);
   return cudaGetLastError() == cudaSuccess ? DORY_OK : DORY_ERR_CUDA;
 }
 

@@ -1,6 +1,7 @@
 // Internal interface between the C-ABI host layer (dory_api.cu) and the
 // sm_100a kernels.  Not installed; not part of the public ABI.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -25,6 +26,29 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// The same with thread-block clusters of cluster_x blocks along x (grid.x
+// a multiple of cluster_x).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k_cluster(void (*kernel)(KArgs...), dim3 grid,
+                                    dim3 block, size_t smem, cudaStream_t st,
+                                    int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster_x;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -138,7 +162,7 @@ void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
 // Prefill: s_new = N(s + alpha (N(h) - s)) per row (+ loop re-injection).
 void launch_update_rows(const float* s_in, const float* h, const float* alpha,
                         float* s_out, bf16* s_bf, float* x_buf, int reinject,
-                        int M, int d, cudaStream_t st);
+                        int M, int d, cudaStream_t st, int h_S = 1);
 // Final greedy argmax over [B][n] partials or full logits rows.
 void launch_argmax_partials(const float* val, const int* idx, int B, int n,
                             int* out, int* n_ctx, int T, cudaStream_t st);
@@ -185,14 +209,25 @@ struct DecAttnArgs {
   bf16* a_out;         // [B][qdim]
   int* err;
 };
-void launch_attn_decode_fused(const DecAttnArgs& a, cudaStream_t st);
+// kv_maps: the TMA maps of this layer slot's K and V (make_kv_tile_map).
+void launch_attn_decode(const DecAttnArgs& a, const CUtensorMap* kv_maps,
+                        cudaStream_t st);
+// Keys per decode-attention tile: ring capacities are multiples of it, and
+// it is the box height of the KV tensor maps.
+int kv_tile_rows();
+// 2-D TMA map over a K or V cache buffer viewed as [rows][hd] bf16 (rows =
+// ring slots or page rows), box kv_tile_rows() x 32 with the 64-byte swizzle.
+bool make_kv_tile_map(CUtensorMap* m, const void* ptr, long rows, int hd);
 
 // ---------------------------------------------------------------- GEMM ----
 // C[M, N] (f32, row stride ldc) = A[M, K] (bf16, row stride lda) * W[N, K]^T
-// optionally times col_scale[n], on tcgen05.  M, N any; K % 64 == 0.
-void launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
-                      int M, int N, int K, const float* col_scale,
-                      cudaStream_t st);
+// optionally times col_scale[n], on tcgen05.  M, N any; K % 64 == 0.  When
+// the output has fewer tiles than SMs (decode batches) and max_splits > 1,
+// K is split: split z writes its partial to C + z * slab.  Returns the number
+// of partials written (1 without a split).
+int launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
+                     int M, int N, int K, const float* col_scale,
+                     cudaStream_t st, int max_splits = 1, long slab = 0);
 // m[M, F] = silu(A W_g^T) * (A W_u^T) as bf16, W = [W_g; W_u] (2F rows).
 void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
                         int ldm, int M, int F, int K, cudaStream_t st);

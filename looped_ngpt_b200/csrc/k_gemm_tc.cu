@@ -20,11 +20,13 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdio>
 #include <map>
 #include <mutex>
 #include <utility>
 
+#include "async_copy.cuh"
 #include "common.cuh"
 
 namespace dory {
@@ -32,51 +34,8 @@ namespace dory {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int kTmemCols = 256;
 constexpr uint32_t kStageA = BM * BK * 2;     // 16 KB
 constexpr uint32_t kStageB = BN * BK * 2;     // 32 KB
-constexpr long kSpin = 1L << 22;    // bounded polls (~1 s)
-
-__device__ __forceinline__ uint32_t su32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* b, int n) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
-                   su32(b)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n"
-      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok)
-      : "r"(su32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
-  for (long i = 0; i < kSpin; ++i)
-    if (mbar_try(b, parity)) return true;
-  return false;
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map,
-                                            int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_"
-      "tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(su32(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(su32(bar))
-      : "memory");
-}
-
 // Shared-memory matrix descriptor of a K-major tile stored by TMA with the
 // 128-byte swizzle: rows of 64 bf16 (128 B), 8-row atoms 1024 B apart.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
@@ -154,6 +113,7 @@ struct TcArgs {
   float* C;             // TC_PLAIN: f32 out [M][ldc]
   bf16* Cb;             // TC_SWIGLU: bf16 out [M][ldc]
   int ldc;
+  long slab;            // TC_PLAIN with K splits: elements between partials
   const float* col_scale;
   int* err;
   // TC_QKV: one tile column = one head of the fused q/k/v/gate projection
@@ -242,11 +202,17 @@ constexpr int kGroupN = 8;
 constexpr int kEpiWarps = 4;
 constexpr int kGemmThreads = 32 * (2 + kEpiWarps);
 constexpr int kAccCols = 256;                 // columns per accumulator buffer
+constexpr int kSmallPair = 72;                // gate (= up) rows of a small-M SwiGLU tile
 
 struct TileGrid {
   int mt, nt;                                 // row / column tiles
-  __device__ __forceinline__ int count() const { return mt * nt; }
-  __device__ __forceinline__ void at(int t, int& m, int& n) const {
+  int ks, kbs;                                // K splits, K blocks per split
+  __device__ __forceinline__ int count() const { return mt * nt * ks; }
+  // work item t -> (row tile m, column tile n, K split z); the K split is
+  // the slowest index, so concurrent CTAs share the A rows of one split
+  __device__ __forceinline__ void at(int t, int& m, int& n, int& z) const {
+    z = t / (mt * nt);
+    t -= z * (mt * nt);
     const int per = kGroupN * mt;             // tiles per column group
     const int g = t / per, r = t - g * per;
     const int gw = min(kGroupN, nt - g * kGroupN);   // width of this group
@@ -315,10 +281,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     if (lane == 0) {
       int g = 0;                                // stage counter over all tiles
       for (int t = blockIdx.x; t < ntiles && !*fail; t += gridDim.x) {
-        int mi, ni;
-        tg.at(t, mi, ni);
+        int mi, ni, z;
+        tg.at(t, mi, ni, z);
         const int m0 = mi * BM, n0 = ni * OUTC;
-        for (int kb = 0; kb < KB; ++kb, ++g) {
+        const int kb0 = z * tg.kbs, kb1 = min(KB, kb0 + tg.kbs);
+        for (int kb = kb0; kb < kb1; ++kb, ++g) {
           const int s = g % STAGES, use = g / STAGES;
           if (use > 0 && !mbar_wait(empty + s, (uint32_t)((use - 1) & 1))) {
             atomicOr(&s_fail, 1);
@@ -351,8 +318,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         tc_fence_after();
         const uint32_t acc = tmem + buf * kAccCols;
+        const int kb0 = (t / (tg.mt * tg.nt)) * tg.kbs;
+        const int kb1 = min(KB, kb0 + tg.kbs);
         bool ok = true;
-        for (int kb = 0; kb < KB; ++kb, ++g) {
+        for (int kb = kb0; kb < kb1; ++kb, ++g) {
           const int s = g % STAGES, use = g / STAGES;
           if (!mbar_wait(full + s, (uint32_t)(use & 1))) {
             atomicOr(&s_fail, 1);
@@ -364,7 +333,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             umma_bf16(acc, smem_desc(a0 + kk * 32), smem_desc(b0 + kk * 32), idesc,
-                      (kb | kk) != 0);
+                      (kb - kb0 | kk) != 0);
           umma_commit(empty + s);                 // stage free once read
         }
         umma_commit(acc_full + buf);              // this tile's accumulator
@@ -385,8 +354,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         break;
       }
       tc_fence_after();
-      int mi, ni;
-      tg.at(t, mi, ni);
+      int mi, ni, z;
+      tg.at(t, mi, ni, z);
       const int m0 = mi * BM, n0 = ni * OUTC;
       const int row = m0 + q * 32 + lane;
       const uint32_t trow = tmem + buf * kAccCols + ((uint32_t)(q * 32) << 16);
@@ -396,7 +365,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           tmem_ld32(trow + c0, v);
           const int col = n0 + c0;
           if (row < a.M && col < a.N) {
-            float* dst = a.C + (size_t)row * a.ldc + col;
+            float* dst = a.C + z * a.slab + (size_t)row * a.ldc + col;
             if (a.col_scale) {
 #pragma unroll
               for (int k = 0; k < 32; ++k)
@@ -419,16 +388,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           tmem_ld32(trow + c0, gt);
           tmem_ld32(trow + TN / 2 + c0, u);
           const int col = n0 + c0;
-          if (row < a.M && col < a.N) {
+          // columns of this tile only (TN / 2 need not be a multiple of 32)
+          const int lim = min(32, min(OUTC - c0, a.N - col));
+          if (row < a.M && lim > 0) {
             bf16* dst = a.Cb + (size_t)row * a.ldc + col;
-            if (col + 32 <= a.N && (a.ldc & 1) == 0) {
+            if (lim == 32 && (a.ldc & 1) == 0) {
 #pragma unroll
               for (int k = 0; k < 32; k += 2)
                 *reinterpret_cast<__nv_bfloat162*>(dst + k) = __floats2bfloat162_rn(
                     gt[k] * sigmoidf_(gt[k]) * u[k],
                     gt[k + 1] * sigmoidf_(gt[k + 1]) * u[k + 1]);
             } else {
-              for (int k = 0; k < 32 && col + k < a.N; ++k)
+              for (int k = 0; k < lim; ++k)
                 dst[k] = __float2bfloat16_rn(gt[k] * sigmoidf_(gt[k]) * u[k]);
             }
           }
@@ -507,6 +478,23 @@ bool make_map(CUtensorMap* m, const void* ptr, long rows, long cols, long ld,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+}  // namespace
+
+bool make_kv_tile_map(CUtensorMap* m, const void* ptr, long rows, int hd) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)hd, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)hd * 2};
+  cuuint32_t box[2] = {32, (cuuint32_t)kv_tile_rows()};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+
 // Tensor maps of weights are built once per (pointer, shape, box).
 std::mutex g_map_mu;
 std::map<std::tuple<const void*, long, long, int>, CUtensorMap> g_maps;
@@ -543,7 +531,7 @@ int num_sms() {
 // at most
 template <int MODE, int TN>
 bool launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const TcArgs& a,
-               int mt, int nt, cudaStream_t st) {
+               int mt, int nt, cudaStream_t st, int ks = 1) {
   static bool configured = false;
   if (!configured) {
     cudaFuncSetAttribute(gemm_tc_kernel<MODE, TN>,
@@ -551,8 +539,10 @@ bool launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const TcArgs& a,
                          (int)tc_smem());
     configured = true;
   }
-  const TileGrid tg{mt, nt};
-  const int tiles = mt * nt;
+  const int KB = a.K / BK;
+  const int kbs = (KB + ks - 1) / ks;
+  const TileGrid tg{mt, nt, (KB + kbs - 1) / kbs, kbs};
+  const int tiles = mt * nt * tg.ks;
   const int grid = tiles < num_sms() ? tiles : num_sms();
   return launch_k(gemm_tc_kernel<MODE, TN>, dim3(grid), dim3(kGemmThreads),
                   tc_smem(), st, ma, mb, a, tg) == cudaSuccess;
@@ -572,19 +562,34 @@ TcArgs base_args(int M, int N, int K) {
 void set_tc_error_word(int* err) { g_err_ptr = err; }
 
 // C[M, N] = A[M, K] W[N, K]^T (f32, optional column scale) on tcgen05.
-void launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
-                      int M, int N, int K, const float* col_scale,
-                      cudaStream_t st) {
+// With max_splits > 1 and fewer output tiles than SMs, K is split so that
+// about one work item runs per SM: split z writes its f32 partial to
+// C + z * slab and the reader sums the partials.  Returns the split count.
+int launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
+                     int M, int N, int K, const float* col_scale,
+                     cudaStream_t st, int max_splits, long slab) {
   CUtensorMap ma, mb;
   if (!make_map(&ma, A, M, K, lda, BM) || !weight_map(&mb, W, N, K, 128)) {
     fprintf(stderr, "dory: tensor map creation failed\n");
-    return;
+    return 1;
   }
   TcArgs a = base_args(M, N, K);
   a.C = C;
   a.ldc = ldc;
+  a.slab = slab;
   a.col_scale = col_scale;
-  launch_tc<TC_PLAIN, BN>(ma, mb, a, (M + BM - 1) / BM, (N + BN - 1) / BN, st);
+  const int mt = (M + BM - 1) / BM, nt = (N + BN - 1) / BN;
+  const int KB = K / BK;
+  int ks = 1;
+  if (max_splits > 1 && !col_scale && mt * nt < num_sms()) {
+    // at least 2 K blocks per split keep the stage ring busy
+    ks = std::min(std::min(max_splits, num_sms() / (mt * nt)), KB / 2);
+    if (ks < 1) ks = 1;
+    const int kbs = (KB + ks - 1) / ks;
+    ks = (KB + kbs - 1) / kbs;                  // no empty split
+  }
+  launch_tc<TC_PLAIN, BN>(ma, mb, a, mt, nt, st, ks);
+  return ks;
 }
 
 // m[M, F] = silu(A W_g^T) * (A W_u^T) (bf16) with W = [W_g; W_u] of 2F rows.
@@ -599,8 +604,20 @@ void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
   a.up_off = F;
   a.Cb = m;
   a.ldc = ldm;
-  launch_tc<TC_SWIGLU, BN>(ma, mb, a, (M + BM - 1) / BM, (F + BN / 2 - 1) / (BN / 2),
-                           st);
+  const int mt = (M + BM - 1) / BM;
+  if (mt == 1 && (F + kSmallPair - 1) / kSmallPair <= num_sms()) {
+    // one row tile (decode batches): 72 gate + 72 up rows per tile, so that
+    // the F / 72 tiles (143 for F = 10240) give every SM one tile
+    CUtensorMap mb2;
+    if (!weight_map(&mb2, W, 2L * F, K, kSmallPair)) {
+      fprintf(stderr, "dory: tensor map creation failed\n");
+      return;
+    }
+    launch_tc<TC_SWIGLU, 2 * kSmallPair>(ma, mb2, a, mt,
+                                         (F + kSmallPair - 1) / kSmallPair, st);
+    return;
+  }
+  launch_tc<TC_SWIGLU, BN>(ma, mb, a, mt, (F + BN / 2 - 1) / (BN / 2), st);
 }
 
 // Fused q/k/v/gate projection with the RoPE / QK-norm / KV-write epilogue.

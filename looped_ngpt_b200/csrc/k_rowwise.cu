@@ -78,13 +78,14 @@ __global__ void embed_kernel(const int* tokens, const bf16* E, int d,
 __global__ void update_rows_kernel(const float* s_in, const float* h,
                                    const float* alpha, float* s_out,
                                    bf16* s_bf, float* x_buf, int reinject,
-                                   int d) {
+                                   int d, int h_S) {
   extern __shared__ float tmp[];
   __shared__ float red[7 * 32];
   pdl_wait();
   pdl_trigger();
   const size_t o = (size_t)blockIdx.x * d;
-  ngpt_update_row(s_in + o, h + o, 1, 0, alpha, d, reinject,
+  // h: h_S K-split partials of the sublayer output, gridDim.x rows apart
+  ngpt_update_row(s_in + o, h + o, h_S, (size_t)gridDim.x * d, alpha, d, reinject,
                   reinject == RJ_NONE ? nullptr : x_buf + o, s_out + o,
                   s_bf + o, tmp, red);
 }
@@ -214,9 +215,9 @@ void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
 
 void launch_update_rows(const float* s_in, const float* h, const float* alpha,
                         float* s_out, bf16* s_bf, float* x_buf, int reinject,
-                        int M, int d, cudaStream_t st) {
+                        int M, int d, cudaStream_t st, int h_S) {
   launch_k(update_rows_kernel, dim3(M), dim3(256), d * sizeof(float), st, s_in,
-           h, alpha, s_out, s_bf, x_buf, reinject, d);
+           h, alpha, s_out, s_bf, x_buf, reinject, d, h_S);
 }
 
 void launch_argmax_partials(const float* val, const int* idx, int B, int n,
