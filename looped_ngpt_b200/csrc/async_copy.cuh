@@ -47,6 +47,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity,
   return false;
 }
 
+// The same wait taken by a whole warp, with one outcome for all lanes (so
+// that .sync.aligned instructions after it see a converged warp).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* b, uint32_t parity,
+                                               long limit = kSpin) {
+  return __all_sync(0xffffffffu, mbar_wait(b, parity, limit));
+}
+
 // 2-D tiled TMA load of the box at element coordinates (x, y) of `map`
 // (x innermost; x times the element size must be a multiple of 16 bytes)
 // into shared memory, completing on `bar` (transaction bytes).

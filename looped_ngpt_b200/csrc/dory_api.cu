@@ -97,7 +97,8 @@ struct dory_cache {
   int* d_block_table;
   std::vector<int> slot_base;   // per block: first entry in `slots`
   std::vector<KVSlot> slots;
-  std::vector<CUtensorMap> kv_maps;   // per slot: TMA maps of K, then V
+  std::vector<CUtensorMap> kv_maps;   // per slot: decode maps of K, then V
+  std::vector<CUtensorMap> pf_maps;   // per slot: prefill maps K64, K32, V64, V32
 };
 
 namespace {
@@ -125,8 +126,9 @@ CacheLayout cache_layout(const dory_model* m, int B, int max_ctx,
   CacheLayout L;
   const Dims& dm = m->dm;
   L.pages_per_seq = (max_ctx + kPage - 1) / kPage;
-  // a multiple of the decode-attention tile, so that no tile wraps the ring
-  const int tr = kv_tile_rows();
+  // a multiple of the decode and prefill attention tiles (powers of two),
+  // so that no tile wraps the ring
+  const int tr = std::max(kv_tile_rows(), pf_tile_keys());
   L.swa_cap = (std::min(max_ctx, dm.window + max_chunk - 1) + tr - 1) / tr * tr;
   L.header = 256;
   L.table = align256((size_t)B * L.pages_per_seq * sizeof(int));
@@ -430,7 +432,22 @@ int dory_kv_cache_bind(dory_model* m, void* d_buf, int64_t bytes, int batch,
     }
     c->kv_maps.push_back(mk);
     c->kv_maps.push_back(mv);
+    CUtensorMap pm[4];
+    const int hd = m->dm.hd, tk = pf_tile_keys();
+    if (!make_map_2d(&pm[0], kv.K, rows, hd, hd, 64, tk) ||
+        !make_map_2d(&pm[1], kv.K, rows, hd, hd, 32, tk) ||
+        !make_map_2d(&pm[2], kv.V, rows, hd, hd, 64, tk) ||
+        !make_map_2d(&pm[3], kv.V, rows, hd, hd, 32, tk)) {
+      delete c;
+      return DORY_ERR_CUDA;
+    }
+    for (int k = 0; k < 4; ++k) c->pf_maps.push_back(pm[k]);
   }
+  // finite contents everywhere: attention tiles also cover rows that no
+  // token has written yet (their probabilities are 0, their values must not
+  // be NaN)
+  cudaMemsetAsync(base + L.header + L.table, 0, L.total - L.header - L.table,
+                  (cudaStream_t)stream);
   launch_cache_init(c->d_nctx, c->d_block_table, batch, L.pages_per_seq,
                     (cudaStream_t)stream);
   if (cudaGetLastError() != cudaSuccess) { delete c; return DORY_ERR_CUDA; }
@@ -689,7 +706,7 @@ void enqueue_forward(const CallCtx& x) {
       Prof p(m, x.st, "attn_prefill",
              x.B * (dm.Hkv * keys * dm.hd * 4.0) + x.M * dm.qdim * 10.0,
              4.0 * x.B * dm.Hq * vis * dm.hd);
-      launch_attn_prefill(aa, x.st);
+      launch_attn_prefill_tc(aa, &x.c->pf_maps[4 * slot_index(x.c, i, t)], x.st);
     }
     int S_o = 1;
     if (gemv) {

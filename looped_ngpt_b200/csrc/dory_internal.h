@@ -191,6 +191,21 @@ struct AttnArgs {
   int* err;
 };
 void launch_attn_prefill(const AttnArgs& a, cudaStream_t st);
+// The same on the tcgen05 tensor cores.  kv_maps: this layer slot's K and V
+// maps for 64-key tiles: K 64-dim boxes, K 32-dim boxes, V 64, V 32
+// (make_map_2d with box_rows = pf_tile_keys()).  Ring capacities must be
+// multiples of pf_tile_keys().
+void launch_attn_prefill_tc(const AttnArgs& a, const CUtensorMap* kv_maps,
+                            cudaStream_t st);
+int pf_tile_keys();
+// 2-D TMA map over a bf16 [rows][cols] matrix (row stride ld elements), box
+// box_rows x box_cols with box_cols 64 (128-byte swizzle) or 32 (64-byte).
+bool make_map_2d(CUtensorMap* m, const void* ptr, long rows, long cols,
+                 long ld, int box_cols, int box_rows);
+inline bool make_act_map(CUtensorMap* m, const void* ptr, long rows, long cols,
+                         int box_cols, int box_rows) {
+  return make_map_2d(m, ptr, rows, cols, cols, box_cols, box_rows);
+}
 
 // Decode (one token per sequence): RoPE/QK-norm/KV write, split-KV attention,
 // split merge and gate in one kernel.

@@ -346,7 +346,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
 
     for (int i = 0; i < ntile; ++i) {
       const int s = i % kStages;
-      if (!mbar_wait(full + s, (uint32_t)((i / kStages) & 1))) {
+      if (!mbar_wait_warp(full + s, (uint32_t)((i / kStages) & 1))) {
         atomicOr(&s_fail, 1);
         break;
       }

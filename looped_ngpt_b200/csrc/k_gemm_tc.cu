@@ -28,6 +28,7 @@
 
 #include "async_copy.cuh"
 #include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace dory {
 
@@ -39,70 +40,12 @@ constexpr uint32_t kStageB = BN * BK * 2;     // 32 KB
 // Shared-memory matrix descriptor of a K-major tile stored by TMA with the
 // 128-byte swizzle: rows of 64 bf16 (128 B), 8-row atoms 1024 B apart.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFF);        // start address
-  d |= (uint64_t)1 << 16;                        // leading byte offset (unused)
-  d |= (uint64_t)(1024 >> 4) << 32;              // stride byte offset
-  d |= (uint64_t)1 << 46;                        // descriptor version (sm_100)
-  d |= (uint64_t)2 << 61;                        // 128-byte swizzle
-  return d;
-}
-
-// Instruction descriptor, kind::f16: f32 accumulator, bf16 A and B, both
-// K-major, shape M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b,
-                                          uint32_t idesc, uint32_t accum) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accum)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 "
-      "[%0];" ::"r"(su32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  return make_sdesc(saddr, 16, 1024, kSw128);
 }
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-// 32 consecutive f32 columns of this thread's TMEM lane (load and wait in
-// one asm statement so no use of the registers can precede the wait).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,"
-      "%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,"
-      "%27,%28,%29,%30,%31}, [%32];\n"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
-        "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
-        "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
-        "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 enum TcMode : int { TC_PLAIN = 0, TC_SWIGLU = 1, TC_QKV = 2 };
@@ -259,15 +202,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     s_fail = 0;
     s_issued = 0;
   }
-  if (warp == 0) {
-    asm volatile(
-        "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-            su32(&tmem_base)),
-        "r"(2 * kAccCols)
-        : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::
-                     : "memory");
-  }
+  if (warp == 0) tmem_alloc(&tmem_base, 2 * kAccCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -440,10 +375,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(
-                     tmem),
-                 "r"(2 * kAccCols)
-                 : "memory");
+    tmem_free(tmem, 2 * kAccCols);
   }
 }
 
@@ -479,6 +411,21 @@ bool make_map(CUtensorMap* m, const void* ptr, long rows, long cols, long ld,
 }
 
 }  // namespace
+
+bool make_map_2d(CUtensorMap* m, const void* ptr, long rows, long cols,
+                 long ld, int box_cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn || (box_cols != 32 && box_cols != 64)) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 bool make_kv_tile_map(CUtensorMap* m, const void* ptr, long rows, int hd) {
   auto fn = encode_fn();
