@@ -113,14 +113,19 @@ int dory_init_weights(const dory_config* cfg, const dory_tensor* tensors,
  * per_loop mode) up to `max_loops` loops.  Layout: a small header, the full
  * attention layers as 64-token pages behind a block table, the
  * sliding-window layers as rings of min(max_ctx, window + max_chunk - 1)
- * positions.  In last_loop mode the size does not depend on max_loops. */
+ * positions rounded up to a multiple of 64 (the attention kernels' key
+ * tiles never wrap a ring).  In last_loop mode the size does not depend on
+ * max_loops. */
 int dory_kv_cache_bytes(const dory_model* m, int batch, int max_ctx,
                         int max_chunk, int max_loops, int kv_mode,
                         int64_t* bytes);
 
 /* Bind a caller-owned device buffer (>= dory_kv_cache_bytes, 256-byte
- * aligned) as an empty cache and enqueue its initialisation on `stream`.
- * The kv_mode is fixed for the life of the cache. */
+ * aligned) as an empty cache and enqueue its initialisation on `stream`:
+ * the length and block table are set and every K/V row is zeroed (attention
+ * tiles also read rows no token has written yet; their weights are 0 and
+ * their contents must be finite).  The kv_mode is fixed for the life of the
+ * cache. */
 int dory_kv_cache_bind(dory_model* m, void* d_buf, int64_t bytes, int batch,
                        int max_ctx, int max_chunk, int max_loops, int kv_mode,
                        void* stream, dory_cache** out);

@@ -155,11 +155,10 @@ CacheLayout cache_layout(const dory_model* m, int B, int max_ctx,
 
 
 struct WS {
-  float *s0, *s1, *sfin, *x, *qkvg, *gate, *h, *part_o, *part_ml, *lg,
+  float *s0, *s1, *sfin, *x, *qkvg, *gate, *h, *lg,
       *rope, *amax_val;
   bf16 *s_bf, *a, *mact, *qb;
   int* amax_idx;
-  int* counters;
   size_t total;
 };
 
@@ -191,12 +190,9 @@ WS ws_layout(const dory_model* m, int B, int T, char* base) {
   w.a = (bf16*)take(M * dm.qdim * 2);
   w.h = (float*)take(slabs_of(M, T) * M * dm.d * 4);
   w.mact = (bf16*)take(M * dm.F * 2);
-  w.part_o = (float*)take((size_t)B * dm.Hq * kMaxSplits * dm.hd * 4);
-  w.part_ml = (float*)take((size_t)B * dm.Hq * kMaxSplits * 2 * 4);
   w.rope = (float*)take((size_t)2 * T * (dm.hd / 2) * 2 * 4);
   w.amax_val = (float*)take((size_t)B * kArgmaxSlots * 4);
   w.amax_idx = (int*)take((size_t)B * kArgmaxSlots * 4);
-  w.counters = (int*)take((size_t)B * dm.Hkv * 4);
   w.lg = (float*)take(B > 8 ? (size_t)B * dm.V * 4 : 0);
   w.total = off;
   return w;
@@ -614,7 +610,7 @@ void enqueue_forward(const CallCtx& x) {
   {
     Prof p(m, x.st, "embed", (double)x.M * dm.d * 8, 0);
     launch_embed(x.tokens, m->embed, x.M, dm.d, w.s0, w.s_bf, m->d_status,
-                 dm.V, w.counters, x.B * dm.Hkv, x.T == 1 ? w.rope : nullptr,
+                 dm.V, x.T == 1 ? w.rope : nullptr,
                  geo.n_ctx, dm.hd, m->th_swa, m->th_full, x.st);
   }
   float* cur = w.s0;
@@ -683,8 +679,7 @@ void enqueue_forward(const CallCtx& x) {
       da.s_q = bw.s_q; da.s_k = bw.s_k;
       da.rope = w.rope + (full ? (size_t)half * 2 : 0);
       da.q_scale = q_scale; da.window = full ? 0 : dm.window;
-      da.kv = kv; da.g = geo; da.part_o = w.part_o; da.part_ml = w.part_ml;
-      da.counters = w.counters; da.a_out = w.a; da.err = m->d_status;
+      da.kv = kv; da.g = geo; da.a_out = w.a; da.err = m->d_status;
       const double nk = full ? x.n_ctx0 + 1.0
                              : std::min(x.n_ctx0 + 1.0, (double)dm.window);
       Prof p(m, x.st, "attn_decode",

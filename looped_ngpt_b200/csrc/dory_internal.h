@@ -59,7 +59,6 @@ enum : int {
 };
 
 constexpr int kPage = 64;           // tokens per page of a full-attention cache
-constexpr int kMaxSplits = 64;      // decode attention: key splits per head
 constexpr int kMaxHeadDim = 256;
 
 struct Dims {
@@ -152,13 +151,13 @@ void launch_dequant_rows(int fmt, const uint8_t* Wq, const uint8_t* Ws, int K,
 // RoPE cos/sin for positions n_ctx + t, t < T; table [2][T][hd/2][2].
 void launch_rope_table(float* table, const CacheGeo& g, int T, int hd,
                        double theta_swa, double theta_full, cudaStream_t st);
-// x0 = N(E[tok]) -> s (f32) and s_bf (bf16), rows M.
-// Block 0 also zeroes `counters` and, if rope != null (one-token calls),
-// writes the RoPE table [2][1][hd/2][2] for position n_ctx.
+// x0 = N(E[tok]) -> s (f32) and s_bf (bf16), rows M.  If rope != null
+// (one-token calls) also writes the RoPE table [2][1][hd/2][2] for position
+// n_ctx.
 void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
-                  bf16* s_bf, int* err, int vocab, int* counters,
-                  int n_counters, float* rope, const int* n_ctx, int hd,
-                  double theta_swa, double theta_full, cudaStream_t st);
+                  bf16* s_bf, int* err, int vocab, float* rope,
+                  const int* n_ctx, int hd, double theta_swa,
+                  double theta_full, cudaStream_t st);
 // Prefill: s_new = N(s + alpha (N(h) - s)) per row (+ loop re-injection).
 void launch_update_rows(const float* s_in, const float* h, const float* alpha,
                         float* s_out, bf16* s_bf, float* x_buf, int reinject,
@@ -185,13 +184,10 @@ struct AttnArgs {
   Dims dm;
   int window;          // 0 = full attention
   KVSlot kv; CacheGeo g;
-  float* part_o;       // decode: [B][Hq][kMaxSplits][hd]
-  float* part_ml;      // decode: [B][Hq][kMaxSplits][2]
   bf16* a_out;         // [M][qdim] = gate * attention output
   int* err;
 };
-void launch_attn_prefill(const AttnArgs& a, cudaStream_t st);
-// The same on the tcgen05 tensor cores.  kv_maps: this layer slot's K and V
+// Prefill attention on the tcgen05 tensor cores.  kv_maps: this layer slot's K and V
 // maps for 64-key tiles: K 64-dim boxes, K 32-dim boxes, V 64, V 32
 // (make_map_2d with box_rows = pf_tile_keys()).  Ring capacities must be
 // multiples of pf_tile_keys().
@@ -218,9 +214,6 @@ struct DecAttnArgs {
   float q_scale;
   int window;
   KVSlot kv; CacheGeo g;
-  float* part_o;       // [B][Hq][kMaxSplits][hd]
-  float* part_ml;      // [B][Hq][kMaxSplits][2]
-  int* counters;       // [B][Hkv] zero on entry; reset to zero on exit
   bf16* a_out;         // [B][qdim]
   int* err;
 };

@@ -30,20 +30,18 @@ __global__ void rope_table_kernel(float* table, const int* n_ctx, int T,
   }
 }
 
-// x0 = N(E[tok]); one block per row.  Block 0 also zeroes the attention
-// ticket counters and, for one-token calls (rope != null), writes the RoPE
-// cos/sin of position n_ctx for both attention types.
+// x0 = N(E[tok]); one block per row.  For one-token calls (rope != null)
+// block 0 also writes the RoPE cos/sin of position n_ctx for both attention
+// types.
 __global__ void embed_kernel(const int* tokens, const bf16* E, int d,
                              int vocab, float* s, bf16* s_bf, int* err,
-                             int* counters, int n_counters, float* rope,
-                             const int* n_ctx, int half, double th_swa,
-                             double th_full) {
+                             float* rope, const int* n_ctx, int half,
+                             double th_swa, double th_full) {
   __shared__ float red[32];
   const int row = blockIdx.x;
   pdl_wait();
   pdl_trigger();
   if (row == 0) {
-    for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
     if (rope) {
       const int p = *n_ctx;
       for (int id = threadIdx.x; id < 2 * half; id += blockDim.x) {
@@ -205,12 +203,11 @@ void launch_rope_table(float* table, const CacheGeo& g, int T, int hd,
 }
 
 void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
-                  bf16* s_bf, int* err, int vocab, int* counters,
-                  int n_counters, float* rope, const int* n_ctx, int hd,
-                  double theta_swa, double theta_full, cudaStream_t st) {
+                  bf16* s_bf, int* err, int vocab, float* rope,
+                  const int* n_ctx, int hd, double theta_swa,
+                  double theta_full, cudaStream_t st) {
   launch_k(embed_kernel, dim3(M), dim3(256), 0, st, tokens, E, d, vocab, s,
-           s_bf, err, counters, n_counters, rope, n_ctx, hd / 2, theta_swa,
-           theta_full);
+           s_bf, err, rope, n_ctx, hd / 2, theta_swa, theta_full);
 }
 
 void launch_update_rows(const float* s_in, const float* h, const float* alpha,
