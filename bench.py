@@ -312,6 +312,7 @@ def run_gpu(args, rank, world, local):
         torch.cuda.empty_cache()
     if not args.no_long:
         out["long_context"] = run_long(gm, args, hbm_peak, dev)
+        out["prefill_t8192_k4_per_loop"] = run_prefill_long(gm, tc_peak, dev)
     if args.quant:
         del gm
         torch.cuda.empty_cache()
@@ -425,6 +426,40 @@ def run_long(gm, args, hbm_peak, dev):
                                                        key=lambda kv: -kv[1]["ms"])}}
         del cache, ws
         torch.cuda.empty_cache()
+    return res
+
+
+def run_prefill_long(gm, tc_peak, dev, T=8192, k=4, mode="per_loop"):
+    """Prefill of one T-token prompt (seeded uniform tokens) at k loops: one
+    warm-up call, one timed call, one profiled call (FLOPs per kernel)."""
+    import torch
+    from synthetic import DORY, make_prompt
+    prompt = torch.from_numpy(make_prompt(DORY, 1, T)).to(dev)
+    cache = gm.new_cache(1, T + 16, T, kv_mode=mode, max_loops=k)
+    ws = gm.workspace(1, T)
+    t = None
+    for rep in range(3):
+        cache.reset()
+        if rep == 2:
+            gm.profile(True)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        gm.prefill(cache, prompt, k, ws)
+        e1.record()
+        torch.cuda.synchronize()
+        if rep == 1:
+            t = e0.elapsed_time(e1) / 1e3
+    st = gm.profile_read()
+    gm.profile(False)
+    assert gm.sync_status() == 0, "device-side check failed"
+    flops = sum(v["flops"] for v in st.values())
+    res = {"tok_s": T / t, "ms": t * 1e3, "flops": flops,
+           "tc_frac": flops / t / (tc_peak * 1e12),
+           "kernels_ms": {n: round(v["ms"], 2)
+                          for n, v in sorted(st.items(), key=lambda kv: -kv[1]["ms"])}}
+    del cache, ws
+    torch.cuda.empty_cache()
     return res
 
 

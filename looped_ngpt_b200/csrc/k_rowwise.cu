@@ -73,19 +73,92 @@ __global__ void embed_kernel(const int* tokens, const bf16* E, int d,
   }
 }
 
+// The nGPT update of whole rows (see ngpt_update_row for the algebra), one
+// row per block of d / 8 threads: thread i holds elements 4i..4i+3 and
+// d/2 + 4i..d/2 + 4i+3 in registers from the first read to the store, so a
+// row is read once and written once (16-byte accesses), with one block
+// reduction of the norm terms in between.  h: h_S K-split partials of the
+// sublayer output, gridDim.x rows apart.  Requires d % 256 == 0, d <= 8192.
 __global__ void update_rows_kernel(const float* s_in, const float* h,
                                    const float* alpha, float* s_out,
                                    bf16* s_bf, float* x_buf, int reinject,
                                    int d, int h_S) {
-  extern __shared__ float tmp[];
   __shared__ float red[7 * 32];
-  pdl_wait();
-  pdl_trigger();
   const size_t o = (size_t)blockIdx.x * d;
-  // h: h_S K-split partials of the sublayer output, gridDim.x rows apart
-  ngpt_update_row(s_in + o, h + o, h_S, (size_t)gridDim.x * d, alpha, d, reinject,
-                  reinject == RJ_NONE ? nullptr : x_buf + o, s_out + o,
-                  s_bf + o, tmp, red);
+  const size_t hs = (size_t)gridDim.x * d;
+  const int half = d / 2;
+  const bool next = reinject == RJ_NEXT;
+  pdl_wait();
+  float4 sv[2], av[2], hv[2], xv[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int i = 4 * threadIdx.x + k * half;
+    sv[k] = *reinterpret_cast<const float4*>(s_in + o + i);
+    av[k] = *reinterpret_cast<const float4*>(alpha + i);
+    hv[k] = *reinterpret_cast<const float4*>(h + o + i);
+    xv[k] = next ? *reinterpret_cast<const float4*>(x_buf + o + i)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int p = 1; p < h_S; ++p)
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float4 t = *reinterpret_cast<const float4*>(h + p * hs + o + 4 * threadIdx.x +
+                                                        k * half);
+      hv[k].x += t.x; hv[k].y += t.y; hv[k].z += t.z; hv[k].w += t.w;
+    }
+  pdl_trigger();
+  float r[7] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  auto acc = [&](float s, float a, float hh, float x) {
+    const float as = (1.f - a) * s, ah = a * hh;
+    r[0] += hh * hh;
+    r[1] += as * as;
+    r[2] += as * ah;
+    r[3] += ah * ah;
+    r[4] += as * x;
+    r[5] += ah * x;
+    r[6] += x * x;
+  };
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    acc(sv[k].x, av[k].x, hv[k].x, xv[k].x);
+    acc(sv[k].y, av[k].y, hv[k].y, xv[k].y);
+    acc(sv[k].z, av[k].z, hv[k].z, xv[k].z);
+    acc(sv[k].w, av[k].w, hv[k].w, xv[k].w);
+  }
+  block_sum_n<7>(r, red);
+  const float inv_h = 1.f / fmaxf(sqrtf(r[0]), 1e-12f);
+  const float tt = r[1] + 2.f * r[2] * inv_h + r[3] * inv_h * inv_h;
+  const float inv_t = 1.f / fmaxf(sqrtf(fmaxf(tt, 0.f)), 1e-12f);
+  float inv_u = 1.f;
+  if (next) {
+    const float dot = (r[4] + r[5] * inv_h) * inv_t;
+    inv_u = 1.f / fmaxf(sqrtf(fmaxf(1.f + 2.f * dot + r[6], 0.f)), 1e-12f);
+  }
+  auto upd = [&](float s, float a, float hh, float x, float* xs) {
+    float v = ((1.f - a) * s + a * hh * inv_h) * inv_t;
+    if (reinject == RJ_FIRST) *xs = v;
+    if (next) v = (v + x) * inv_u;
+    return v;
+  };
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int i = 4 * threadIdx.x + k * half;
+    float4 xo, vo;
+    vo.x = upd(sv[k].x, av[k].x, hv[k].x, xv[k].x, &xo.x);
+    vo.y = upd(sv[k].y, av[k].y, hv[k].y, xv[k].y, &xo.y);
+    vo.z = upd(sv[k].z, av[k].z, hv[k].z, xv[k].z, &xo.z);
+    vo.w = upd(sv[k].w, av[k].w, hv[k].w, xv[k].w, &xo.w);
+    if (reinject == RJ_FIRST && x_buf) *reinterpret_cast<float4*>(x_buf + o + i) = xo;
+    if (s_out) *reinterpret_cast<float4*>(s_out + o + i) = vo;
+    if (s_bf) {
+      uint2 u;
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(vo.x, vo.y);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(vo.z, vo.w);
+      u.x = *reinterpret_cast<const uint32_t*>(&lo);
+      u.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(s_bf + o + i) = u;
+    }
+  }
 }
 
 // Lowest index among the maxima; NaN entries never win.
@@ -213,8 +286,8 @@ void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
 void launch_update_rows(const float* s_in, const float* h, const float* alpha,
                         float* s_out, bf16* s_bf, float* x_buf, int reinject,
                         int M, int d, cudaStream_t st, int h_S) {
-  launch_k(update_rows_kernel, dim3(M), dim3(256), d * sizeof(float), st, s_in,
-           h, alpha, s_out, s_bf, x_buf, reinject, d, h_S);
+  launch_k(update_rows_kernel, dim3(M), dim3(d / 8), 0, st, s_in, h, alpha,
+           s_out, s_bf, x_buf, reinject, d, h_S);
 }
 
 void launch_argmax_partials(const float* val, const int* idx, int B, int n,
