@@ -19,6 +19,8 @@
 //   warp 0 lane 0   TMA: the Q tile once, then K and V tiles through a
 //                   3-stage ring (a 64-key tile is one 64-token page or one
 //                   64-slot run of a ring, whose capacity is a multiple of 64);
+//                   a stage's K slot is refilled as soon as S = Q K^T has
+//                   read it, its V slot once O += P V has;
 //   warp 1 lane 0   MMA: S_j = Q K_j^T (M 128, N 64, K 16 per instruction)
 //                   into one of two TMEM S buffers, then, once the softmax
 //                   has written P_j, O += P_j V_j (V as the MN-major B
@@ -52,7 +54,8 @@ constexpr int PST = 3;                  // K/V stages
 constexpr int kSmWarps = 8;             // softmax warps (2 per lane quarter)
 constexpr int kPfThreads = (2 + kSmWarps) * 32;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kOCol = 2 * PK;      // O accumulator after two S buffers
+constexpr int NSB = 3;                  // TMEM S buffers (S issued 2 tiles ahead)
+constexpr uint32_t kOCol = NSB * PK;    // O accumulator after the S buffers
 constexpr float kHeadroom = 8.f;        // log2 growth of m before O rescales
 
 // Shared-memory operand of `rows` rows x HD dims: N128 panels of 64 dims
@@ -110,14 +113,18 @@ attn_prefill_tc_kernel(const __grid_constant__ PfMaps mp, const AttnArgs a) {
   uint8_t* sQ = base;
   uint8_t* sKV = base + L::Q;
   uint8_t* sP = sKV + PST * L::STAGE;
-  __shared__ __align__(8) uint64_t q_full, kv_full[PST], kv_empty[PST];
-  // per tile parity b (tile j uses index j & 1, phase j >> 1), so that no
-  // barrier can run two phases ahead of its waiter:
-  //   s_full / s_free: S buffer b filled / read;  p_full: P buffer b written;
-  //   o_done: O += P V of a tile of parity b complete (with all before it)
-  __shared__ __align__(8) uint64_t s_full[2], s_free[2], p_full[2], o_done[2], mma_done;
+  // K and V slots of a stage fill and free separately: K_j is free once
+  // S_j = Q K_j^T completes, V_j once O += P_j V_j completes
+  __shared__ __align__(8) uint64_t q_full, k_full[PST], k_empty[PST], v_full[PST],
+      v_empty[PST];
+  // indexed so that no barrier can run two phases ahead of its waiter:
+  //   s_full / s_free[j % NSB] (phase j / NSB): S buffer filled / read;
+  //   p_full[j & 1] (phase j >> 1): P buffer written;
+  //   o_done[j & 1] (phase j >> 1): O += P_j V_j complete (and all before it)
+  __shared__ __align__(8) uint64_t s_full[NSB], s_free[NSB], p_full[2], o_done[2],
+      mma_done;
   __shared__ uint32_t tmem_base;
-  __shared__ int s_fail, s_issued;
+  __shared__ int s_fail, s_issued_k, s_issued_v;
   __shared__ float xch[2][PQ];                      // row max / sum exchange
   volatile int* fail = &s_fail;
 
@@ -132,19 +139,24 @@ attn_prefill_tc_kernel(const __grid_constant__ PfMaps mp, const AttnArgs a) {
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
     for (int i = 0; i < PST; ++i) {
-      mbar_init(kv_full + i, 1);
-      mbar_init(kv_empty + i, 1);
+      mbar_init(k_full + i, 1);
+      mbar_init(k_empty + i, 1);
+      mbar_init(v_full + i, 1);
+      mbar_init(v_empty + i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NSB; ++i) {
       mbar_init(s_full + i, 1);
       mbar_init(s_free + i, kSmWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(p_full + i, kSmWarps);
       mbar_init(o_done + i, 1);
     }
     mbar_init(&mma_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     s_fail = 0;
-    s_issued = 0;
+    s_issued_k = 0;
+    s_issued_v = 0;
   }
   if (warp == 0) tmem_alloc(&tmem_base, kTmemCols);
   tc_fence_before();
@@ -171,25 +183,40 @@ attn_prefill_tc_kernel(const __grid_constant__ PfMaps mp, const AttnArgs a) {
       if (L::N64)
         tma_load_2d(sQ + L::N128 * PQ * 128, &mp.q64, h * HD + 64 * L::N128, qrow,
                     &q_full);
-      for (int j = 0; j < nkt && !*fail; ++j) {
-        const int s = j % PST;
-        if (j >= PST && !mbar_wait(kv_empty + s, (uint32_t)((j / PST - 1) & 1))) {
+      // K tiles run up to PST ahead of V tiles; both wait (non-blocking
+      // checks, bounded in total) for their slot of PST tiles earlier
+      auto load = [&](int jt, bool is_v) {
+        const int s = jt % PST;
+        const int row = pf_tile_row(a.kv, a.g, dm.Hkv, b, kvh, t_lo + jt);
+        uint8_t* dst = sKV + s * L::STAGE + (is_v ? L::KV : 0);
+        uint64_t* bar = (is_v ? v_full : k_full) + s;
+        const CUtensorMap* m128 = is_v ? &mp.v128 : &mp.k128;
+        const CUtensorMap* m64 = is_v ? &mp.v64 : &mp.k64;
+        mbar_expect_tx(bar, L::KV);
+        for (int i = 0; i < L::N128; ++i) tma_load_2d(dst + i * PK * 128, m128, 64 * i, row, bar);
+        if (L::N64) tma_load_2d(dst + L::N128 * PK * 128, m64, 64 * L::N128, row, bar);
+      };
+      int jk = 0, jv = 0;
+      long idle = 0;
+      while (jv < nkt && !*fail) {
+        bool did = false;
+        if (jk < nkt &&
+            (jk < PST || mbar_try(k_empty + jk % PST, (uint32_t)((jk / PST - 1) & 1)))) {
+          load(jk++, false);
+          s_issued_k = jk;
+          did = true;
+        }
+        if (jv < jk &&
+            (jv < PST || mbar_try(v_empty + jv % PST, (uint32_t)((jv / PST - 1) & 1)))) {
+          load(jv++, true);
+          s_issued_v = jv;
+          did = true;
+        }
+        if (did) idle = 0;
+        else if (++idle > kSpin) {
           atomicOr(&s_fail, 1);
           break;
         }
-        const int row = pf_tile_row(a.kv, a.g, dm.Hkv, b, kvh, t_lo + j);
-        uint8_t* kt = sKV + s * L::STAGE;
-        uint8_t* vt = kt + L::KV;
-        mbar_expect_tx(kv_full + s, L::STAGE);
-        for (int i = 0; i < L::N128; ++i) {
-          tma_load_2d(kt + i * PK * 128, &mp.k128, 64 * i, row, kv_full + s);
-          tma_load_2d(vt + i * PK * 128, &mp.v128, 64 * i, row, kv_full + s);
-        }
-        if (L::N64) {
-          tma_load_2d(kt + L::N128 * PK * 128, &mp.k64, 64 * L::N128, row, kv_full + s);
-          tma_load_2d(vt + L::N128 * PK * 128, &mp.v64, 64 * L::N128, row, kv_full + s);
-        }
-        s_issued = j + 1;
       }
     }
   } else if (warp == 1) {
@@ -201,9 +228,9 @@ attn_prefill_tc_kernel(const __grid_constant__ PfMaps mp, const AttnArgs a) {
       const uint32_t q_s = su32(sQ), p_s = su32(sP);
       bool ok = mbar_wait(&q_full, 0);
       auto issue_s = [&](int j) {
-        const int s = j % PST, bb = j & 1;
-        if (!mbar_wait(kv_full + s, (uint32_t)((j / PST) & 1)) ||
-            (j >= 2 && !mbar_wait(s_free + bb, (uint32_t)(((j - 2) >> 1) & 1))))
+        const int s = j % PST, bb = j % NSB;
+        if (!mbar_wait(k_full + s, (uint32_t)((j / PST) & 1)) ||
+            (j >= NSB && !mbar_wait(s_free + bb, (uint32_t)((j / NSB - 1) & 1))))
           return false;
         tc_fence_after();
         const uint32_t k_s = su32(sKV + s * L::STAGE);
@@ -211,13 +238,16 @@ attn_prefill_tc_kernel(const __grid_constant__ PfMaps mp, const AttnArgs a) {
         for (int kk = 0; kk < L::KS; ++kk)
           umma_bf16(tmem + bb * PK, kmajor_desc<HD>(q_s, PQ, kk),
                     kmajor_desc<HD>(k_s, PK, kk), id_s, kk > 0);
+        umma_commit(k_empty + s);             // K_j read
         umma_commit(s_full + bb);
         return true;
       };
       auto issue_pv = [&](int j) {
-        if (!mbar_wait(p_full + (j & 1), (uint32_t)((j >> 1) & 1))) return false;
-        tc_fence_after();
         const int s = j % PST;
+        if (!mbar_wait(p_full + (j & 1), (uint32_t)((j >> 1) & 1)) ||
+            !mbar_wait(v_full + s, (uint32_t)((j / PST) & 1)))
+          return false;
+        tc_fence_after();
         const uint32_t v_s = su32(sKV + s * L::STAGE + L::KV);
         const uint32_t pj = p_s + (j & 1) * L::P;
 #pragma unroll
@@ -233,13 +263,15 @@ attn_prefill_tc_kernel(const __grid_constant__ PfMaps mp, const AttnArgs a) {
                                  kSw64),
                       id_o64, (j | kk) != 0);
         }
-        umma_commit(kv_empty + s);            // K_j, V_j read
+        umma_commit(v_empty + s);             // V_j read
         umma_commit(o_done + (j & 1));        // O holds P_0 V_0 + .. + P_j V_j
         return true;
       };
-      ok = ok && issue_s(0);
-      for (int j = 1; ok && j < nkt; ++j) ok = issue_s(j) && issue_pv(j - 1);
-      ok = ok && issue_pv(nkt - 1);
+      // S runs NSB - 1 tiles ahead of O += P V, so the softmax of tile j + 1
+      // never waits for its scores behind O += P_j V_j
+      for (int j = 0; ok && j < NSB - 1 && j < nkt; ++j) ok = issue_s(j);
+      for (int j = 0; ok && j < nkt; ++j)
+        ok = (j + NSB - 1 >= nkt || issue_s(j + NSB - 1)) && issue_pv(j);
       if (!ok) atomicOr(&s_fail, 1);
       umma_commit(&mma_done);
     }
@@ -256,8 +288,8 @@ attn_prefill_tc_kernel(const __grid_constant__ PfMaps mp, const AttnArgs a) {
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkt; ++j) {
-      const int bb = j & 1;
-      if (!mbar_wait_warp(s_full + bb, (uint32_t)((j >> 1) & 1))) { ok = false; break; }
+      const int bb = j % NSB;
+      if (!mbar_wait_warp(s_full + bb, (uint32_t)((j / NSB) & 1))) { ok = false; break; }
       tc_fence_after();
       float sv[32];
       tmem_ld32(trow + bb * PK + 32 * hf, sv);
@@ -376,9 +408,12 @@ attn_prefill_tc_kernel(const __grid_constant__ PfMaps mp, const AttnArgs a) {
     if (*fail) {
       atomicOr(a.err, ERRBIT_TIMEOUT);
       mbar_wait(&q_full, 0);
-      const int hi = s_issued, lo = hi > PST ? hi - PST : 0;
-      for (int j = lo; j < hi; ++j)
-        if (!mbar_wait(kv_full + j % PST, (uint32_t)((j / PST) & 1))) break;
+      for (int which = 0; which < 2; ++which) {
+        const int hi = which ? s_issued_v : s_issued_k, lo = hi > PST ? hi - PST : 0;
+        uint64_t* full = which ? v_full : k_full;
+        for (int j = lo; j < hi; ++j)
+          if (!mbar_wait(full + j % PST, (uint32_t)((j / PST) & 1))) break;
+      }
     }
   }
   tc_fence_before();
