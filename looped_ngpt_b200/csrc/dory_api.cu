@@ -656,8 +656,9 @@ void enqueue_forward(const CallCtx& x) {
         std::swap(cur, other);
       }
       if (x.T == 1) {
-        // one partial: every attention block re-reads the q/k/v rows of its
-        // KV head, so K-split partials would multiply that traffic
+        // one partial: the attention cluster's owner warps sum the q/k/v
+        // partials on the critical path before the cluster's first barrier;
+        // at B = 64 a 5-way split saved 0.45 ms here and cost 1.2 ms there
         gemm_run(m, w.s_bf, dm.d, bw.w_qkvg, w.qkvg, dm.rows_qkvg, x.M,
                  dm.rows_qkvg, dm.d, nullptr, x.st, "gemm_qkvg");
       } else {
