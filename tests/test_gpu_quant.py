@@ -1,7 +1,7 @@
 """MXFP8 / NVFP4 weight-only models on the GPU.
 
 * In-register weight decode is bit-exact against the oracle's decode of the
-  same bytes (spec: dequantised weights bit-exact).
+  same bytes (dequantised weights must match bit for bit).
 * Quantised decode (prompt fed one token per call, k=2, last_loop) matches
   the oracle run on the same quantised bytes within the BF16 tolerances."""
 import numpy as np
