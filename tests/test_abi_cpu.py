@@ -86,3 +86,22 @@ def test_null_handles_rejected():
     assert lib.dory_decode_step(None, None, None, 1, 1, 1, None, None, None,
                                 0, None) == -1
     assert lib.dory_sync_status(None, None) == -1
+
+
+def test_debug_gemm_arguments_validated_before_any_launch():
+    """Bad shapes and pointers are rejected by the host checks alone (no
+    device work), for the plain and the K-split debug GEMM."""
+    lib = _lib.load()
+    n = ctypes.c_int(0)
+    p = ctypes.c_void_p(0x1000)
+    # null operands, K not a multiple of 64, lda < K, no split slabs
+    assert lib.dory_debug_gemm_bf16(None, 64, p, p, 1, 1, 64, None) == -1
+    assert lib.dory_debug_gemm_bf16(p, 96, p, p, 1, 1, 96, None) == -1
+    assert lib.dory_debug_gemm_bf16(p, 32, p, p, 1, 1, 64, None) == -1
+    assert lib.dory_debug_gemm_bf16_split(p, 64, p, p, 1, 1, 64, 0,
+                                          ctypes.byref(n), None) == -1
+    assert lib.dory_debug_gemm_bf16_split(p, 64, p, p, 1, 1, 64, 4, None,
+                                          None) == -1
+    assert lib.dory_debug_gemm_bf16_split(p, 64, p, p, 0, 1, 64, 4,
+                                          ctypes.byref(n), None) == -1
+    assert n.value == 0
