@@ -113,10 +113,14 @@ class Clocks:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return
+        # the sampler takes a moment to start: let it run before the timed
+        # region so that its 50 ms samples fall inside it
+        time.sleep(0.3)
 
     def stop(self):
         if self.proc is None:
