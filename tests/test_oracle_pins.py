@@ -323,3 +323,125 @@ def test_loop_boundaries_follow_printed_equation(tiny_w):
     assert order[n_in:n_in + 3 * len(loop)] == loop * 3
     assert order[n_in + 3 * len(loop):] == [(k, i) for i in gout
                                             for k in ("attn", "mlp")]
+
+
+# ------------------------------------------------- sublayers from raw slices
+def _bf(t):
+    return (np.asarray(t).astype(np.uint32) << 16).view(np.float32).astype(
+        np.float64)
+
+
+def _small_shape(**kw):
+    return tiny_with_blocks(1, 1, 0, **kw)
+
+
+def _n(v):
+    return v / np.linalg.norm(v, axis=-1, keepdims=True)
+
+
+def _sig(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def _unit_rows(T, d, seed):
+    r = np.random.default_rng(seed).standard_normal((1, T, d))
+    return _n(r)
+
+
+def _expected_attn_uniform(w, sh, s, window):
+    """Attention sublayer output when every score is equal (no key carries
+    information): each query averages the values of its visible positions
+    (paperlayer summary §2: gated, normalised attention output blended into
+    the residual; paper summary, 技术新颖性: sigmoid output gate), written
+    from the raw rows of w_qkvg in the order q, k, v, gate."""
+    qd, kvd, h = sh.qdim, sh.kvdim, sh.head_dim
+    G = sh.n_q_heads // sh.n_kv_heads
+    W = _bf(w["blk0.w_qkvg"])
+    Wv, Wg = W[qd + kvd:qd + 2 * kvd], W[qd + 2 * kvd:]
+    T = s.shape[1]
+    out = np.empty_like(s)
+    for p in range(T):
+        lo = max(0, p - window + 1) if window else 0
+        vmean = np.mean([Wv @ s[0, j] for j in range(lo, p + 1)], axis=0)
+        o = np.concatenate([vmean[(hq // G) * h:(hq // G + 1) * h]
+                            for hq in range(sh.n_q_heads)])
+        a = _n(_sig(Wg @ s[0, p]) * o)
+        hA = _bf(w["blk0.w_o"]) @ a
+        al = np.asarray(w["blk0.alpha_a"], np.float64)
+        out[0, p] = _n(s[0, p] + al * (_n(hA) - s[0, p]))
+    return out
+
+
+@pytest.mark.parametrize("zero", ["q", "k"])
+def test_attn_sublayer_uniform_scores_closed_form(zero):
+    """With the query rows (or the key rows) of w_qkvg set to zero, every
+    score is 0 and each query's output is the mean of the visible values.
+    The expected state is written from the raw v / gate / W_o rows, so a
+    wrong q/k/v/gate slice, a missing sigmoid, another gate granularity or
+    another GQA head order fails here."""
+    sh = _small_shape()
+    w = dict(make_weights(sh, seed=3))
+    qd, kvd = sh.qdim, sh.kvdim
+    W = w["blk0.w_qkvg"].copy()
+    if zero == "q":
+        W[:qd] = 0
+    else:
+        W[qd:qd + kvd] = 0
+    w["blk0.w_qkvg"] = W
+    T = 13                          # longer than the 8-token window
+    s = _unit_rows(T, sh.d, 11)
+    for full, window in ((0, sh.swa_window), (1, 0)):
+        lt = (full,) + sh.layer_types[1:]
+        sh2 = _small_shape(layer_types=lt)
+        m = om.Model(sh2, w)
+        got = m.attn_sublayer(0, s, np.arange(T), 0)
+        want = _expected_attn_uniform(w, sh2, s, window)
+        assert np.allclose(got, want, atol=1e-12)
+
+
+def test_attn_sublayer_single_token_returns_gated_value():
+    """One token, empty cache: the softmax over one key is 1, so head h
+    outputs v of KV head h // (Hq/Hkv) whatever q and k are."""
+    sh = _small_shape()
+    w = make_weights(sh, seed=4)
+    s = _unit_rows(1, sh.d, 12)
+    got = om.Model(sh, w).attn_sublayer(0, s, np.arange(1), 0)
+    want = _expected_attn_uniform(w, sh, s, 0)
+    assert np.allclose(got, want, atol=1e-12)
+
+
+def test_mlp_sublayer_gate_rows_then_up_rows():
+    """SwiGLU over the fused gate/up matrix: rows [0, F) are the gate (through
+    silu), rows [F, 2F) the up projection (paperlayer summary §2: SwiGLU
+    activations normalised before the down projection).  Swapping the halves
+    gives another state, so the test sees the order."""
+    sh = _small_shape()
+    w = make_weights(sh, seed=5)
+    F = sh.ffn
+    s = _unit_rows(3, sh.d, 13)
+    Wgu = _bf(w["blk0.w_gu"])
+    g, u = s @ Wgu[:F].T, s @ Wgu[F:].T
+    al = np.asarray(w["blk0.alpha_m"], np.float64)
+
+    def state(gate, up):
+        m = _n(gate * _sig(gate) * up)
+        hM = m @ _bf(w["blk0.w_down"]).T
+        return _n(s + al * (_n(hM) - s))
+
+    got = om.Model(sh, w).mlp_sublayer(0, s)
+    assert np.allclose(got, state(g, u), atol=1e-12)
+    assert not np.allclose(got, state(u, g), atol=1e-6)
+
+
+def test_lm_head_across_row_chunks_with_logit_scale():
+    """z = s_z * (W_lm s) for a vocabulary larger than the oracle's 16384-row
+    chunk, with a non-uniform logit scale (paperlayer summary §2: logit-scale
+    parameters)."""
+    sh = _small_shape(vocab=40000)
+    w = dict(make_weights(sh, seed=6, names=["lm_head", "s_z"]))
+    w["s_z"] = np.linspace(0.5, 3.0, sh.vocab).astype(np.float32)
+    s = _unit_rows(2, sh.d, 14)
+    got = om.Model(sh, w).lm_head(s)
+    want = w["s_z"].astype(np.float64) * (s @ _bf(w["lm_head"]).T)
+    assert got.shape == (1, 2, sh.vocab)
+    assert np.allclose(got, want, atol=1e-12)
