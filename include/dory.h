@@ -22,7 +22,9 @@
  * Conventions for every entry point:
  *   - Return 0 (DORY_OK) or a negative DORY_ERR_* code; dory_strerror()
  *     names it.  A failed call leaves caller buffers unspecified but the
- *     library state valid.
+ *     library state valid.  DORY_ERR_CUDA also covers a launch plan that
+ *     could not be built on the host (a TMA descriptor the driver rejects);
+ *     with DORY_DEBUG=1 in the environment the library names it on stderr.
  *   - Pointers prefixed d_ are device pointers (global memory of the current
  *     device); others are host pointers.  The caller allocates and owns every
  *     device buffer (weights, cache, workspace, outputs); the library keeps
@@ -110,7 +112,13 @@ int dory_init_weights(const dory_config* cfg, const dory_tensor* tensors,
 
 /* Bytes of device memory a KV cache needs for `batch` sequences of up to
  * `max_ctx` tokens, calls of up to `max_chunk` tokens per sequence, and (in
- * per_loop mode) up to `max_loops` loops.  Layout: a small header, the full
+ * per_loop mode) up to `max_loops` loops.  The two modes are the pages'
+ * recurrent KV-cache modes: per_loop keeps one cache per loop of every
+ * recurrent attention layer, last_loop one cache per recurrent attention
+ * layer that every loop overwrites, so its footprint equals the k = 1
+ * footprint at any k ("Dory1.0-4B: A Looped Normalized-GPT", §6.1
+ * Last-Loop KV Caching; MXFP8 explainer page, "循环 + KV 缓存" section).
+ * Input and output blocks keep one cache each in both modes.  Layout: a small header, the full
  * attention layers as 64-token pages behind a block table, the
  * sliding-window layers as rings of min(max_ctx, window + max_chunk - 1)
  * positions rounded up to a multiple of 64 (the attention kernels' key
@@ -121,7 +129,9 @@ int dory_kv_cache_bytes(const dory_model* m, int batch, int max_ctx,
                         int64_t* bytes);
 
 /* Bind a caller-owned device buffer (>= dory_kv_cache_bytes, 256-byte
- * aligned) as an empty cache and enqueue its initialisation on `stream`:
+ * aligned) as an empty cache of the layout above (paperlayer §6.1;
+ * sliding-window layers keep only their window, paper summary, 技术新颖性)
+ * and enqueue its initialisation on `stream`:
  * the length and block table are set and every K/V row is zeroed (attention
  * tiles also read rows no token has written yet; their weights are 0 and
  * their contents must be finite).  The kv_mode is fixed for the life of the
@@ -157,7 +167,14 @@ int dory_workspace_bytes(const dory_model* m, int batch, int max_chunk,
                          int64_t* bytes);
 
 /* Append T tokens per sequence (d_tokens int32 [B, T], row-major) and run
- * the looped forward pass over them with `n_loops` recurrent loops.
+ * the looped forward pass over them with `n_loops` recurrent loops: the
+ * input blocks once, the shared recurrent blocks n_loops times with the
+ * re-injection u_t = N(s_{t-1} + x), the output blocks once, then the
+ * logits (paper summary, 核心方法; the loop count is a per-request runtime
+ * knob, MXFP8 explainer page, deployment section).  Inside a loop every
+ * attention layer first writes the K/V of all T tokens to the slot the
+ * kv_mode selects, then every query reads what each visible position holds
+ * (paperlayer §6.1).
  * B must equal the bound batch, 1 <= T <= max_chunk, n_ctx + T <= max_ctx,
  * kv_mode must equal the cache's; a per_loop cache takes the loop count of
  * its first call and rejects any other (DORY_ERR_CACHE).
@@ -169,8 +186,11 @@ int dory_prefill(dory_model* m, dory_cache* c, const int32_t* d_tokens, int B,
                  float* d_logits, int32_t* d_argmax, void* d_workspace,
                  int64_t ws_bytes, void* stream);
 
-/* One decode step: one token per sequence (d_tokens int32 [B]).  Same rules
- * as dory_prefill with T = 1.  The step is replayed from a CUDA graph once
+/* One decode step: one token per sequence (d_tokens int32 [B]) through the
+ * same looped forward pass as dory_prefill with T = 1 (paper summary,
+ * 核心方法; in last_loop mode every loop's query reads the final-loop
+ * entries of the earlier tokens, paperlayer §6.1).  Same rules as
+ * dory_prefill.  The step is replayed from a CUDA graph once
  * its launch plan has been seen with the same pointers, B and n_loops. */
 int dory_decode_step(dory_model* m, dory_cache* c, const int32_t* d_tokens,
                      int B, int n_loops, int kv_mode, float* d_logits,
@@ -218,8 +238,10 @@ int dory_decode_step_static(dory_model* m, dory_cache* c,
  * d_C f32 [M, N] (row-major) = d_A bf16 [M, K] (row stride lda >= K, a
  * multiple of 8) times d_W bf16 [N, K]^T, on the tcgen05 tensor cores.
  * K must be a multiple of 64; device pointers 16-byte aligned.  Enqueued on
- * `stream`; errors: DORY_ERR_ARG, DORY_ERR_CUDA (timeouts of its bounded
- * waits are reported by dory_sync_status of any model). */
+ * `stream`; errors: DORY_ERR_ARG, DORY_ERR_CUDA (also when the operands'
+ * TMA descriptors cannot be built, e.g. for a pointer that is not 16-byte
+ * aligned; nothing is enqueued then); timeouts of its bounded waits are
+ * reported by dory_sync_status of any model. */
 int dory_debug_gemm_bf16(const void* d_A, int lda, const void* d_W,
                          float* d_C, int M, int N, int K, void* stream);
 
@@ -233,6 +255,32 @@ int dory_debug_gemm_bf16(const void* d_A, int lda, const void* d_W,
 int dory_debug_gemm_bf16_split(const void* d_A, int lda, const void* d_W,
                                float* d_C, int M, int N, int K, int max_splits,
                                int* n_partials, void* stream);
+
+/* Test access to the failure path of the bounded device waits: enqueue one
+ * block whose thread waits on an mbarrier that nothing ever arrives on,
+ * gives up after `polls` polls (1 <= polls <= 2^20; each poll returns
+ * within microseconds) and records a timeout in the model's device status
+ * word, then exits normally.  The next dory_sync_status() returns
+ * DORY_ERR_TIMEOUT and clears the word; the context stays usable.  Errors:
+ * DORY_ERR_ARG, DORY_ERR_CUDA. */
+int dory_debug_bounded_wait(dory_model* m, int polls, void* stream);
+
+/* Test access to the decode GEMV exactly as the forward pass runs it (same
+ * kernel, same in-register weight decode, same K split): d_out = the block
+ * projection `tensor` (e.g. "blk3.w_down"; "blk<i>.w_gu" as one [2F, K]
+ * matrix) times the bf16 rows d_x [B, K] (1 <= B <= 8, 16-byte aligned),
+ * written as *n_partials K-split partial slabs f32 [n][B][N] (d_out holds
+ * max_partials slabs; at most 8 are written) whose sum is
+ * the product.  Quantised models multiply the decoded weights (f16, exact)
+ * by the activations rounded to f16, apply the group scale to each 8-term
+ * sum and the NVFP4 tensor scale to the total; with a one-hot row x = e_k the
+ * result is weight (n, k) times its scales, rounded once to f32, which is
+ * how the tests compare the production decode bit for bit with the format
+ * definitions.  Errors: DORY_ERR_ARG (bad name, B, alignment, or more
+ * partials than max_partials), DORY_ERR_CUDA. */
+int dory_debug_gemv(const dory_model* m, const char* tensor, const void* d_x,
+                    int B, float* d_out, int max_partials, int* n_partials,
+                    void* stream);
 
 /* Test access to the in-register weight decode of quantised models: write
  * rows [row0, row0 + nrows) of block projection `tensor` (e.g.

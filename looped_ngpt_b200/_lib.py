@@ -61,6 +61,9 @@ SIGNATURES = {
     "dory_debug_gemm_bf16_split": (c_int, [_P, c_int, _P, _P, c_int, c_int,
                                            c_int, c_int, POINTER(c_int), _P]),
     "dory_debug_dequant": (c_int, [_P, c_char_p, c_int, c_int, _P, _P]),
+    "dory_debug_bounded_wait": (c_int, [_P, c_int, _P]),
+    "dory_debug_gemv": (c_int, [_P, c_char_p, _P, c_int, _P, c_int,
+                                POINTER(c_int), _P]),
     "dory_copy_state": (c_int, [_P, _P, c_int, c_int, c_int, _P, _P]),
     "dory_sync_status": (c_int, [_P, _P]),
     "dory_profile_enable": (c_int, [_P, c_int]),

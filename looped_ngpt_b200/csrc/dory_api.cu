@@ -14,12 +14,27 @@
 
 #include "dory.h"
 #include "dory_internal.h"
+#include "async_copy.cuh"
 
 using namespace dory;
 
 static __device__ int g_dory_status;   // or-ed ERRBIT_* from device checks
 
 namespace dory {
+namespace {
+thread_local bool t_host_failure = false;
+}
+void note_host_failure(const char* what) {
+  t_host_failure = true;
+  const char* e = getenv("DORY_DEBUG");
+  if (e && e[0] == '1') fprintf(stderr, "dory: %s could not be built\n", what);
+}
+bool take_host_failure() {
+  const bool f = t_host_failure;
+  t_host_failure = false;
+  return f;
+}
+
 bool pdl_enabled() {
   static const bool on = [] {
     const char* e = getenv("DORY_NO_PDL");
@@ -163,10 +178,17 @@ struct WS {
 };
 
 constexpr int kMaxS = 8;
-// K-split partial slabs of the f32 projection outputs (qkvg, h): decode
-// batches that go through the tensor-core GEMM (one row tile) split K up
-// to 16 ways; the GEMV splits at most kMaxS ways.
+// K-split partials that a call may write into the f32 projection outputs
+// (qkvg, h): decode batches that go through the tensor-core GEMM (one row
+// tile) split K up to 16 ways, the GEMV at most kMaxS ways; multi-token
+// calls split the W_o / W_down GEMMs only when their output has fewer tiles
+// than the GPU has SMs (gemm_split_count, at most kMaxS).
 int slabs_of(size_t M, int T) { return T == 1 && M <= 128 ? 16 : kMaxS; }
+int h_slabs(const Dims& dm, int M, int T) {
+  if (T == 1) return slabs_of(M, T);
+  return std::max(gemm_split_count(M, dm.d, dm.qdim, kMaxS),
+                  gemm_split_count(M, dm.d, dm.F, kMaxS));
+}
 constexpr int kArgmaxSlots = 2048;
 
 WS ws_layout(const dory_model* m, int B, int T, char* base) {
@@ -184,11 +206,12 @@ WS ws_layout(const dory_model* m, int B, int T, char* base) {
   w.sfin = (float*)take(M * dm.d * 4);
   w.x = (float*)take(M * dm.d * 4);
   w.s_bf = (bf16*)take(M * dm.d * 2);
-  w.qkvg = (float*)take(slabs_of(M, T) * M * dm.rows_qkvg * 4);
+  // multi-token calls project q/k/v/gate inside the QKV GEMM epilogue
+  w.qkvg = (float*)take(T == 1 ? slabs_of(M, T) * M * dm.rows_qkvg * 4 : 0);
   w.qb = (bf16*)take(M * dm.qdim * 2);
   w.gate = (float*)take(M * dm.qdim * 4);
   w.a = (bf16*)take(M * dm.qdim * 2);
-  w.h = (float*)take(slabs_of(M, T) * M * dm.d * 4);
+  w.h = (float*)take((size_t)h_slabs(dm, (int)M, T) * M * dm.d * 4);
   w.mact = (bf16*)take(M * dm.F * 2);
   w.rope = (float*)take((size_t)2 * T * (dm.hd / 2) * 2 * 4);
   w.amax_val = (float*)take((size_t)B * kArgmaxSlots * 4);
@@ -489,9 +512,12 @@ void dory_cache_free(dory_cache* c) {
 int dory_workspace_bytes(const dory_model* m, int batch, int max_chunk,
                          int64_t* bytes) {
   if (!m || !bytes || batch < 1 || max_chunk < 1) return DORY_ERR_ARG;
-  // decode calls (T = 1) lay out more K-split slabs per row
-  *bytes = (int64_t)std::max(ws_layout(m, batch, max_chunk, nullptr).total,
-                             ws_layout(m, batch, 1, nullptr).total);
+  // the split-K slab count depends on the call's token count, so a shorter
+  // call can need more bytes than a longer one: take the largest layout
+  size_t mx = 0;
+  for (int T = 1; T <= max_chunk; ++T)
+    mx = std::max(mx, ws_layout(m, batch, T, nullptr).total);
+  *bytes = (int64_t)mx;
   return DORY_OK;
 }
 
@@ -835,6 +861,7 @@ int run_call(dory_model* m, dory_cache* c, const int32_t* tokens, int B,
   CallCtx x{m, c, w, B, T, B * T, n_loops, logits_all, c->n_ctx, tokens,
             logits, argmax, (cudaStream_t)stream};
   cudaGetLastError();   // clear stale errors from earlier, unrelated calls
+  take_host_failure();
 
   bool done = false;
   if (decode && m->use_graphs && !m->prof) {
@@ -858,7 +885,9 @@ int run_call(dory_model* m, dory_cache* c, const int32_t* tokens, int B,
           cudaSuccess) {
         enqueue_forward(cx);
         const cudaError_t e1 = cudaStreamEndCapture(m->cap_stream, &graph);
-        if (e1 == cudaSuccess && graph &&
+        // a launcher that enqueued nothing leaves an incomplete graph
+        const bool partial = take_host_failure();
+        if (e1 == cudaSuccess && graph && !partial &&
             cudaGraphInstantiate(&ge.exec, graph, 0) != cudaSuccess)
           ge.exec = nullptr;
         if (graph) cudaGraphDestroy(graph);
@@ -874,7 +903,8 @@ int run_call(dory_model* m, dory_cache* c, const int32_t* tokens, int B,
     }
   }
   if (!done) enqueue_forward(x);
-  if (cudaGetLastError() != cudaSuccess) return DORY_ERR_CUDA;
+  if (take_host_failure() | (cudaGetLastError() != cudaSuccess))
+    return DORY_ERR_CUDA;
   c->n_ctx += T;
   if (kv_mode == DORY_KV_PER_LOOP && !c->loops_bound) c->loops_bound = n_loops;
   return DORY_OK;
@@ -984,6 +1014,27 @@ extern "C" int dory_decode_step_static(dory_model* m, dory_cache* c,
                   d_argmax, ws, (int64_t)DORY_STATIC_WS_BYTES, stream, false);
 }
 
+// A bounded wait that runs out on purpose: one thread waits on an mbarrier
+// that nothing arrives on, gives up after `polls` polls and records
+// ERRBIT_TIMEOUT, exactly as the streaming kernels do when a copy or a peer
+// stalls.  No copy is in flight and no tensor memory is held.
+__global__ void bounded_wait_kernel(int polls, int* err) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (!mbar_wait(&bar, 0, polls)) atomicOr(err, ERRBIT_TIMEOUT);
+  }
+}
+
+extern "C" int dory_debug_bounded_wait(dory_model* m, int polls,
+                                       void* stream) {
+  if (!m || polls < 1 || polls > (1 << 20)) return DORY_ERR_ARG;
+  cudaGetLastError();
+  bounded_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(polls, m->d_status);
+  return cuda_rc(cudaGetLastError());
+}
+
 extern "C" int dory_debug_gemm_bf16(const void* d_A, int lda, const void* d_W,
                                     float* d_C, int M, int N, int K,
                                     void* stream) {
@@ -991,8 +1042,10 @@ extern "C" int dory_debug_gemm_bf16(const void* d_A, int lda, const void* d_W,
       lda < K || lda % 8)
     return DORY_ERR_ARG;
   cudaGetLastError();
+  take_host_failure();
   launch_gemm_bf16((const bf16*)d_A, lda, (const bf16*)d_W, d_C, N, M, N, K,
                    nullptr, (cudaStream_t)stream);
+  if (take_host_failure()) return DORY_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? DORY_OK : DORY_ERR_CUDA;
 }
 
@@ -1004,9 +1057,14 @@ extern "C" int dory_debug_gemm_bf16_split(const void* d_A, int lda,
       K % 64 || lda < K || lda % 8 || max_splits < 1)
     return DORY_ERR_ARG;
   cudaGetLastError();
+  take_host_failure();
   *n_partials = launch_gemm_bf16((const bf16*)d_A, lda, (const bf16*)d_W, d_C,
                                  N, M, N, K, nullptr, (cudaStream_t)stream,
                                  max_splits, (long)M * N);
+  if (take_host_failure()) {
+    *n_partials = 0;
+    return DORY_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? DORY_OK : DORY_ERR_CUDA;
 }
 
@@ -1043,28 +1101,79 @@ extern "C" int dory_cache_fill_synthetic(dory_model* m, dory_cache* c,
   return DORY_OK;
 }
 
+namespace {
+
+// Block projection `tensor` ("blk<i>.<w>") of a model: its matrix and shape.
+bool find_proj(const dory_model* m, const char* tensor, const QMat** q,
+               long* N, long* K) {
+  if (!tensor) return false;
+  const std::string n = tensor;
+  if (n.compare(0, 3, "blk") != 0) return false;
+  const size_t dot = n.find('.');
+  if (dot == std::string::npos || dot == 3) return false;
+  for (size_t c = 3; c < dot; ++c)
+    if (n[c] < '0' || n[c] > '9') return false;
+  const int i = atoi(n.substr(3, dot - 3).c_str());
+  if (i < 0 || i >= m->nblk) return false;
+  const std::string leaf = n.substr(dot + 1);
+  const BlockW& b = m->blk[i];
+  const Dims& dm = m->dm;
+  if (leaf == "w_qkvg") { *q = &b.m_qkvg; *N = dm.rows_qkvg; *K = dm.d; }
+  else if (leaf == "w_o") { *q = &b.m_o; *N = dm.d; *K = dm.qdim; }
+  else if (leaf == "w_gu") { *q = &b.m_gu; *N = 2L * dm.F; *K = dm.d; }
+  else if (leaf == "w_down") { *q = &b.m_down; *N = dm.d; *K = dm.F; }
+  else return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" int dory_debug_gemv(const dory_model* m, const char* tensor,
+                               const void* d_x, int B, float* d_out,
+                               int max_partials, int* n_partials,
+                               void* stream) {
+  if (!m || !d_x || !d_out || !n_partials || B < 1 || B > 8 ||
+      max_partials < 1 || ((uintptr_t)d_x & 15))
+    return DORY_ERR_ARG;
+  *n_partials = 0;
+  const QMat* q = nullptr;
+  long N = 0, K = 0;
+  if (!find_proj(m, tensor, &q, &N, &K)) return DORY_ERR_ARG;
+  GemvArgs g{};
+  g.W = q->w;
+  g.fmt = WF_BF16;
+  if (!q->w) {
+    g.fmt = m->wfmt == DORY_W_MXFP8 ? WF_MXFP8 : WF_NVFP4;
+    g.Wq = q->q;
+    g.Ws = q->s;
+    g.Wt = q->t;
+  }
+  g.K = (int)K;
+  g.n_items = (int)N;
+  g.B = B;
+  g.epi = EPI_F32;
+  g.pro = PRO_BF16;
+  g.xin = (const bf16*)d_x;
+  g.xin_stride = (int)K;
+  g.out = d_out;
+  g.err = m->d_status;
+  g.S = gemv_splits(g);
+  if (g.S > max_partials) return DORY_ERR_ARG;
+  cudaGetLastError();
+  launch_gemv(g, gemv_grid(g, m->num_sms), (cudaStream_t)stream);
+  if (cudaGetLastError() != cudaSuccess) return DORY_ERR_CUDA;
+  *n_partials = g.S;
+  return DORY_OK;
+}
+
 extern "C" int dory_debug_dequant(const dory_model* m, const char* tensor,
                                   int row0, int nrows, float* d_out,
                                   void* stream) {
   if (!m || !tensor || !d_out || row0 < 0 || nrows < 1) return DORY_ERR_ARG;
   if (m->wfmt == DORY_W_BF16) return DORY_ERR_UNSUPPORTED;
-  const std::string n = tensor;
-  const std::string pre = "blk";
-  if (n.compare(0, 3, pre) != 0) return DORY_ERR_ARG;
-  const size_t dot = n.find('.');
-  if (dot == std::string::npos) return DORY_ERR_ARG;
-  const int i = atoi(n.substr(3, dot - 3).c_str());
-  if (i < 0 || i >= m->nblk) return DORY_ERR_ARG;
-  const std::string leaf = n.substr(dot + 1);
-  const BlockW& b = m->blk[i];
-  const Dims& dm = m->dm;
   const QMat* q = nullptr;
   long N = 0, K = 0;
-  if (leaf == "w_qkvg") { q = &b.m_qkvg; N = dm.rows_qkvg; K = dm.d; }
-  else if (leaf == "w_o") { q = &b.m_o; N = dm.d; K = dm.qdim; }
-  else if (leaf == "w_gu") { q = &b.m_gu; N = 2L * dm.F; K = dm.d; }
-  else if (leaf == "w_down") { q = &b.m_down; N = dm.d; K = dm.F; }
-  else return DORY_ERR_ARG;
+  if (!find_proj(m, tensor, &q, &N, &K)) return DORY_ERR_ARG;
   if ((long)row0 + nrows > N) return DORY_ERR_ARG;
   cudaGetLastError();
   launch_dequant_rows(m->wfmt == DORY_W_MXFP8 ? WF_MXFP8 : WF_NVFP4, q->q, q->s,

@@ -52,6 +52,13 @@ inline cudaError_t launch_k_cluster(void (*kernel)(KArgs...), dim3 grid,
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Host-side failure of a launcher that enqueued nothing (a tensor map that
+// could not be encoded).  The launcher records it; every entry point clears
+// the record before it enqueues work and returns DORY_ERR_CUDA if it is set
+// afterwards.  Per host thread.
+void note_host_failure(const char* what);
+bool take_host_failure();
+
 // Device error bits (or-ed into the status word the host reads back).
 enum : int {
   ERRBIT_BOUNDS = 1,   // a position or index fell outside its buffer
@@ -236,6 +243,9 @@ bool make_kv_tile_map(CUtensorMap* m, const void* ptr, long rows, int hd);
 int launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
                      int M, int N, int K, const float* col_scale,
                      cudaStream_t st, int max_splits = 1, long slab = 0);
+// Number of K-split partials launch_gemm_bf16 writes for this shape and
+// max_splits (without a column scale).
+int gemm_split_count(int M, int N, int K, int max_splits);
 // m[M, F] = silu(A W_g^T) * (A W_u^T) as bf16, W = [W_g; W_u] (2F rows).
 void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
                         int ldm, int M, int F, int K, cudaStream_t st);

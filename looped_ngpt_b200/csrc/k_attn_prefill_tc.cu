@@ -437,7 +437,7 @@ void launch_pf_t(const AttnArgs& a, const CUtensorMap* kv_maps, cudaStream_t st)
   const long M = (long)a.B * a.T;
   if (!make_act_map(&mp.q128, a.q, M, a.dm.qdim, 64, PQ) ||
       !make_act_map(&mp.q64, a.q, M, a.dm.qdim, 32, PQ)) {
-    fprintf(stderr, "dory: tensor map creation failed\n");
+    note_host_failure("prefill attention: tensor map");
     return;
   }
   mp.k128 = kv_maps[0];

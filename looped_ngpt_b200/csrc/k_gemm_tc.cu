@@ -517,7 +517,7 @@ int launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
                      cudaStream_t st, int max_splits, long slab) {
   CUtensorMap ma, mb;
   if (!make_map(&ma, A, M, K, lda, BM) || !weight_map(&mb, W, N, K, 128)) {
-    fprintf(stderr, "dory: tensor map creation failed\n");
+    note_host_failure("gemm: tensor map");
     return 1;
   }
   TcArgs a = base_args(M, N, K);
@@ -526,16 +526,22 @@ int launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
   a.slab = slab;
   a.col_scale = col_scale;
   const int mt = (M + BM - 1) / BM, nt = (N + BN - 1) / BN;
+  const int ks = gemm_split_count(M, N, K, col_scale ? 1 : max_splits);
+  launch_tc<TC_PLAIN, BN>(ma, mb, a, mt, nt, st, ks);
+  return ks;
+}
+
+int gemm_split_count(int M, int N, int K, int max_splits) {
+  const int mt = (M + BM - 1) / BM, nt = (N + BN - 1) / BN;
   const int KB = K / BK;
   int ks = 1;
-  if (max_splits > 1 && !col_scale && mt * nt < num_sms()) {
+  if (max_splits > 1 && mt * nt < num_sms()) {
     // at least 2 K blocks per split keep the stage ring busy
     ks = std::min(std::min(max_splits, num_sms() / (mt * nt)), KB / 2);
     if (ks < 1) ks = 1;
     const int kbs = (KB + ks - 1) / ks;
     ks = (KB + kbs - 1) / kbs;                  // no empty split
   }
-  launch_tc<TC_PLAIN, BN>(ma, mb, a, mt, nt, st, ks);
   return ks;
 }
 
@@ -544,7 +550,7 @@ void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
                         int ldm, int M, int F, int K, cudaStream_t st) {
   CUtensorMap ma, mb;
   if (!make_map(&ma, A, M, K, lda, BM) || !weight_map(&mb, W, 2L * F, K, 128)) {
-    fprintf(stderr, "dory: tensor map creation failed\n");
+    note_host_failure("gemm: tensor map");
     return;
   }
   TcArgs a = base_args(M, F, K);
@@ -557,7 +563,7 @@ void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
     // the F / 72 tiles (143 for F = 10240) give every SM one tile
     CUtensorMap mb2;
     if (!weight_map(&mb2, W, 2L * F, K, kSmallPair)) {
-      fprintf(stderr, "dory: tensor map creation failed\n");
+      note_host_failure("gemm: tensor map");
       return;
     }
     launch_tc<TC_SWIGLU, 2 * kSmallPair>(ma, mb2, a, mt,
@@ -575,7 +581,7 @@ void launch_gemm_qkv(const bf16* A, int lda, const bf16* W, const QkvGemmArgs& q
   CUtensorMap ma, mb;
   if (!make_map(&ma, A, q.M, q.dm.d, lda, BM) ||
       !weight_map(&mb, W, rows, q.dm.d, hd)) {
-    fprintf(stderr, "dory: tensor map creation failed\n");
+    note_host_failure("gemm: tensor map");
     return;
   }
   TcArgs a = base_args(q.M, rows, q.dm.d);

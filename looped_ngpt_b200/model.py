@@ -206,6 +206,23 @@ class DoryModel:
             ctypes.c_void_p(out.data_ptr()), _stream_ptr(stream)))
         return out
 
+    def debug_gemv(self, tensor, x, stream=None):
+        """dory_debug_gemv: the production decode GEMV of block projection
+        `tensor` on bf16 rows x [B, K]; returns the f32 partial slabs
+        [n, B, N] (their sum is the product)."""
+        B, K = x.shape
+        N = {"w_qkvg": self.shape.qkvg_rows, "w_o": self.shape.d,
+             "w_gu": 2 * self.shape.ffn, "w_down": self.shape.d}[
+                 tensor.split(".", 1)[1]]
+        cap = 16
+        out = torch.empty((cap, B, N), dtype=torch.float32, device=self.device)
+        n = ctypes.c_int()
+        check("dory_debug_gemv", _lib.load().dory_debug_gemv(
+            self.handle, tensor.encode(), ctypes.c_void_p(x.data_ptr()), B,
+            ctypes.c_void_p(out.data_ptr()), cap, ctypes.byref(n),
+            _stream_ptr(stream)))
+        return out[:n.value]
+
     def sync_status(self, stream=None):
         return _lib.load().dory_sync_status(self.handle, _stream_ptr(stream))
 

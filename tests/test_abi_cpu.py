@@ -105,3 +105,18 @@ def test_debug_gemm_arguments_validated_before_any_launch():
     assert lib.dory_debug_gemm_bf16_split(p, 64, p, p, 0, 1, 64, 4,
                                           ctypes.byref(n), None) == -1
     assert n.value == 0
+
+
+def test_debug_gemm_unbuildable_descriptor_is_an_error():
+    """An operand the TMA descriptor cannot describe (a base address that is
+    not 16-byte aligned) makes the launcher enqueue nothing; the entry point
+    must report DORY_ERR_CUDA, never DORY_OK.  The A descriptor is built
+    first and fails, so no kernel is launched on any machine."""
+    lib = _lib.load()
+    n = ctypes.c_int(0)
+    bad = ctypes.c_void_p(0x1002)
+    p = ctypes.c_void_p(0x1000)
+    assert lib.dory_debug_gemm_bf16(bad, 64, p, p, 1, 128, 64, None) == -4
+    assert lib.dory_debug_gemm_bf16_split(bad, 64, p, p, 1, 128, 64, 4,
+                                          ctypes.byref(n), None) == -4
+    assert n.value == 0

@@ -71,3 +71,21 @@ def test_gemm_k_split_partials_sum_to_product(M, N, K):
     ref = bf16_bits_to_f32(A).astype(np.float64) @ bf16_bits_to_f32(W).astype(np.float64).T
     tol = 1e-5 * np.sqrt(K) * (np.abs(ref).max() + 1)
     assert np.abs(got - ref).max() <= tol, np.abs(got - ref).max()
+
+
+def test_gemm_misaligned_operand_reports_error():
+    """A operand 2 bytes past a 16-byte boundary: the TMA descriptor cannot be
+    built, nothing is launched, the call returns DORY_ERR_CUDA and the
+    output keeps its contents."""
+    M, N, K = 64, 256, 128
+    buf = torch.zeros(M * K + 8, dtype=torch.int16, device="cuda")
+    dW = torch.zeros((N, K), dtype=torch.int16, device="cuda")
+    dC = torch.full((M, N), float("nan"), device="cuda")
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    lib = _lib.load()
+    assert lib.dory_debug_gemm_bf16(ctypes.c_void_p(buf.data_ptr() + 2), K,
+                                    ctypes.c_void_p(dW.data_ptr()),
+                                    ctypes.c_void_p(dC.data_ptr()), M, N, K,
+                                    s) == -4
+    torch.cuda.synchronize()
+    assert torch.isnan(dC).all()

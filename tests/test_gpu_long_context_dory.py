@@ -1,7 +1,8 @@
 """Decode over seeded synthetic cached context at the full Dory1.0-4B shape,
 in the launch configuration bench.py times for long context: B=64 sequences,
-k=2, per_loop (one 16-block cluster per (sequence, KV head) in the decode
-attention, split-K tensor-core GEMMs for the batch-64 projections).
+k=2, per_loop and last_loop (one 16-block cluster per (sequence, KV head) in
+the decode attention, split-K tensor-core GEMMs for the batch-64
+projections).
 
   * 4096 cached tokens: sequences 0 and 63 against the float64 oracle given
     the same cache entries (synthetic.kvgen), one decode step: the logits
@@ -33,14 +34,17 @@ def dory_long():
     return w, lb.DoryModel(DORY, w, device="cuda:0")
 
 
-def oracle_for(w, seqs, n_ctx):
+def oracle_for(w, seqs, n_ctx, kv_mode="per_loop"):
     """Oracle model whose batch rows are the sampled sequences `seqs`, each
-    slot's cache filled with that sequence's synthetic entries."""
-    m = Model(DORY, w, batch=len(seqs), kv_mode="per_loop")
+    slot's cache filled with that sequence's synthetic entries (the
+    generator's slot index is the loop t for per_loop recurrent blocks, 0
+    for every single-slot block)."""
+    m = Model(DORY, w, batch=len(seqs), kv_mode=kv_mode)
     _, grec, _ = DORY.block_groups()
     pos = np.arange(n_ctx)
     for i in range(DORY.n_blocks):
-        for s in (range(1, K_LOOPS + 1) if i in grec else [0]):
+        per_loop = i in grec and kv_mode == "per_loop"
+        for s in (range(1, K_LOOPS + 1) if per_loop else [0]):
             Kc = np.zeros((len(seqs), DORY.n_kv_heads, n_ctx, DORY.head_dim))
             Vc = np.zeros_like(Kc)
             for r, b in enumerate(seqs):
@@ -51,8 +55,8 @@ def oracle_for(w, seqs, n_ctx):
     return m
 
 
-def gpu_step(gm, n_ctx, tok):
-    cache = gm.new_cache(B, n_ctx + 8, 1, kv_mode="per_loop", max_loops=K_LOOPS)
+def gpu_step(gm, n_ctx, tok, kv_mode="per_loop"):
+    cache = gm.new_cache(B, n_ctx + 8, 1, kv_mode=kv_mode, max_loops=K_LOOPS)
     cache.fill_synthetic(n_ctx, SEED)
     ws = gm.workspace(B, 1)
     z, a = gm.decode_step(cache, torch.from_numpy(tok).cuda(), K_LOOPS, ws)
@@ -65,16 +69,17 @@ def gpu_step(gm, n_ctx, tok):
     return out
 
 
-def test_b64_ctx4k_sampled_sequences_match_oracle(dory_long):
+@pytest.mark.parametrize("kv_mode", ["per_loop", "last_loop"])
+def test_b64_ctx4k_sampled_sequences_match_oracle(dory_long, kv_mode):
     w, gm = dory_long
     n_ctx = 4096
     tok = np.random.default_rng(7).integers(0, DORY.vocab, size=B).astype(np.int32)
-    z, a, s, length, status = gpu_step(gm, n_ctx, tok)
+    z, a, s, length, status = gpu_step(gm, n_ctx, tok, kv_mode)
     assert status == 0 and length == n_ctx + 1
     seqs = [0, B - 1]
-    ref = oracle_for(w, seqs, n_ctx)
+    ref = oracle_for(w, seqs, n_ctx, kv_mode)
     zr = ref.decode_step(tok[seqs], K_LOOPS)
-    compare(z[seqs], zr, "dory B=64 ctx 4096 sampled")
+    compare(z[seqs], zr, f"dory B=64 ctx 4096 {kv_mode} sampled")
     assert np.array_equal(a, np.argmax(z, -1))
     assert np.abs(np.linalg.norm(s, axis=-1) - 1).max() <= NORM_TOL
 

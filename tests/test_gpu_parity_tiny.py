@@ -112,6 +112,26 @@ def test_bad_token_sets_device_error(tiny):
     assert gm.sync_status() == 0                     # the word was cleared
 
 
+def test_bounded_wait_timeout_is_reported(tiny):
+    """A device wait that nothing ends (an mbarrier no one arrives on) gives
+    up after its poll budget, records a timeout, and the host reads it as
+    DORY_ERR_TIMEOUT; the word is cleared and the context stays usable."""
+    from looped_ngpt_b200 import _lib
+    import ctypes
+    w, gm = tiny
+    lib = _lib.load()
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.dory_debug_bounded_wait(gm.handle, 0, s) == -1
+    assert lib.dory_debug_bounded_wait(gm.handle, 1024, s) == 0
+    assert gm.sync_status() == -5
+    assert gm.sync_status() == 0
+    cache = gm.new_cache(1, 8, 1, kv_mode="last_loop")
+    ws = gm.workspace(1, 1)
+    gm.decode_step(cache, torch.tensor([3], dtype=torch.int32,
+                                       device="cuda:0"), 1, ws)
+    assert gm.sync_status() == 0
+
+
 def test_pooled_top1_agreement(tiny):
     """Raw top-1 agreement >= 99.5% over 1024 prompt positions (B=4 x 256,
     k=2, last_loop; every position's logits compared)."""
