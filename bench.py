@@ -38,16 +38,18 @@ def parse():
     ap.add_argument("--steps", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=4)
     ap.add_argument("--impl", default="dory", choices=["dory", "reference"])
-    ap.add_argument("--loops", default="1,2,4")
+    ap.add_argument("--loops", default="1,2,3,4")
     ap.add_argument("--kv-mode", default="last_loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prompt", type=int, default=PROMPT)
     ap.add_argument("--no-long", action="store_true",
                     help="skip the long-context batched-decode workloads")
     ap.add_argument("--long-steps", type=int, default=8)
-    ap.add_argument("--quant", action="store_true",
-                    help="also time MXFP8 / NVFP4 weight-only models (B=1 at "
+    ap.add_argument("--no-quant", action="store_true",
+                    help="skip the MXFP8 / NVFP4 weight-only models (B=1 at "
                          "2048 context and B=4 at 131072 context, k=2)")
+    ap.add_argument("--no-per-loop", action="store_true",
+                    help="skip the per_loop rows of the 2048-token workload")
     ap.add_argument("--profile-decode", type=int, default=0, metavar="K",
                     help="only: prefill, warm up, then one decode step at "
                          "k=K inside the NVTX range 'decode_step' (for ncu)")
@@ -193,12 +195,46 @@ def blas_threads():
 
 
 # --------------------------------------------------------------- oracle arm --
-def oracle_decode_sample(w, n_loops, tokens=1):
-    """Time the oracle on a bounded sample of the decode workload: `tokens`
-    decode steps from an empty cache (context 1..tokens)."""
+def arm_config(prompt, world, kv_mode):
+    """The workload both arms name in their JSON line."""
+    return {"workload": (f"Dory-shape BF16 looped nGPT decode, batch 1 per GPU "
+                         f"at a {prompt}-token context, k={HEADLINE_K}, "
+                         f"{kv_mode}"),
+            "global_batch": world, "seq_len": prompt,
+            "parallelism": f"replicas x{world}",
+            "l2": "no flush: 12 GB of weights streamed per token > L2"}
+
+
+def oracle_at_context(w, n_ctx, kv_mode="last_loop", n_loops=HEADLINE_K,
+                      extra=64):
+    """The oracle holding n_ctx tokens of seeded synthetic context (the same
+    counter generator the library's cache fill uses), every slot sized for
+    `extra` more tokens."""
     from oracle.model import Model
     from synthetic import DORY
-    m = Model(DORY, w, batch=1, kv_mode="last_loop")
+    from synthetic.kvgen import kv_rows
+    m = Model(DORY, w, batch=1, kv_mode=kv_mode)
+    _, grec, _ = DORY.block_groups()
+    pos = np.arange(n_ctx)
+    for i in range(DORY.n_blocks):
+        per_loop = i in grec and kv_mode == "per_loop"
+        for slot in (range(1, n_loops + 1) if per_loop else [0]):
+            K = np.zeros((1, DORY.n_kv_heads, n_ctx + extra, DORY.head_dim))
+            V = np.zeros_like(K)
+            for h in range(DORY.n_kv_heads):
+                K[0, h, :n_ctx], V[0, h, :n_ctx] = kv_rows(DORY, 2, i, slot, 0,
+                                                          h, pos)
+            m.cache[(i, slot)] = (K, V)
+    m.n_ctx = n_ctx
+    if kv_mode == "per_loop":
+        m.n_loops_fixed = n_loops
+    return m
+
+
+def oracle_decode_sample(w, n_loops, n_ctx, tokens=1):
+    """Time the oracle on a bounded sample of the decode workload: `tokens`
+    greedy decode steps at a context of n_ctx cached tokens."""
+    m = oracle_at_context(w, n_ctx, n_loops=n_loops, extra=tokens + 1)
     t0 = time.perf_counter()
     tok = 7
     for _ in range(tokens):
@@ -209,6 +245,69 @@ def oracle_decode_sample(w, n_loops, tokens=1):
 
 
 # ------------------------------------------------------------------ GPU arm --
+# ------------------------------------------------------------------ GPU arm --
+def decode_prefill_at(gm, prompt, k, kv_mode, ws, K, W, world, max_ctx,
+                      tc_peak, hbm_peak, clocks=None):
+    """The 2048-token workload at k loops in one KV mode: the prompt's
+    prefill (one warm-up call, one timed, one profiled for FLOPs), then W + K
+    greedy decode steps (CUDA-graph replays; the argmax of each step is
+    written straight into the token buffer the next step reads), then P
+    profiled eager steps (CUDA events around every kernel)."""
+    import torch
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    cache = gm.new_cache(1, max_ctx, prompt.shape[1], kv_mode=kv_mode,
+                         max_loops=k)
+    t_pre = None
+    for rep in range(3):
+        cache.reset()
+        if rep == 2:
+            gm.profile(True)
+        torch.cuda.synchronize()
+        e0, e1 = ev(), ev()
+        e0.record()
+        _, am = gm.prefill(cache, prompt, k, ws)
+        e1.record()
+        torch.cuda.synchronize()
+        if rep == 1:
+            t_pre = e0.elapsed_time(e1) / 1e3
+    pst = gm.profile_read()
+    gm.profile(False)
+    pflops = sum(v["flops"] for v in pst.values())
+    gm.decode_step(cache, am, k, ws, want_logits=False)
+    tok = cache._dec_bufs[0]
+    for _ in range(W):
+        gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
+    torch.cuda.synchronize()
+    barrier(world)
+    if clocks:
+        clocks.start()
+    e0, e1 = ev(), ev()
+    e0.record()
+    for _ in range(K):
+        gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    dt = e0.elapsed_time(e1) / 1e3
+    ck = clocks.stop() if clocks else None
+    gm.profile(True)
+    P = 4
+    for _ in range(P):
+        gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
+    st = gm.profile_read()
+    gm.profile(False)
+    assert gm.sync_status() == 0, "device-side check failed"
+    bytes_tok = sum(v["bytes"] for v in st.values()) / P
+    return dict(
+        prefill_tok_s=prompt.shape[1] / t_pre, prefill_flops=pflops,
+        prefill_tc_frac=pflops / t_pre / (tc_peak * 1e12),
+        decode_tok_s=K / dt, decode_bytes_per_token=bytes_tok,
+        decode_hbm_frac=bytes_tok * K / dt / (hbm_peak * 1e9),
+        kv_cache_gb=cache.nbytes / 1e9,
+        dt=dt, clocks=ck, stats=st, P=P, cache=cache,
+        launches=sum(v["launches"] for v in st.values()) / P)
+
+
 def run_gpu(args, rank, world, local):
     import torch
     import looped_ngpt_b200 as lb
@@ -225,69 +324,27 @@ def run_gpu(args, rank, world, local):
     K, W = args.steps, args.warmup
     max_ctx = args.prompt + 2 * (W + K) + 16
     ws = gm.workspace(1, args.prompt)
-    ev = lambda: torch.cuda.Event(enable_timing=True)
-    out = {"decode_tok_s": {}, "prefill_tok_s": {}, "decode_hbm_frac": {},
-           "prefill_tc_frac": {}, "decode_bytes_per_token": {},
-           "prefill_flops": {}}
+    modes = [args.kv_mode]
+    if not args.no_per_loop:
+        modes += [m for m in ("last_loop", "per_loop") if m != args.kv_mode]
+    out = {}
     headline = None
-    for k in ks:
-        cache = gm.new_cache(1, max_ctx, args.prompt, kv_mode=args.kv_mode,
-                             max_loops=k)
-        # prefill: one warm-up call, one timed, one profiled (counts FLOPs)
-        t_pre = None
-        for rep in range(3):
-            cache.reset()
-            if rep == 2:
-                gm.profile(True)
-            torch.cuda.synchronize()
-            e0, e1 = ev(), ev()
-            e0.record()
-            _, am = gm.prefill(cache, prompt, k, ws)
-            e1.record()
-            torch.cuda.synchronize()
-            if rep == 1:
-                t_pre = e0.elapsed_time(e1) / 1e3
-        pst = gm.profile_read()
-        gm.profile(False)
-        pflops = sum(v["flops"] for v in pst.values())
-        out["prefill_tok_s"][f"k{k}"] = args.prompt / t_pre
-        out["prefill_flops"][f"k{k}"] = pflops
-        out["prefill_tc_frac"][f"k{k}"] = pflops / t_pre / (tc_peak * 1e12)
-        # decode: the argmax of each step is written straight into the token
-        # buffer that the next step reads
-        gm.decode_step(cache, am, k, ws, want_logits=False)
-        tok = cache._dec_bufs[0]
-        for _ in range(W):
-            gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
-        clocks = Clocks(local) if k == HEADLINE_K else None
-        torch.cuda.synchronize()
-        barrier(world)
-        if clocks:
-            clocks.start()
-        e0, e1 = ev(), ev()
-        e0.record()
-        for _ in range(K):
-            gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
-        e1.record()
-        torch.cuda.synchronize()
-        barrier(world)
-        dt = e0.elapsed_time(e1) / 1e3
-        ck = clocks.stop() if clocks else None
-        # profiled steps (eager, CUDA events around each kernel)
-        gm.profile(True)
-        P = 4
-        for _ in range(P):
-            gm.decode_step(cache, tok, k, ws, argmax=tok, want_logits=False)
-        st = gm.profile_read()
-        gm.profile(False)
-        assert gm.sync_status() == 0, "device-side check failed"
-        bytes_tok = sum(v["bytes"] for v in st.values()) / P
-        out["decode_tok_s"][f"k{k}"] = K / dt
-        out["decode_bytes_per_token"][f"k{k}"] = bytes_tok
-        out["decode_hbm_frac"][f"k{k}"] = bytes_tok * K / dt / (hbm_peak * 1e9)
-        if k == HEADLINE_K:
-            headline = dict(dt=dt, clocks=ck, stats=st, P=P, cache=cache,
-                            launches=sum(v["launches"] for v in st.values()) / P)
+    for mode in modes:
+        rows = {"decode_tok_s": {}, "prefill_tok_s": {}, "decode_hbm_frac": {},
+                "prefill_tc_frac": {}, "decode_bytes_per_token": {},
+                "prefill_flops": {}, "kv_cache_gb": {}}
+        for k in ks:
+            head = mode == args.kv_mode and k == HEADLINE_K
+            r = decode_prefill_at(gm, prompt, k, mode, ws, K, W, world, max_ctx,
+                                  tc_peak, hbm_peak,
+                                  Clocks(local) if head else None)
+            for key in rows:
+                rows[key][f"k{k}"] = r[key]
+            if head:
+                headline = r
+            else:
+                del r["cache"]
+        out[mode] = rows
     # end-to-end through host buffers at the headline k
     k = HEADLINE_K
     cache = headline["cache"]
@@ -314,13 +371,12 @@ def run_gpu(args, rank, world, local):
         host_tok.copy_(host_out)
     e2e_dt = time.perf_counter() - t0
     barrier(world)
-    if not args.no_long or args.quant:
-        del cache, headline["cache"]
-        torch.cuda.empty_cache()
+    del cache, headline["cache"]
+    torch.cuda.empty_cache()
     if not args.no_long:
         out["long_context"] = run_long(gm, args, hbm_peak, dev)
         out["prefill_t8192_k4_per_loop"] = run_prefill_long(gm, tc_peak, dev)
-    if args.quant:
+    if not args.no_quant:
         del gm
         torch.cuda.empty_cache()
         out["quantized"] = run_quant(w, args, hbm_peak, dev)
@@ -537,7 +593,7 @@ def main():
     value = world * K / dt
     e2e_dt = max_over_ranks(r["e2e_dt"], world)
     st = h["stats"]
-    # dominant kernel: largest share of the profiled step time
+    # dominant kernel: largest share of the profiled (eager) step
     dom = max(st, key=lambda n: st[n]["ms"])
     d = st[dom]
     bound = "hbm" if d["flops"] / max(d["bytes"], 1) < 100 else "tensor"
@@ -547,14 +603,17 @@ def main():
     else:
         achieved = d["flops"] / d["launches"] / (d["ms"] / d["launches"] / 1e3) / 1e12
         peak, unit = r["tc_peak"], "TFLOP/s"
-    total_ms = sum(v["ms"] for v in st.values())
+    eager_ms = sum(v["ms"] for v in st.values())
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, secs = oracle_decode_sample(r["w"], HEADLINE_K, tokens=1)
+        tps, secs = oracle_decode_sample(r["w"], HEADLINE_K, args.prompt)
         cpu = {"value": tps, "unit": "tok/s", "cores": blas_threads(),
                "kind": "oracle",
-               "sample": f"1 decode step at k={HEADLINE_K} from an empty "
-                         f"cache, Dory-shape weights ({secs:.1f} s of CPU)"}
+               "sample": (f"1 greedy decode step at k={HEADLINE_K}, "
+                          f"{args.kv_mode}, at a {args.prompt}-token context "
+                          f"(seeded synthetic cached entries from the "
+                          f"generator the library's cache fill uses), "
+                          f"Dory-shape weights, fp64 NumPy ({secs:.1f} s)")}
     if rank != 0:
         return 0
     line = {
@@ -562,27 +621,31 @@ def main():
         "steps": K, "warmup": W, "ms_per_step": dt / K * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": (f"Dory-shape BF16 looped nGPT decode, batch 1 "
-                                f"per GPU after a {args.prompt}-token prompt, "
-                                f"k={HEADLINE_K}, {args.kv_mode}"),
-                   "global_batch": world, "seq_len": args.prompt,
-                   "parallelism": f"replicas x{world}",
-                   "l2": "no flush: 12 GB of weights streamed per token > L2"},
+        "config": arm_config(args.prompt, world, args.kv_mode),
         "roofline": {"bound": bound, "kernel": dom, "achieved": achieved,
                      "peak": peak, "unit": unit, "frac": achieved / peak,
                      "peak_source": r["peak_kind"], "traffic": dram_traffic(dom),
-                     "share_of_step": d["ms"] / total_ms},
+                     "share_of_eager_pass": d["ms"] / eager_ms},
         "cpu_baseline": cpu,
         "e2e": {"value": world * K / e2e_dt, "unit": "tok/s",
                 "h2d_bytes_per_step": 4, "d2h_bytes_per_step": 4},
         "gpu_launches": int(round(h["launches"] * K)),
         "clocks": h["clocks"],
         "breakdown": r["out"],
-        "kernels": {n: {"launches_per_step": v["launches"] / h["P"],
-                        "us_per_step": v["ms"] / h["P"] * 1e3,
-                        "GBps": v["bytes"] / (v["ms"] / 1e3) / 1e9
-                        if v["ms"] > 0 else None}
-                    for n, v in sorted(st.items(), key=lambda kv: -kv[1]["ms"])},
+        # per-kernel figures of P extra steps launched eagerly with CUDA
+        # events around every kernel (no graph, no overlap between
+        # kernels): their sum exceeds the graph-replayed step time, so they
+        # rank kernels and give each one's own rate, not shares of the
+        # timed step (the ncu launch list under profiles/ gives those)
+        "kernels_eager": {
+            "eager_pass_ms": eager_ms / h["P"],
+            "timed_step_ms": dt / K * 1e3,
+            "per_kernel": {n: {"launches_per_step": v["launches"] / h["P"],
+                               "us_per_step": v["ms"] / h["P"] * 1e3,
+                               "GBps": v["bytes"] / (v["ms"] / 1e3) / 1e9
+                               if v["ms"] > 0 else None}
+                           for n, v in sorted(st.items(),
+                                              key=lambda kv: -kv[1]["ms"])}},
     }
     print(json.dumps(line))
     if world > 1:
@@ -592,28 +655,41 @@ def main():
 
 
 def main_reference(args):
-    """The oracle on the host cores: bounded decode samples of the same
-    workload (Dory shapes, k=2), same metric and unit."""
+    """The oracle on the host cores, on the GPU arm's workload (Dory shapes,
+    batch 1, k=2, decode at the prompt-length context) and metric.  One
+    oracle decode token takes about 20 s, so a step is a bounded sample: 1/C
+    of a token, C the smallest divisor of --steps that keeps the timed run
+    at 3 tokens or fewer; the K steps run as K / C whole tokens, timed
+    together."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from synthetic import DORY, make_weights
+    K, W = max(1, args.steps), max(0, args.warmup)
+    C = next(c for c in range(1, K + 1) if K % c == 0 and K // c <= 3)
+    n_tok, n_warm = K // C, -(-W // C)
     w = make_weights(DORY, seed=0)
-    K, W = max(1, min(args.steps, 2)), max(0, min(args.warmup, 1))
-    for _ in range(W):
-        oracle_decode_sample(w, HEADLINE_K, tokens=1)
-    tps, secs = oracle_decode_sample(w, HEADLINE_K, tokens=K)
-    sample = (f"{K} decode steps at k={HEADLINE_K} from an empty cache, "
-              f"Dory-shape weights, fp64 NumPy ({secs:.1f} s)")
+    m = oracle_at_context(w, args.prompt, args.kv_mode, HEADLINE_K,
+                          extra=n_tok + n_warm + 1)
+    tok = 7
+    for _ in range(n_warm):
+        tok = int(np.argmax(m.decode_step([tok], HEADLINE_K)[0]))
+    t0 = time.perf_counter()
+    for _ in range(n_tok):
+        tok = int(np.argmax(m.decode_step([tok], HEADLINE_K)[0]))
+    secs = time.perf_counter() - t0
+    tps = n_tok / secs
+    sample = (f"{K} steps of 1/{C} decode token each, run as {n_tok} whole "
+              f"greedy decode tokens at k={HEADLINE_K}, {args.kv_mode}, "
+              f"after a {args.prompt}-token seeded synthetic cached context "
+              f"({n_warm} warm-up tokens), Dory-shape weights, fp64 NumPy "
+              f"({secs:.1f} s timed)")
     line = {"metric": METRIC, "value": tps, "unit": "tok/s", "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": secs / K * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": (f"Dory-shape looped nGPT decode, batch 1, "
-                                    f"k={HEADLINE_K}, last_loop"),
-                       "global_batch": 1, "seq_len": args.prompt,
-                       "parallelism": "none"},
+            "config": arm_config(args.prompt, world, args.kv_mode),
             "cpu_baseline": {"value": tps, "unit": "tok/s",
                              "cores": blas_threads(), "kind": "oracle",
                              "sample": sample},

@@ -6,9 +6,11 @@ The pages fix the formats only by name: MXFP8 W8A16 with group size 32
 (MXFP8 explainer page, deployment section) and NVFP4 as E2M1 values with
 E4M3 scale factors (paper summary, 前置知识 / NVFP4).  The element encodings
 below follow the public OCP Microscaling (MX) format definitions and NVIDIA's
-NVFP4 description; the quantisers use maximum scaling (paperlayer §5.2 says
-MXFP8 uses standard max scaling; the MSE scale search it names for NVFP4 is
-not reproduced, since both sides decode the same bytes).
+NVFP4 description.  The quantisers use maximum scaling (paperlayer §5.2:
+MXFP8 uses standard max scaling), and quant_nvfp4_mse the dynamic MSE block
+scale selection that the same section names for NVFP4 (its search range is
+a reading, stated there).  Both sides decode the same bytes, so the choice
+of quantiser changes accuracy, not parity.
 
 Layouts (row-major, K = input/contraction axis):
   MXFP8: q uint8 [N, K] (E4M3 codes), e uint8 [N, K/32] (E8M0 codes).
@@ -109,6 +111,41 @@ def quant_nvfp4(w):
     S = np.float32(amax_t / (6.0 * 448.0)) if amax_t > 0 else np.float32(1.0)
     g = w.reshape(N, K // 16, 16)
     sb = round_e4m3(np.abs(g).max(axis=-1) / (6.0 * float(S)))
+    den = e4m3_decode(sb) * float(S)
+    safe = np.where(den > 0, den, 1.0)
+    codes = np.where(den[..., None] > 0, round_e2m1(g / safe[..., None]), 0)
+    codes = codes.reshape(N, K).astype(np.uint8)
+    packed = (codes[:, 0::2] & 0xF) | ((codes[:, 1::2] & 0xF) << 4)
+    return packed.astype(np.uint8), sb, S
+
+
+def quant_nvfp4_mse(w, below=8, above=1):
+    """NVFP4 with dynamic MSE block-scale selection (paperlayer summary §5.2:
+    NVFP4 uses dynamic MSE scale selection, MXFP8 and the other formats max
+    scaling).  The pages give no search range; the reading taken here: the
+    tensor scale S stays the max-scaling one, and for every 16-weight block
+    the E4M3 scale code is the one, among the max-scaling code c and the
+    codes c - below .. c + above (within the finite positive codes 1..126;
+    `below` = 8 spans one binade), whose decoded block has the smallest sum
+    of squared errors; ties go to the larger code.  All-zero blocks keep
+    code 0.  Values are rounded as in quant_nvfp4."""
+    w = np.asarray(w, dtype=np.float64)
+    N, K = w.shape
+    amax_t = float(np.abs(w).max())
+    S = np.float32(amax_t / (6.0 * 448.0)) if amax_t > 0 else np.float32(1.0)
+    g = w.reshape(N, K // 16, 16)
+    c_max = round_e4m3(np.abs(g).max(axis=-1) / (6.0 * float(S))).astype(np.int64)
+    best_c = c_max.copy()
+    best_err = np.full(c_max.shape, np.inf)
+    for off in range(above, -below - 1, -1):            # larger codes first
+        c = np.clip(c_max + off, 1, 126)
+        den = e4m3_decode(c) * float(S)
+        codes = round_e2m1(g / den[..., None])
+        err = np.sum((g - e2m1_decode(codes) * den[..., None]) ** 2, axis=-1)
+        better = err < best_err
+        best_err = np.where(better, err, best_err)
+        best_c = np.where(better, c, best_c)
+    sb = np.where(c_max > 0, best_c, 0).astype(np.uint8)
     den = e4m3_decode(sb) * float(S)
     safe = np.where(den > 0, den, 1.0)
     codes = np.where(den[..., None] > 0, round_e2m1(g / safe[..., None]), 0)

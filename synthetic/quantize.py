@@ -2,7 +2,8 @@
 checkpoint formats the Dory pages name: MXFP8 W8A16 (E4M3 values, E8M0 scale
 per 32 weights; MXFP8 explainer page, deployment section) and NVFP4 W4A16
 (E2M1 values, E4M3 scale per 16 weights, f32 tensor scale; paper summary,
-前置知识 / NVFP4).  Maximum scaling (paperlayer §5.2).  This is input
+前置知识 / NVFP4).  Maximum scaling, and for NVFP4 also the dynamic MSE
+block-scale selection (paperlayer §5.2).  This is input
 preparation only; a test checks that it produces exactly the bytes of the
 oracle's own quantiser.
 
@@ -71,6 +72,27 @@ def encode_nvfp4(w):
     return packed.astype(np.uint8), sb, np.array([S], dtype=np.float32)
 
 
+def _nvfp4_block_codes(g, S, e4, below=8, above=1):
+    """E4M3 block-scale codes of 16-weight blocks g [n, K/16, 16] chosen by
+    minimum squared error among the max-scaling code c and c - below ..
+    c + above (finite positive codes only; ties to the larger code; all-zero
+    blocks keep code 0).  Input preparation for the NVFP4 'dynamic MSE'
+    checkpoints (paperlayer summary §5.2)."""
+    c0 = _nearest(np.abs(g).max(-1) / (6.0 * float(S)), e4).astype(np.int64)
+    e2 = _e2m1_values()
+    best, best_err = c0.copy(), np.full(c0.shape, np.inf)
+    for off in range(above, -below - 1, -1):
+        c = np.clip(c0 + off, 1, 126)
+        den = e4[c] * float(S)
+        y = g / den[..., None]
+        v = e2[_nearest(y, e2)] * np.where(np.signbit(y), -1.0, 1.0)
+        err = np.sum((g - v * den[..., None]) ** 2, axis=-1)
+        better = err < best_err
+        best_err = np.where(better, err, best_err)
+        best = np.where(better, c, best)
+    return np.where(c0 > 0, best, 0).astype(np.uint8)
+
+
 def _encode_rows(w, fmt, rows=2048):
     """Encode in row chunks (bounded float64 temporaries).  The NVFP4 tensor
     scale needs the whole-matrix maximum first."""
@@ -85,7 +107,10 @@ def _encode_rows(w, fmt, rows=2048):
         g = np.asarray(w[r:r + rows], dtype=np.float64)
         n, K = g.shape
         g = g.reshape(n, K // 16, 16)
-        sb = _nearest(np.abs(g).max(-1) / (6.0 * float(S)), e4).astype(np.uint8)
+        if fmt == "nvfp4_mse":
+            sb = _nvfp4_block_codes(g, S, e4)
+        else:
+            sb = _nearest(np.abs(g).max(-1) / (6.0 * float(S)), e4).astype(np.uint8)
         den = e4[sb] * float(S)
         y = g / np.where(den > 0, den, 1.0)[..., None]
         c = _nearest(y, _e2m1_values()) | np.where(np.signbit(y), 0x8, 0)
@@ -97,12 +122,13 @@ def _encode_rows(w, fmt, rows=2048):
 
 
 def quantize_weights(weights, fmt, workers=None):
-    """Copy of `weights` with the block projections in `fmt` ('mxfp8' or
-    'nvfp4'); embeddings, LM head and vectors unchanged.  Matrices are
+    """Copy of `weights` with the block projections in `fmt` ('mxfp8',
+    'nvfp4', or 'nvfp4_mse': the NVFP4 format with block scales chosen by
+    minimum squared error); embeddings, LM head and vectors unchanged.  Matrices are
     encoded on a thread pool (NumPy releases the GIL in the bulk work)."""
     import os
     from concurrent.futures import ThreadPoolExecutor
-    if fmt not in ("mxfp8", "nvfp4"):
+    if fmt not in ("mxfp8", "nvfp4", "nvfp4_mse"):
         raise ValueError(fmt)
     names = [n for n in weights if n.split(".", 1)[-1] in QUANT_LEAVES]
     out = {n: t for n, t in weights.items() if n not in names}
@@ -112,6 +138,6 @@ def quantize_weights(weights, fmt, workers=None):
                                                  fmt), names))
     for n, r in zip(names, res):
         out[n + ".q"], out[n + ".s"] = r[0], r[1]
-        if fmt == "nvfp4":
+        if fmt != "mxfp8":
             out[n + ".t"] = r[2]
     return out

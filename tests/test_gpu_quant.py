@@ -1,7 +1,9 @@
 """MXFP8 / NVFP4 weight-only models on the GPU.
 
 * In-register weight decode is bit-exact against the oracle's decode of the
-  same bytes (dequantised weights must match bit for bit).
+  same bytes (dequantised weights must match bit for bit).  NVFP4 is also
+  run with block scales chosen by minimum squared error (the same format,
+  other bytes).
 * Quantised decode (prompt fed one token per call, k=2, last_loop) matches
   the oracle run on the same quantised bytes within the BF16 tolerances."""
 import numpy as np
@@ -17,7 +19,7 @@ from tests.gpu_util import compare
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module", params=["mxfp8", "nvfp4"])
+@pytest.fixture(scope="module", params=["mxfp8", "nvfp4", "nvfp4_mse"])
 def qmodel(request):
     import looped_ngpt_b200 as lb
     qw = quantize_weights(make_weights(TINY, seed=0), request.param)

@@ -87,3 +87,61 @@ def test_decoded_products_exact_in_bf16(fmt):
     f = wd.astype(np.float32)
     assert np.array_equal(f.astype(np.float64), wd)
     assert np.all((f.view(np.uint32) & 0xFFFF) == 0)
+
+
+def test_nvfp4_mse_scales_never_worse_than_max_scaling():
+    """Per block, the MSE-selected scale's squared error is at most that of
+    the max-scaling scale (which is among the candidates), and strictly
+    smaller somewhere on Gaussian weights."""
+    w = rng.standard_normal((16, 128)) * 0.04
+    pm, sm, Sm = q.quant_nvfp4(w)
+    pe, se, Se = q.quant_nvfp4_mse(w)
+    assert Sm == Se
+    em = ((q.dequant_nvfp4(pm, sm, Sm) - w) ** 2).reshape(16, 8, 16).sum(-1)
+    ee = ((q.dequant_nvfp4(pe, se, Se) - w) ** 2).reshape(16, 8, 16).sum(-1)
+    assert np.all(ee <= em + 1e-18)
+    assert np.any(ee < em * 0.99)
+
+
+def test_nvfp4_mse_matches_scalar_search():
+    """Brute force, one block at a time in scalar Python: try every code of
+    the window around the max-scaling code, decode, keep the smallest sum of
+    squared errors (first found among codes taken from high to low)."""
+    w = rng.standard_normal((3, 48)) * 0.05
+    _, sb, S = q.quant_nvfp4_mse(w)
+    S = float(S)
+    e2 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for r in range(3):
+        for b in range(3):
+            blk = [float(v) for v in w[r, 16 * b:16 * b + 16]]
+            c_max = int(q.round_e4m3(max(abs(v) for v in blk) / (6 * S)))
+            best, best_err = None, None
+            for c in range(min(126, c_max + 1), max(1, c_max - 8) - 1, -1):
+                sc = float(q.e4m3_decode(c)) * S
+                err = 0.0
+                for v in blk:
+                    y = abs(v) / sc
+                    # nearest E2M1 magnitude, ties to the even code
+                    d = [abs(y - m) for m in e2]
+                    k = min(range(8), key=lambda i: (d[i], i % 2))
+                    if y >= 6.0:
+                        k = 7
+                    err += (abs(v) - e2[k] * sc) ** 2
+                if best_err is None or err < best_err:
+                    best, best_err = c, err
+            assert sb[r, b] == best, (r, b, sb[r, b], best)
+
+
+def test_nvfp4_mse_exact_block_has_zero_error():
+    """A block of E2M1 values (largest magnitude 6) times the scale of code
+    0x30 (0.5) and the tensor scale S = 2^-10 (fixed by a tensor maximum of
+    6 * 448 * 2^-10 in the other block) is reproduced exactly: the search
+    keeps the max-scaling code 0x30, whose error is 0."""
+    vals = np.array([0.5, -1.0, 1.5, 2.0, -3.0, 4.0, 0.0, 6.0] * 2)
+    S0 = 2.0 ** -10
+    w = np.zeros((1, 32))
+    w[0, :16] = vals * 0.5 * S0
+    w[0, 16] = 6.0 * 448.0 * S0
+    p, sb, S = q.quant_nvfp4_mse(w)
+    assert float(S) == S0 and sb[0, 0] == 0x30
+    assert np.array_equal(q.dequant_nvfp4(p, sb, S)[0, :16], w[0, :16])

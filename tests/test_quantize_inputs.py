@@ -28,7 +28,18 @@ def test_encoders_match_oracle_quantisers(w, name):
     assert np.float32(t1[0]) == np.float32(t2)
 
 
-@pytest.mark.parametrize("fmt,tol", [("mxfp8", 0.05), ("nvfp4", 0.35)])
+@pytest.mark.parametrize("name", ["blk0.w_qkvg", "blk3.w_down"])
+def test_mse_encoder_matches_oracle(w, name):
+    from synthetic.quantize import _encode_rows
+    m = bf16_bits_to_f32(w[name])
+    p1, s1, t1 = _encode_rows(m, "nvfp4_mse", rows=100)
+    p2, s2, t2 = quant.quant_nvfp4_mse(m)
+    assert np.array_equal(p1, p2) and np.array_equal(s1, s2)
+    assert np.float32(t1[0]) == np.float32(t2)
+
+
+@pytest.mark.parametrize("fmt,tol", [("mxfp8", 0.05), ("nvfp4", 0.35),
+                                     ("nvfp4_mse", 0.35)])
 def test_quantised_model_close_to_bf16(w, fmt, tol):
     """Weight-only quantisation perturbs the logits by a bounded amount
     (E4M3: ~2^-4 relative per weight; E2M1 much coarser)."""
