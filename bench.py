@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--no-quant", action="store_true",
                     help="skip the MXFP8 / NVFP4 weight-only models (B=1 at "
                          "2048 context and B=4 at 131072 context, k=2)")
+    ap.add_argument("--no-spec", action="store_true",
+                    help="skip self-speculative decoding (k=1 draft, k=4 "
+                         "verify, 4 drafts per step)")
     ap.add_argument("--no-per-loop", action="store_true",
                     help="skip the per_loop rows of the 2048-token workload")
     ap.add_argument("--profile-decode", type=int, default=0, metavar="K",
@@ -373,6 +376,14 @@ def run_gpu(args, rank, world, local):
     barrier(world)
     del cache, headline["cache"]
     torch.cuda.empty_cache()
+    if not args.no_spec:
+        sp = run_spec(gm, prompt)
+        ar = out.get("per_loop", {}).get("decode_tok_s", {}).get("k4")
+        if ar:
+            sp["autoregressive_k4_per_loop_tok_s"] = ar
+            sp["speedup_vs_autoregressive"] = sp["tok_s"] / ar
+            sp["break_even_tokens_per_step"] = sp["ms_per_step"] / 1e3 * ar
+        out["self_speculative_b1_k1_draft_k4_verify"] = sp
     if not args.no_long:
         out["long_context"] = run_long(gm, args, hbm_peak, dev)
         out["prefill_t8192_k4_per_loop"] = run_prefill_long(gm, tc_peak, dev)
@@ -382,6 +393,40 @@ def run_gpu(args, rank, world, local):
         out["quantized"] = run_quant(w, args, hbm_peak, dev)
     return dict(out=out, headline=headline, e2e_dt=e2e_dt, w=w,
                 hbm_peak=hbm_peak, tc_peak=tc_peak, peak_kind=peak_kind)
+
+
+def run_spec(gm, prompt, steps=16, gamma=4, k_draft=1, k_verify=4):
+    """Self-speculative greedy decoding after the prompt (per_loop cache):
+    gamma drafts at k_draft loops, one verify pass at k_verify.  Every step
+    synchronises once (the emitted count); wall-clock timing."""
+    import torch
+    T = prompt.shape[1]
+    cache = gm.new_cache(1, T + (steps + 4) * (gamma + 1) + 16, T,
+                         kv_mode="per_loop", max_loops=k_verify)
+    ws = gm.workspace(1, T)
+    sws = gm.spec_workspace(1, gamma)
+    _, a = gm.prefill(cache, prompt, k_verify, ws)
+    last = a.clone()
+    for _ in range(3):
+        out, n = gm.spec_decode_step(cache, last, gamma, k_draft, k_verify, sws)
+        last = out[:, n - 1].contiguous()
+    torch.cuda.synchronize()
+    emitted = []
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        out, n = gm.spec_decode_step(cache, last, gamma, k_draft, k_verify, sws)
+        last = out[:, n - 1].contiguous()
+        emitted.append(n)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert gm.sync_status() == 0, "device-side check failed"
+    # cost of one step when no draft is kept, and the break-even count
+    res = {"tok_s": sum(emitted) / dt, "ms_per_step": dt / steps * 1e3,
+           "tokens_per_step": sum(emitted) / steps, "gamma": gamma,
+           "k_draft": k_draft, "k_verify": k_verify, "emitted": emitted}
+    del cache, ws, sws
+    torch.cuda.empty_cache()
+    return res
 
 
 def timed_decode(gm, B, ctx, k, mode, steps, hbm_peak, dev, prompt=None):

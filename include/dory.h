@@ -79,8 +79,11 @@ typedef struct {
  *   "blk<i>.<w>.s"  uint8 scales: MXFP8 E8M0 [N, K/32]; NVFP4 E4M3 [N, K/16]
  *   "blk<i>.<w>.t"  f32 [1] per-tensor scale (NVFP4 only)
  * with w = e4m3(q) * 2^(s - 127), or e2m1(q) * e4m3(s) * t.  Embedding and
- * LM head stay BF16.  Quantised models run decode-style calls (T = 1,
- * B <= 8); other calls return DORY_ERR_UNSUPPORTED.
+ * LM head stay BF16.  One-token calls of up to 8 sequences decode the
+ * weights in registers inside the GEMV; other calls (prefill, batches over
+ * 8) decode each projection to bf16 in the workspace (exact: the products
+ * have at most 8 significant bits) just before its tensor-core GEMM, which
+ * applies the NVFP4 tensor scale t to its products.
  *
  * One named weight tensor in device memory (non-owning).  Names and shapes
  * (row-major, K = contraction axis last):
@@ -196,6 +199,62 @@ int dory_decode_step(dory_model* m, dory_cache* c, const int32_t* d_tokens,
                      int B, int n_loops, int kv_mode, float* d_logits,
                      int32_t* d_argmax, void* d_workspace, int64_t ws_bytes,
                      void* stream);
+
+/* Self-speculative decoding ("Dory1.0-4B: A Looped Normalized-GPT", §6.2
+ * Self-Speculative Decoding): the same weights at k_draft loops draft gamma
+ * tokens one decode step at a time (greedy), then the k_verify-loop model
+ * checks the last accepted token and the gamma drafts in one multi-token
+ * pass, and rejection sampling decides how many drafts to keep.
+ *   - d_last int32 [B]: the last accepted token of every sequence (not yet
+ *     in the cache).  d_tokens_out int32 [B, gamma + 1] receives the
+ *     emitted tokens, *n_out (host) their count n (1 <= n <= gamma + 1, the
+ *     same for every sequence; entries past n are -1).  The cache advances
+ *     by n: the emitted tokens except the last one, which is the next
+ *     d_last.
+ *   - temperature 0: greedy.  Draft j is kept while it equals the
+ *     verifier's argmax, and the token after the kept drafts is the
+ *     verifier's argmax there, so the output equals plain greedy decoding
+ *     at k_verify loops.  temperature > 0: draft j is kept with probability
+ *     p(draft j), p = softmax(logits / temperature) of the verifier, tested
+ *     against d_uniform [B, gamma + 1] (values in [0, 1); entry j for draft
+ *     j + 1); at the first rejection the token is drawn by inverse CDF with
+ *     entry gamma from p restricted to the other tokens, and if all drafts
+ *     are kept from p at the last position.  The output is distributed as
+ *     sampling from the k_verify-loop model.  With several sequences every
+ *     sequence advances by the smallest count; a sequence that kept more
+ *     emits its own kept draft at the last position.
+ *   - per_loop caches only, as on the pages (DORY_ERR_CACHE otherwise: in
+ *     last_loop mode the tokens of one multi-token pass read each other's
+ *     same-loop entries, so a verify pass would not reproduce one-token
+ *     decoding).  The cache must be bound with max_loops >= k_verify and
+ *     filled at k_verify loops (the draft reads the first k_draft slots,
+ *     which the verifier's passes write).  The verifier rewrites every slot
+ *     of the drafted positions before reading them.
+ *   - The draft steps and the verify pass are replayed from CUDA graphs
+ *     after their first use with the same pointers.  This entry point
+ *     synchronises `stream` once, to read n.
+ *   - Workspace: dory_spec_workspace_bytes.  BF16 weights only
+ *     (DORY_ERR_UNSUPPORTED otherwise).  Errors as dory_prefill; gamma in
+ *     1..15 with gamma + 1 <= max_chunk. */
+int dory_spec_workspace_bytes(const dory_model* m, int B, int gamma,
+                              int64_t* bytes);
+int dory_spec_decode_step(dory_model* m, dory_cache* c, const int32_t* d_last,
+                          int B, int gamma, int k_draft, int k_verify,
+                          float temperature, const float* d_uniform,
+                          int32_t* d_tokens_out, int* n_out,
+                          void* d_workspace, int64_t ws_bytes, void* stream);
+
+/* Test access to the acceptance step of dory_spec_decode_step alone, on
+ * caller buffers: d_draft int32 [B, gamma + 1] (last token, then drafts),
+ * d_target int32 [B, gamma + 1] (verifier argmax; greedy), d_logits f32
+ * [B, gamma + 1, V] and d_uniform f32 [B, gamma + 1] (temperature > 0).
+ * Writes d_tokens_out [B, gamma + 1] and d_scratch int32 [B + 2]
+ * (d_scratch[0] = n). */
+int dory_debug_spec_accept(const int32_t* d_draft, const int32_t* d_target,
+                           const float* d_logits, const float* d_uniform,
+                           int B, int gamma, int V, float temperature,
+                           int32_t* d_tokens_out, int32_t* d_scratch,
+                           void* stream);
 
 /* Copy the final residual state s (input of the LM head, f32) of the last
  * call that used this workspace: [B, T, d] for a logits_all prefill, else

@@ -65,6 +65,12 @@ SIGNATURES = {
     "dory_debug_gemv": (c_int, [_P, c_char_p, _P, c_int, _P, c_int,
                                 POINTER(c_int), _P]),
     "dory_copy_state": (c_int, [_P, _P, c_int, c_int, c_int, _P, _P]),
+    "dory_spec_workspace_bytes": (c_int, [_P, c_int, c_int, _I64P]),
+    "dory_spec_decode_step": (c_int, [_P, _P, _P, c_int, c_int, c_int, c_int,
+                                      ctypes.c_float, _P, _P, POINTER(c_int),
+                                      _P, c_int64, _P]),
+    "dory_debug_spec_accept": (c_int, [_P, _P, _P, _P, c_int, c_int, c_int,
+                                       ctypes.c_float, _P, _P, _P]),
     "dory_sync_status": (c_int, [_P, _P]),
     "dory_profile_enable": (c_int, [_P, c_int]),
     "dory_profile_read": (c_int, [_P, POINTER(DoryKernelStat), c_int,

@@ -70,6 +70,29 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
                : "memory");
 }
 
+// Share of prefetch ranges taken by one of `parts` cooperating CTAs: each
+// range is cut into `parts` 16-byte-aligned slices, and the slice of part
+// `part` is issued in chunks of up to 32 KB by `nthr` threads (thread
+// index `t`).
+template <int NR>
+__device__ __forceinline__ void l2_prefetch_share(const void* const (&p)[NR],
+                                                  const long (&bytes)[NR],
+                                                  int part, int parts, int t,
+                                                  int nthr) {
+  constexpr long kChunk = 32768;
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    if (!p[r] || bytes[r] <= 0) continue;
+    const long per = ((bytes[r] + parts - 1) / parts + 15) & ~15L;
+    const long lo = (long)part * per;
+    const long hi = lo + per < bytes[r] ? lo + per : bytes[r];
+    for (long off = lo + (long)t * kChunk; off < hi; off += (long)nthr * kChunk) {
+      const long n = hi - off < kChunk ? hi - off : kChunk;
+      prefetch_l2(static_cast<const char*>(p[r]) + off, (uint32_t)n);
+    }
+  }
+}
+
 __device__ __forceinline__ float sigmoidf_(float x) {
   return 1.f / (1.f + __expf(-x));
 }

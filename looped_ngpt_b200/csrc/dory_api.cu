@@ -173,6 +173,8 @@ struct WS {
   float *s0, *s1, *sfin, *x, *qkvg, *gate, *h, *lg,
       *rope, *amax_val;
   bf16 *s_bf, *a, *mact, *qb;
+  bf16* wdq;          // quantised models, tensor-core calls: the projection
+                      // being multiplied, dequantised to bf16
   int* amax_idx;
   size_t total;
 };
@@ -217,6 +219,11 @@ WS ws_layout(const dory_model* m, int B, int T, char* base) {
   w.amax_val = (float*)take((size_t)B * kArgmaxSlots * 4);
   w.amax_idx = (int*)take((size_t)B * kArgmaxSlots * 4);
   w.lg = (float*)take(B > 8 ? (size_t)B * dm.V * 4 : 0);
+  size_t wq = 0;
+  if (m->wfmt != DORY_W_BF16 && !(T == 1 && B <= 8))
+    wq = std::max(std::max((size_t)dm.rows_qkvg * dm.d, (size_t)dm.d * dm.qdim),
+                  std::max((size_t)2 * dm.F * dm.d, (size_t)dm.d * dm.F)) * 2;
+  w.wdq = (bf16*)take(wq);
   w.total = off;
   return w;
 }
@@ -588,12 +595,29 @@ int gemv_run(dory_model* m, const GemvArgs& g0, cudaStream_t st,
 // Returns the number of K-split partials written (C + z * M * ldc).
 int gemm_run(dory_model* m, const bf16* A, int lda, const bf16* W, float* C,
              int ldc, int M, int N, int K, const float* scale,
-             cudaStream_t st, const char* name, int max_splits = 1) {
+             cudaStream_t st, const char* name, int max_splits = 1,
+             const float* out_scale = nullptr) {
   Prof p(m, st, name,
          (double)M * K * 2 + (double)N * K * 2 + (double)M * N * 4,
          2.0 * M * N * K);
   return launch_gemm_bf16(A, lda, W, C, ldc, M, N, K, scale, st, max_splits,
-                          (long)M * ldc);
+                          (long)M * ldc, out_scale);
+}
+
+// BF16 operand of a projection for the tensor-core GEMM: the weights
+// themselves, or (quantised models) their exact bf16 decode written to the
+// workspace just before the GEMM that reads it.  The NVFP4 tensor scale is
+// left out and applied by the GEMM to its products (*out_scale).
+const bf16* gemm_weight(dory_model* m, const QMat& q, long N, long K, bf16* wdq,
+                        cudaStream_t st, const float** out_scale) {
+  *out_scale = nullptr;
+  if (q.w) return q.w;
+  const int fmt = m->wfmt == DORY_W_MXFP8 ? WF_MXFP8 : WF_NVFP4;
+  const double per = fmt == WF_MXFP8 ? 1.0 + 1.0 / 32 : 0.5 + 1.0 / 16;
+  Prof p(m, st, "dequant", (double)N * K * (per + 2.0), 0);
+  launch_dequant_bf16(fmt, q.q, q.s, N, (int)K, wdq, st);
+  *out_scale = q.t;
+  return wdq;
 }
 
 struct CallCtx {
@@ -617,6 +641,48 @@ KVSlot slot_for(const dory_cache* c, int i, int t) {
 }
 
 bool use_gemv(int B, int T) { return T == 1 && B <= 8; }
+
+// Decode attention at short context reads a few MB and is bound by latency,
+// leaving HBM idle: once its predecessor has finished, it asks L2 for a
+// leading share of the gate and of the up rows of W_gu, which the gate/up
+// GEMV then reads from L2.  Measured at batch 1, k = 2, 2048-token context
+// (percent of the rows -> tok/s): 0 -> 306, 10 -> 310, 20 -> 313,
+// 30 -> 307, 35 -> 301; W_o (whose GEMV loads it during the attention
+// anyway) and W_down shares only cost.  Issued before the dependency wait
+// the same prefetch slowed the step (it competes with the QKVG GEMV's own
+// stream).  Above kL2pfMaxKvBytes of K/V per call the attention itself
+// streams HBM and nothing is prefetched.  DORY_L2PF_WO / _GU / _DOWN
+// (percent) override the shares.
+constexpr double kL2pfMaxKvBytes = 64e6;
+// A percentage from the environment as a fraction in [0, 1].
+double env_fraction(const char* name, double dflt) {
+  const char* e = getenv(name);
+  const double v = e ? atof(e) / 100.0 : dflt;
+  return v < 0.0 ? 0.0 : (v > 1.0 ? 1.0 : v);
+}
+void set_l2_prefetch(const dory_model* m, const BlockW& bw, L2Range* r) {
+  const double f_o = env_fraction("DORY_L2PF_WO", 0.0);
+  const double f_gu = env_fraction("DORY_L2PF_GU", 0.2);
+  const double f_dn = env_fraction("DORY_L2PF_DOWN", 0.0);
+  const Dims& dm = m->dm;
+  // bytes per weight row of a projection with K inputs
+  auto row_bytes = [&](const QMat& q, long K) -> long {
+    if (q.w) return K * 2;
+    return m->wfmt == DORY_W_MXFP8 ? K : K / 2;
+  };
+  auto base = [](const QMat& q) -> const char* {
+    return q.w ? (const char*)q.w : (const char*)q.q;
+  };
+  const long ro = row_bytes(bw.m_o, dm.qdim);
+  const long rg = row_bytes(bw.m_gu, dm.d);
+  const long n_o = (long)(dm.d * f_o);
+  const long n_g = (long)(dm.F * f_gu);
+  r[0] = L2Range{base(bw.m_o), n_o * ro};
+  r[1] = L2Range{base(bw.m_gu), n_g * rg};
+  r[2] = L2Range{base(bw.m_gu) + (long)dm.F * rg, n_g * rg};
+  const long rd = row_bytes(bw.m_down, dm.F);
+  r[3] = L2Range{base(bw.m_down), (long)(dm.d * f_dn) * rd};
+}
 
 // Enqueue one forward pass: embedding, input blocks, n_loops passes of the
 // recurrent blocks with re-injection, output blocks, LM head.
@@ -681,12 +747,15 @@ void enqueue_forward(const CallCtx& x) {
                            dm.d, x.st, prev_S);
         std::swap(cur, other);
       }
+      const float* osc = nullptr;
+      const bf16* Wqkvg = gemm_weight(m, bw.m_qkvg, dm.rows_qkvg, dm.d, w.wdq,
+                                      x.st, &osc);
       if (x.T == 1) {
         // one partial: the attention cluster's owner warps sum the q/k/v
         // partials on the critical path before the cluster's first barrier;
         // at B = 64 a 5-way split saved 0.45 ms here and cost 1.2 ms there
-        gemm_run(m, w.s_bf, dm.d, bw.w_qkvg, w.qkvg, dm.rows_qkvg, x.M,
-                 dm.rows_qkvg, dm.d, nullptr, x.st, "gemm_qkvg");
+        gemm_run(m, w.s_bf, dm.d, Wqkvg, w.qkvg, dm.rows_qkvg, x.M,
+                 dm.rows_qkvg, dm.d, nullptr, x.st, "gemm_qkvg", 1, osc);
       } else {
         QkvGemmArgs qg{};
         qg.M = x.M; qg.T = x.T; qg.dm = dm; qg.s_q = bw.s_q; qg.s_k = bw.s_k;
@@ -697,7 +766,7 @@ void enqueue_forward(const CallCtx& x) {
                (double)x.M * dm.d * 2 + (double)dm.rows_qkvg * dm.d * 2 +
                    (double)x.M * (dm.qdim * 6.0 + dm.kvdim * 4.0),
                2.0 * x.M * dm.rows_qkvg * dm.d);
-        launch_gemm_qkv(w.s_bf, dm.d, bw.w_qkvg, qg, x.st);
+        launch_gemm_qkv(w.s_bf, dm.d, Wqkvg, qg, x.st, osc);
       }
     }
     if (x.T == 1) {
@@ -709,6 +778,8 @@ void enqueue_forward(const CallCtx& x) {
       da.kv = kv; da.g = geo; da.a_out = w.a; da.err = m->d_status;
       const double nk = full ? x.n_ctx0 + 1.0
                              : std::min(x.n_ctx0 + 1.0, (double)dm.window);
+      if (gemv && x.B * dm.Hkv * nk * dm.hd * 4.0 < kL2pfMaxKvBytes)
+        set_l2_prefetch(m, bw, da.l2pf);
       Prof p(m, x.st, "attn_decode",
              x.B * (dm.Hkv * nk * dm.hd * 4.0 + S_qkvg * dm.rows_qkvg * 4.0),
              4.0 * x.B * dm.Hq * nk * dm.hd);
@@ -738,8 +809,10 @@ void enqueue_forward(const CallCtx& x) {
       g.pro = PRO_BF16; g.xin = w.a; g.xin_stride = dm.qdim;
       S_o = gemv_run(m, g, x.st, "gemv_o", &bw.m_o);
     } else {
-      S_o = gemm_run(m, w.a, dm.qdim, bw.w_o, w.h, dm.d, x.M, dm.d, dm.qdim,
-                     nullptr, x.st, "gemm_o", slabs);
+      const float* osc = nullptr;
+      const bf16* Wo = gemm_weight(m, bw.m_o, dm.d, dm.qdim, w.wdq, x.st, &osc);
+      S_o = gemm_run(m, w.a, dm.qdim, Wo, w.h, dm.d, x.M, dm.d, dm.qdim,
+                     nullptr, x.st, "gemm_o", slabs, osc);
     }
 
     // ---- MLP sublayer ---------------------------------------------------
@@ -764,15 +837,20 @@ void enqueue_forward(const CallCtx& x) {
       }
       std::swap(cur, other);
       {
+        const float* osc = nullptr;
+        const bf16* Wgu = gemm_weight(m, bw.m_gu, 2L * dm.F, dm.d, w.wdq, x.st,
+                                      &osc);
         Prof p(m, x.st, "gemm_gateup",
                (double)x.M * dm.d * 2 + 2.0 * dm.F * dm.d * 2 +
                    (double)x.M * dm.F * 2,
                2.0 * x.M * 2.0 * dm.F * dm.d);
-        launch_gemm_swiglu(w.s_bf, dm.d, bw.w_gu, w.mact, dm.F, x.M, dm.F, dm.d,
-                           x.st);
+        launch_gemm_swiglu(w.s_bf, dm.d, Wgu, w.mact, dm.F, x.M, dm.F, dm.d,
+                           x.st, osc);
       }
-      prev_S = gemm_run(m, w.mact, dm.F, bw.w_down, w.h, dm.d, x.M, dm.d, dm.F,
-                        nullptr, x.st, "gemm_down", slabs);
+      const float* osc = nullptr;
+      const bf16* Wd = gemm_weight(m, bw.m_down, dm.d, dm.F, w.wdq, x.st, &osc);
+      prev_S = gemm_run(m, w.mact, dm.F, Wd, w.h, dm.d, x.M, dm.d, dm.F,
+                        nullptr, x.st, "gemm_down", slabs, osc);
     }
     prev_alpha = bw.alpha_m;
   }
@@ -841,21 +919,31 @@ void enqueue_forward(const CallCtx& x) {
   launch_advance(x.c->d_nctx, x.T, x.st);
 }
 
+// run_call flags: replay the call from a CUDA graph once its launch plan
+// has been seen with the same pointers and shape (calls of up to kMaxGraphT
+// tokens); a step of self-speculative decoding (loop counts other than the
+// one a per_loop cache is bound to are allowed: the draft runs fewer loops
+// than the verifier, whose pass rewrites every slot of the drafted
+// positions).
+constexpr int kCallGraph = 1, kCallSpec = 2;
+constexpr int kMaxGraphT = 16;
+
 int run_call(dory_model* m, dory_cache* c, const int32_t* tokens, int B,
              int T, int n_loops, int kv_mode, int logits_all, float* logits,
              int32_t* argmax, void* ws, int64_t ws_bytes, void* stream,
-             bool decode) {
+             int flags) {
+  const bool graphs_ok = (flags & kCallGraph) && T <= kMaxGraphT;
+  const bool spec = (flags & kCallSpec) != 0;
   if (!m || !c || c->m != m || !tokens || !ws) return DORY_ERR_ARG;
   if (B != c->B || T < 1 || T > c->max_chunk || n_loops < 1) return DORY_ERR_ARG;
   if (logits_all && !logits) return DORY_ERR_ARG;
   if ((uintptr_t)ws & 255) return DORY_ERR_ARG;
   if (kv_mode != c->kv_mode) return DORY_ERR_CACHE;
   if (kv_mode == DORY_KV_PER_LOOP &&
-      (n_loops > c->max_loops || (c->loops_bound && c->loops_bound != n_loops)))
+      (n_loops > c->max_loops ||
+       (!spec && c->loops_bound && c->loops_bound != n_loops)))
     return DORY_ERR_CACHE;
   if ((int64_t)c->n_ctx + T > c->max_ctx) return DORY_ERR_CACHE;
-  // quantised weights: decode-style calls only (one token, B <= 8)
-  if (m->wfmt != DORY_W_BF16 && !use_gemv(B, T)) return DORY_ERR_UNSUPPORTED;
   const WS w = ws_layout(m, B, T, (char*)ws);
   if ((int64_t)w.total > ws_bytes) return DORY_ERR_WORKSPACE;
   CallCtx x{m, c, w, B, T, B * T, n_loops, logits_all, c->n_ctx, tokens,
@@ -864,8 +952,9 @@ int run_call(dory_model* m, dory_cache* c, const int32_t* tokens, int B,
   take_host_failure();
 
   bool done = false;
-  if (decode && m->use_graphs && !m->prof) {
-    const GraphKey key(B, n_loops, tokens, logits, argmax, ws, c);
+  if (graphs_ok && m->use_graphs && !m->prof) {
+    const GraphKey key(B, n_loops + 256 * T + (logits_all << 24), tokens,
+                       logits, argmax, ws, c);
     if (m->graphs.size() > 64 && !m->graphs.count(key)) {
       for (auto& kv : m->graphs)
         if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
@@ -906,7 +995,8 @@ int run_call(dory_model* m, dory_cache* c, const int32_t* tokens, int B,
   if (take_host_failure() | (cudaGetLastError() != cudaSuccess))
     return DORY_ERR_CUDA;
   c->n_ctx += T;
-  if (kv_mode == DORY_KV_PER_LOOP && !c->loops_bound) c->loops_bound = n_loops;
+  if (kv_mode == DORY_KV_PER_LOOP && !c->loops_bound && !spec)
+    c->loops_bound = n_loops;
   return DORY_OK;
 }
 
@@ -919,7 +1009,7 @@ int dory_prefill(dory_model* m, dory_cache* c, const int32_t* d_tokens, int B,
                  float* d_logits, int32_t* d_argmax, void* d_workspace,
                  int64_t ws_bytes, void* stream) {
   return run_call(m, c, d_tokens, B, T, n_loops, kv_mode, logits_all ? 1 : 0,
-                  d_logits, d_argmax, d_workspace, ws_bytes, stream, false);
+                  d_logits, d_argmax, d_workspace, ws_bytes, stream, 0);
 }
 
 int dory_decode_step(dory_model* m, dory_cache* c, const int32_t* d_tokens,
@@ -927,7 +1017,151 @@ int dory_decode_step(dory_model* m, dory_cache* c, const int32_t* d_tokens,
                      int32_t* d_argmax, void* d_workspace, int64_t ws_bytes,
                      void* stream) {
   return run_call(m, c, d_tokens, B, 1, n_loops, kv_mode, 0, d_logits,
-                  d_argmax, d_workspace, ws_bytes, stream, true);
+                  d_argmax, d_workspace, ws_bytes, stream, kCallGraph);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Self-speculative decoding scratch at the head of the caller's workspace:
+// draft tokens step-major [gamma+1][B] and row-major [B][gamma+1], the
+// verifier's picks [B][gamma+1] and logits [B][gamma+1][V], per-row
+// accepted counts, the emitted count.  The forward-pass workspace follows.
+struct SpecWS {
+  int *steps, *rows, *target, *r, *n_out;
+  float* logits;
+  size_t total;
+};
+
+SpecWS spec_layout(const dory_model* m, int B, int gamma, char* base) {
+  const size_t G1 = (size_t)gamma + 1;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  SpecWS w;
+  w.steps = (int*)take(G1 * B * 4);
+  w.rows = (int*)take(G1 * B * 4);
+  w.target = (int*)take(G1 * B * 4);
+  w.r = (int*)take((size_t)B * 4);
+  w.n_out = (int*)take(4);
+  w.logits = (float*)take(G1 * B * m->dm.V * 4);
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dory_spec_workspace_bytes(const dory_model* m, int B, int gamma,
+                              int64_t* bytes) {
+  if (!m || !bytes || B < 1 || gamma < 1 || gamma > 15) return DORY_ERR_ARG;
+  int64_t fw = 0;
+  const int rc = dory_workspace_bytes(m, B, gamma + 1, &fw);
+  if (rc) return rc;
+  *bytes = (int64_t)spec_layout(m, B, gamma, nullptr).total + fw;
+  return DORY_OK;
+}
+
+int dory_spec_decode_step(dory_model* m, dory_cache* c, const int32_t* d_last,
+                          int B, int gamma, int k_draft, int k_verify,
+                          float temperature, const float* d_uniform,
+                          int32_t* d_tokens_out, int* n_out,
+                          void* d_workspace, int64_t ws_bytes, void* stream) {
+  if (!m || !c || c->m != m || !d_last || !d_tokens_out || !n_out ||
+      !d_workspace || B != c->B || gamma < 1 || gamma > 15 || k_draft < 1 ||
+      k_verify < k_draft || !(temperature >= 0.f) ||
+      (temperature > 0.f && !d_uniform) || ((uintptr_t)d_workspace & 255))
+    return DORY_ERR_ARG;
+  *n_out = 0;
+  if (m->wfmt != DORY_W_BF16) return DORY_ERR_UNSUPPORTED;
+  if (gamma + 1 > c->max_chunk) return DORY_ERR_ARG;
+  const int n0 = c->n_ctx;
+  if ((int64_t)n0 + gamma + 1 > c->max_ctx) return DORY_ERR_CACHE;
+  // per_loop only: there a multi-token pass computes what one-token steps
+  // compute, so the verifier's picks are those of plain decoding (in
+  // last_loop mode a chunk's tokens read same-loop entries of each other)
+  if (c->kv_mode != DORY_KV_PER_LOOP || k_verify > c->max_loops ||
+      (c->loops_bound && c->loops_bound != k_verify))
+    return DORY_ERR_CACHE;
+  const SpecWS sw = spec_layout(m, B, gamma, (char*)d_workspace);
+  if ((int64_t)sw.total >= ws_bytes) return DORY_ERR_WORKSPACE;
+  char* fws = (char*)d_workspace + sw.total;
+  const int64_t fws_bytes = ws_bytes - (int64_t)sw.total;
+  const cudaStream_t st = (cudaStream_t)stream;
+  const int G1 = gamma + 1;
+  cudaGetLastError();
+  if (cudaMemcpyAsync(sw.steps, d_last, (size_t)B * 4, cudaMemcpyDeviceToDevice,
+                      st) != cudaSuccess)
+    return DORY_ERR_CUDA;
+  // draft: gamma greedy decode steps at k_draft loops, each token written
+  // straight into the input of the next
+  for (int j = 0; j < gamma; ++j) {
+    const int rc = run_call(m, c, sw.steps + (size_t)j * B, B, 1, k_draft,
+                            c->kv_mode, 0, nullptr, sw.steps + (size_t)(j + 1) * B,
+                            fws, fws_bytes, stream, kCallGraph | kCallSpec);
+    if (rc) {
+      c->n_ctx = n0;
+      launch_set_nctx(c->d_nctx, n0, st);
+      return rc;
+    }
+  }
+  // verify: the last accepted token and the gamma drafts at k_verify loops
+  // in one multi-token pass from position n0; every slot of those positions
+  // is rewritten before it is read
+  c->n_ctx = n0;
+  launch_set_nctx(c->d_nctx, n0, st);
+  launch_spec_transpose(sw.steps, sw.rows, B, G1, st);
+  int rc = run_call(m, c, sw.rows, B, G1, k_verify, c->kv_mode, 1, sw.logits,
+                    sw.target, fws, fws_bytes, stream, kCallGraph | kCallSpec);
+  if (rc) {
+    c->n_ctx = n0;
+    launch_set_nctx(c->d_nctx, n0, st);
+    return rc;
+  }
+  SpecArgs a{};
+  a.draft = sw.rows; a.target = sw.target; a.logits = sw.logits;
+  a.uniform = d_uniform; a.B = B; a.gamma = gamma; a.V = m->dm.V;
+  a.inv_temp = temperature > 0.f ? 1.f / temperature : 0.f;
+  a.r = sw.r; a.out = d_tokens_out; a.n_out = sw.n_out; a.n_ctx = c->d_nctx;
+  a.n0 = n0;
+  launch_spec_accept(a, st);
+  int n = 0;
+  if (cudaGetLastError() != cudaSuccess ||
+      cudaMemcpyAsync(&n, sw.n_out, 4, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess || n < 1 || n > G1) {
+    c->n_ctx = n0;
+    return DORY_ERR_CUDA;
+  }
+  c->n_ctx = n0 + n;
+  if (!c->loops_bound) c->loops_bound = k_verify;
+  *n_out = n;
+  return DORY_OK;
+}
+
+int dory_debug_spec_accept(const int32_t* d_draft, const int32_t* d_target,
+                           const float* d_logits, const float* d_uniform,
+                           int B, int gamma, int V, float temperature,
+                           int32_t* d_tokens_out, int32_t* d_scratch,
+                           void* stream) {
+  if (!d_draft || !d_target || !d_tokens_out || !d_scratch || B < 1 ||
+      gamma < 1 || V < 2 || !(temperature >= 0.f) ||
+      (temperature > 0.f && (!d_uniform || !d_logits)))
+    return DORY_ERR_ARG;
+  SpecArgs a{};
+  a.draft = d_draft; a.target = d_target; a.logits = d_logits;
+  a.uniform = d_uniform; a.B = B; a.gamma = gamma; a.V = V;
+  a.inv_temp = temperature > 0.f ? 1.f / temperature : 0.f;
+  a.r = d_scratch + 2; a.out = d_tokens_out; a.n_out = d_scratch;
+  a.n_ctx = d_scratch + 1; a.n0 = 0;
+  cudaGetLastError();
+  launch_spec_accept(a, (cudaStream_t)stream);
+  return cuda_rc(cudaGetLastError());
 }
 
 int dory_copy_state(const dory_model* m, const void* d_workspace, int B,
@@ -1009,9 +1243,9 @@ extern "C" int dory_decode_step_static(dory_model* m, dory_cache* c,
   void* ws = nullptr;
   const int rc = static_ws_address(&ws);
   if (rc) return rc;
-  // decode = false: the kernels are launched directly, never via a graph.
+  // flags 0: the kernels are launched directly, never via a graph.
   return run_call(m, c, d_tokens, B, 1, n_loops, kv_mode, 0, d_logits,
-                  d_argmax, ws, (int64_t)DORY_STATIC_WS_BYTES, stream, false);
+                  d_argmax, ws, (int64_t)DORY_STATIC_WS_BYTES, stream, 0);
 }
 
 // A bounded wait that runs out on purpose: one thread waits on an mbarrier

@@ -148,6 +148,12 @@ int gemv_splits(const GemvArgs& a);
 int gemv_grid(const GemvArgs& a, int num_sms);
 void launch_gemv(const GemvArgs& a, int grid, cudaStream_t st);
 
+// Whole quantised matrix [N][K] to bf16 (e4m3 * 2^(e8m0 - 127), or
+// e2m1 * e4m3 without the NVFP4 tensor scale; exact in bf16), the operand
+// of the tensor-core GEMM for multi-token calls of quantised models.
+void launch_dequant_bf16(int fmt, const uint8_t* Wq, const uint8_t* Ws, long N,
+                         int K, bf16* out, cudaStream_t st);
+
 // Decode rows [row0, row0 + nrows) of a quantised matrix to f32 (the values
 // the GEMV multiplies: e4m3 * 2^(e8m0 - 127), or e2m1 * e4m3 without the
 // NVFP4 tensor scale).  out [nrows][K].
@@ -212,6 +218,14 @@ inline bool make_act_map(CUtensorMap* m, const void* ptr, long rows, long cols,
 
 // Decode (one token per sequence): RoPE/QK-norm/KV write, split-KV attention,
 // split merge and gate in one kernel.
+// A byte range of immutable data (weights) that a kernel asks the L2 cache
+// to fetch ahead of the kernels that will read it.
+struct L2Range {
+  const void* p;
+  long bytes;          // multiple of 16; p 16-byte aligned
+};
+constexpr int kMaxL2Ranges = 4;
+
 struct DecAttnArgs {
   const float* qkvg;   // QKVG partials [S][B][rows_qkvg]
   int S, B;
@@ -223,6 +237,9 @@ struct DecAttnArgs {
   KVSlot kv; CacheGeo g;
   bf16* a_out;         // [B][qdim]
   int* err;
+  // weights of the following projections, fetched into L2 while this
+  // kernel (latency-bound at short context) leaves HBM idle
+  L2Range l2pf[kMaxL2Ranges];
 };
 // kv_maps: the TMA maps of this layer slot's K and V (make_kv_tile_map).
 void launch_attn_decode(const DecAttnArgs& a, const CUtensorMap* kv_maps,
@@ -240,15 +257,19 @@ bool make_kv_tile_map(CUtensorMap* m, const void* ptr, long rows, int hd);
 // the output has fewer tiles than SMs (decode batches) and max_splits > 1,
 // K is split: split z writes its partial to C + z * slab.  Returns the number
 // of partials written (1 without a split).
+// out_scale (device scalar or null) multiplies every product: the f32
+// tensor scale of NVFP4 weights dequantised without it.
 int launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
                      int M, int N, int K, const float* col_scale,
-                     cudaStream_t st, int max_splits = 1, long slab = 0);
+                     cudaStream_t st, int max_splits = 1, long slab = 0,
+                     const float* out_scale = nullptr);
 // Number of K-split partials launch_gemm_bf16 writes for this shape and
 // max_splits (without a column scale).
 int gemm_split_count(int M, int N, int K, int max_splits);
 // m[M, F] = silu(A W_g^T) * (A W_u^T) as bf16, W = [W_g; W_u] (2F rows).
 void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
-                        int ldm, int M, int F, int K, cudaStream_t st);
+                        int ldm, int M, int F, int K, cudaStream_t st,
+                        const float* out_scale = nullptr);
 // Prefill q/k/v/gate projection with the RoPE, per-head L2 norm, scales,
 // KV-cache write and gate sigmoid in the GEMM epilogue (one tile column per
 // head).  A: bf16 [M][d] activations.
@@ -263,7 +284,27 @@ struct QkvGemmArgs {
   float* gate_out;     // [M][qdim]
 };
 void launch_gemm_qkv(const bf16* A, int lda, const bf16* W,
-                     const QkvGemmArgs& q, cudaStream_t st);
+                     const QkvGemmArgs& q, cudaStream_t st,
+                     const float* out_scale = nullptr);
+// ------------------------------------------------- speculative decoding ----
+struct SpecArgs {
+  const int* draft;     // [B][gamma+1]: last accepted token, then the drafts
+  const int* target;    // [B][gamma+1]: the verifier's argmax per position
+  const float* logits;  // [B][gamma+1][V]: verifier logits (inv_temp > 0)
+  const float* uniform; // [B][gamma+1]: u_j for the test of draft j + 1,
+                        // u_gamma for the one draw from the residual
+  int B, gamma, V;
+  float inv_temp;       // 1 / temperature; 0 = greedy
+  int* r;               // [B] scratch: accepted drafts per sequence
+  int* out;             // [B][gamma+1] emitted tokens (-1 past n_out)
+  int* n_out;           // [1] tokens emitted per sequence
+  int* n_ctx;           // device cache length, set to n0 + n_out
+  int n0;
+};
+void launch_spec_accept(const SpecArgs& a, cudaStream_t st);
+void launch_spec_transpose(const int* src, int* dst, int B, int G1,
+                           cudaStream_t st);
+
 // Device status word the tensor-core GEMM reports timeouts to.
 void set_tc_error_word(int* err);
 

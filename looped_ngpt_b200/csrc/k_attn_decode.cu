@@ -258,6 +258,20 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     cluster_arrive();                         // (1): nothing to publish
     pdl_wait();
     pdl_trigger();
+    if (lane != 0) {
+      // weights of the next projections into L2, once the predecessor's
+      // weight stream has ended
+      const void* pp[kMaxL2Ranges];
+      long pb[kMaxL2Ranges];
+#pragma unroll
+      for (int r = 0; r < kMaxL2Ranges; ++r) {
+        pp[r] = a.l2pf[r].p;
+        pb[r] = a.l2pf[r].bytes;
+      }
+      const int parts = C * dm.Hkv * a.B;
+      const int part = rank + C * (kvh + dm.Hkv * b);
+      l2_prefetch_share<kMaxL2Ranges>(pp, pb, part, parts, lane - 1, 31);
+    }
     if (lane == 0) {
       for (int i = kStages; i < ntile && !*fail; ++i) {
         // the consumers have released this stage's previous tile

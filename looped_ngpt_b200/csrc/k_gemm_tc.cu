@@ -58,6 +58,8 @@ struct TcArgs {
   int ldc;
   long slab;            // TC_PLAIN with K splits: elements between partials
   const float* col_scale;
+  const float* out_scale;   // scalar factor on every product (NVFP4 tensor
+                            // scale of dequantised weights), or null
   int* err;
   // TC_QKV: one tile column = one head of the fused q/k/v/gate projection
   int T;                // tokens per sequence (rows are b * T + t)
@@ -298,6 +300,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         for (int c0 = 0; c0 < TN; c0 += 32) {
           float v[32];
           tmem_ld32(trow + c0, v);
+          if (a.out_scale) {
+            const float os = *a.out_scale;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] *= os;
+          }
           const int col = n0 + c0;
           if (row < a.M && col < a.N) {
             float* dst = a.C + z * a.slab + (size_t)row * a.ldc + col;
@@ -322,6 +329,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           float gt[32], u[32];
           tmem_ld32(trow + c0, gt);
           tmem_ld32(trow + TN / 2 + c0, u);
+          if (a.out_scale) {
+            const float os = *a.out_scale;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              gt[k] *= os;
+              u[k] *= os;
+            }
+          }
           const int col = n0 + c0;
           // columns of this tile only (TN / 2 need not be a multiple of 32)
           const int lim = min(32, min(OUTC - c0, a.N - col));
@@ -347,6 +362,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           tmem_ld32(trow + c0, t32);
 #pragma unroll
           for (int k = 0; k < 32; ++k) v[c0 + k] = t32[k];
+        }
+        if (a.out_scale) {
+          const float os = *a.out_scale;
+#pragma unroll
+          for (int k = 0; k < TN; ++k) v[k] *= os;
         }
         if (row < a.M) qkv_epilogue<TN>(a, ni, row, v);
       }
@@ -514,7 +534,8 @@ void set_tc_error_word(int* err) { g_err_ptr = err; }
 // C + z * slab and the reader sums the partials.  Returns the split count.
 int launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
                      int M, int N, int K, const float* col_scale,
-                     cudaStream_t st, int max_splits, long slab) {
+                     cudaStream_t st, int max_splits, long slab,
+                     const float* out_scale) {
   CUtensorMap ma, mb;
   if (!make_map(&ma, A, M, K, lda, BM) || !weight_map(&mb, W, N, K, 128)) {
     note_host_failure("gemm: tensor map");
@@ -525,6 +546,7 @@ int launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
   a.ldc = ldc;
   a.slab = slab;
   a.col_scale = col_scale;
+  a.out_scale = out_scale;
   const int mt = (M + BM - 1) / BM, nt = (N + BN - 1) / BN;
   const int ks = gemm_split_count(M, N, K, col_scale ? 1 : max_splits);
   launch_tc<TC_PLAIN, BN>(ma, mb, a, mt, nt, st, ks);
@@ -547,13 +569,15 @@ int gemm_split_count(int M, int N, int K, int max_splits) {
 
 // m[M, F] = silu(A W_g^T) * (A W_u^T) (bf16) with W = [W_g; W_u] of 2F rows.
 void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
-                        int ldm, int M, int F, int K, cudaStream_t st) {
+                        int ldm, int M, int F, int K, cudaStream_t st,
+                        const float* out_scale) {
   CUtensorMap ma, mb;
   if (!make_map(&ma, A, M, K, lda, BM) || !weight_map(&mb, W, 2L * F, K, 128)) {
     note_host_failure("gemm: tensor map");
     return;
   }
   TcArgs a = base_args(M, F, K);
+  a.out_scale = out_scale;
   a.up_off = F;
   a.Cb = m;
   a.ldc = ldm;
@@ -575,7 +599,7 @@ void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
 
 // Fused q/k/v/gate projection with the RoPE / QK-norm / KV-write epilogue.
 void launch_gemm_qkv(const bf16* A, int lda, const bf16* W, const QkvGemmArgs& q,
-                     cudaStream_t st) {
+                     cudaStream_t st, const float* out_scale) {
   const int hd = q.dm.hd;
   const int rows = q.dm.rows_qkvg;
   CUtensorMap ma, mb;
@@ -585,6 +609,7 @@ void launch_gemm_qkv(const bf16* A, int lda, const bf16* W, const QkvGemmArgs& q
     return;
   }
   TcArgs a = base_args(q.M, rows, q.dm.d);
+  a.out_scale = out_scale;
   a.T = q.T;
   a.Hq = q.dm.Hq;
   a.Hkv = q.dm.Hkv;

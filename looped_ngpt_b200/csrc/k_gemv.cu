@@ -893,7 +893,46 @@ __global__ void dequant_rows_kernel(const uint8_t* Wq, const uint8_t* Ws, int K,
   }
 }
 
+// The same decode for a whole matrix, written as bf16 (the products have at
+// most 8 significant bits: exact); one thread per 8 consecutive weights,
+// 16-byte stores.
+template <int FMT>
+__global__ void dequant_bf16_kernel(const uint8_t* Wq, const uint8_t* Ws,
+                                    long N, int K, bf16* out) {
+  pdl_wait();
+  pdl_trigger();
+  const long total = N * (K / 8);
+  for (long id = blockIdx.x * (long)blockDim.x + threadIdx.x; id < total;
+       id += (long)gridDim.x * blockDim.x) {
+    const long row = id / (K / 8);
+    const int k = (int)(id - row * (K / 8)) * 8;
+    float w[8];
+    decode8<FMT>(Wq + (row * K + k) / 8 * FmtInfo<FMT>::LB, w);
+    const float sc = group_scale<FMT>(Ws, K, row, k);
+    uint4 u;
+    uint32_t* q = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 h =
+          __floats2bfloat162_rn(w[2 * e] * sc, w[2 * e + 1] * sc);
+      q[e] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(out + row * K + k) = u;
+  }
+}
+
 }  // namespace
+
+void launch_dequant_bf16(int fmt, const uint8_t* Wq, const uint8_t* Ws, long N,
+                         int K, bf16* out, cudaStream_t st) {
+  const dim3 grid(148 * 8), block(256);
+  if (fmt == WF_MXFP8)
+    launch_k(dequant_bf16_kernel<WF_MXFP8>, grid, block, 0, st, Wq, Ws, N, K,
+             out);
+  else
+    launch_k(dequant_bf16_kernel<WF_NVFP4>, grid, block, 0, st, Wq, Ws, N, K,
+             out);
+}
 
 int gemv_splits(const GemvArgs& a) { return make_plan(a, nb_of(a.B)).S; }
 

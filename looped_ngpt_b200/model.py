@@ -170,6 +170,29 @@ class DoryModel:
             ws.numel(), _stream_ptr(stream)))
         return logits, argmax
 
+    def spec_workspace(self, batch, gamma):
+        n = ctypes.c_int64()
+        check("dory_spec_workspace_bytes", _lib.load().dory_spec_workspace_bytes(
+            self.handle, batch, gamma, ctypes.byref(n)))
+        return torch.empty(n.value, dtype=torch.uint8, device=self.device)
+
+    def spec_decode_step(self, cache, last, gamma, k_draft, k_verify, ws,
+                         temperature=0.0, uniform=None, out=None, stream=None):
+        """dory_spec_decode_step: draft gamma tokens at k_draft loops, verify
+        at k_verify; returns (tokens int32 [B, gamma + 1], n emitted)."""
+        B = last.shape[0]
+        if out is None:
+            out = torch.empty((B, gamma + 1), dtype=torch.int32,
+                              device=self.device)
+        n = ctypes.c_int()
+        check("dory_spec_decode_step", _lib.load().dory_spec_decode_step(
+            self.handle, cache.handle, ctypes.c_void_p(last.data_ptr()), B,
+            gamma, k_draft, k_verify, float(temperature),
+            ctypes.c_void_p(uniform.data_ptr() if uniform is not None else 0),
+            ctypes.c_void_p(out.data_ptr()), ctypes.byref(n),
+            ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream_ptr(stream)))
+        return out, n.value
+
     def copy_state(self, ws, B, T, logits_all=False, stream=None):
         """dory_copy_state: final residual state of the last call."""
         rows = B * T if logits_all else B

@@ -5,7 +5,8 @@
   run with block scales chosen by minimum squared error (the same format,
   other bytes).
 * Quantised decode (prompt fed one token per call, k=2, last_loop) matches
-  the oracle run on the same quantised bytes within the BF16 tolerances."""
+  the oracle run on the same quantised bytes within the BF16 tolerances, and
+  so do quantised prefill and decode batches over 8 (tensor-core path)."""
 import numpy as np
 import pytest
 import torch
@@ -57,12 +58,30 @@ def test_quantised_decode_matches_oracle(qmodel):
     compare(np.array(zg), np.array(zr), f"{fmt} decode")
 
 
-def test_quantised_prefill_unsupported(qmodel):
-    import looped_ngpt_b200 as lb
+def test_quantised_prefill_and_batch_over_8(qmodel):
+    """Multi-token calls and batches over 8 run the tensor-core GEMM on the
+    projection dequantised to bf16 (exact) just before it, with the NVFP4
+    tensor scale applied to the products: a 20-token prompt per sequence
+    (every position compared) and two teacher-forced decode steps at B = 10,
+    k = 2, per_loop."""
     fmt, qw, gm = qmodel
-    cache = gm.new_cache(1, 16, 4, kv_mode="last_loop")
-    ws = gm.workspace(1, 4)
-    with pytest.raises(lb.DoryError) as e:
-        gm.prefill(cache, torch.zeros((1, 4), dtype=torch.int32, device="cuda:0"),
-                   1, ws)
-    assert e.value.code == -2
+    B, T, k = 10, 20, 2
+    prompt = make_prompt(TINY, B, T, seed=17)
+    ref = Model(TINY, qw, batch=B, kv_mode="per_loop")
+    zr = ref.forward(prompt, k, all_logits=True)
+    cache = gm.new_cache(B, 32, T, kv_mode="per_loop", max_loops=k)
+    ws = gm.workspace(B, T)
+    zg, _ = gm.prefill(cache, torch.from_numpy(prompt).cuda(), k, ws,
+                       logits_all=True)
+    zg = zg.cpu().numpy()
+    tok = np.argmax(zr[:, -1], -1)
+    dr, dg = [], []
+    for _ in range(2):
+        dr.append(ref.decode_step(tok, k))
+        g, _ = gm.decode_step(cache, torch.from_numpy(tok.astype(np.int32)).cuda(),
+                              k, ws)
+        dg.append(g.cpu().numpy().copy())
+        tok = np.argmax(dr[-1], -1)
+    assert gm.sync_status() == 0
+    compare(zg, zr, f"{fmt} prefill B={B} T={T}")
+    compare(np.array(dg), np.array(dr), f"{fmt} decode B={B}")

@@ -11,6 +11,8 @@ the full model is exercised at a fraction of its size.
   section: E4M3 values with an E8M0 scale per 32 weights; paper summary,
   前置知识: NVFP4 = E2M1 values with E4M3 block scales), at K = 2560 and
   K = 10240, for batch rows 1, 2, 4 and 8.
+* A 1100-token prefill at k = 2 through the tensor-core path (projections
+  dequantised to bf16 just before each GEMM), every position compared.
 * Batch-4 decode at k = 2, last_loop, after a seeded synthetic context of
   131000 cached tokens (the long-context quantised workload: RoPE angles at
   positions near 131072, base 1e7 on the full-attention block), sequences 0
@@ -132,3 +134,23 @@ def test_quantised_decode_at_131k_context(qmodel):
     zr = [ref.decode_step(toks[j][seqs], k) for j in range(steps)]
     compare(np.array(zg), np.array(zr), f"{fmt} B=4 ctx 131000")
     assert max(np.abs(np.linalg.norm(s, axis=-1) - 1).max() for s in sg) <= NORM_TOL
+
+
+def test_quantised_prefill_dory_widths(qmodel):
+    """A 1100-token prompt (across the 1024-token window) at k = 2, per_loop,
+    through the tensor-core path with dequantised projections: every
+    position against the oracle on the same quantised bytes."""
+    from synthetic import make_prompt
+    fmt, qw, gm = qmodel
+    T, k = 1100, 2
+    prompt = make_prompt(QSHAPE, 1, T, seed=23)
+    cache = gm.new_cache(1, T + 8, T, kv_mode="per_loop", max_loops=k)
+    ws = gm.workspace(1, T)
+    zg, _ = gm.prefill(cache, torch.from_numpy(prompt).cuda(), k, ws,
+                       logits_all=True)
+    zg = zg.cpu().numpy()
+    assert gm.sync_status() == 0
+    del cache, ws
+    torch.cuda.empty_cache()
+    zr = Model(QSHAPE, qw, kv_mode="per_loop").forward(prompt, k, True)
+    compare(zg, zr, f"{fmt} prefill T={T} Dory widths")
