@@ -163,6 +163,23 @@ int dory_cache_reset(dory_cache* c, void* stream);
 int dory_cache_fill_synthetic(dory_model* m, dory_cache* c, int n_ctx,
                               uint64_t seed, void* stream);
 
+/* Prefix caching (long-context serving: a shared prompt prefix is computed
+ * once and reused; the MXFP8 explainer page, deployment section, serves
+ * contexts up to 256K): make every sequence of `dst` hold the first
+ * n_tokens positions of sequence src_b of `src`, as if dst had prefilled
+ * them itself; dst's length becomes n_tokens (its older contents are
+ * dropped).  Full-attention layers copy every position; sliding-window
+ * layers the window's last W - 1 positions that later queries can see.
+ * Both caches must belong to the same model and kv_mode; a per_loop
+ * source's loop count carries over (dst max_loops must hold it).  Errors:
+ * DORY_ERR_ARG; DORY_ERR_CACHE (mode mismatch, n_tokens beyond the source's
+ * length or dst's max_ctx, or a source ring that has already overwritten
+ * positions the window still needs); DORY_ERR_CUDA.  Enqueued on
+ * `stream`: order it after the source's writes and before dst's next call. */
+int dory_cache_copy_prefix(dory_model* m, dory_cache* dst,
+                           const dory_cache* src, int src_b, int n_tokens,
+                           void* stream);
+
 /* Workspace bytes for calls of `batch` sequences x up to `max_chunk`
  * tokens.  The workspace holds activations only; its contents between
  * calls are meaningless except for dory_copy_state(). */
@@ -255,6 +272,28 @@ int dory_debug_spec_accept(const int32_t* d_draft, const int32_t* d_target,
                            int B, int gamma, int V, float temperature,
                            int32_t* d_tokens_out, int32_t* d_scratch,
                            void* stream);
+
+/* Mixed loop counts in one batch (elastic depth per request: the loop count
+ * is a per-request knob of a single checkpoint, paper summary, 研究动机 and
+ * 核心方法): sequence b runs d_row_loops[b] recurrent loops (device int32
+ * [B], each in 1..max_loops); the call runs max_loops loops, and in loop t
+ * every sequence with d_row_loops[b] < t keeps its state and writes no K/V,
+ * so each sequence computes exactly what a call with its own loop count
+ * would.  Otherwise as dory_prefill / dory_decode_step with n_loops =
+ * max_loops (a per_loop cache is bound to max_loops; each sequence must
+ * keep its own count on every call, which the library cannot check).  The
+ * decode step is replayed from a CUDA graph keyed by the pointers, the
+ * d_row_loops buffer included (its contents may change between steps). */
+int dory_prefill_mixed(dory_model* m, dory_cache* c, const int32_t* d_tokens,
+                       int B, int T, const int32_t* d_row_loops, int max_loops,
+                       int kv_mode, int logits_all, float* d_logits,
+                       int32_t* d_argmax, void* d_workspace, int64_t ws_bytes,
+                       void* stream);
+int dory_decode_step_mixed(dory_model* m, dory_cache* c,
+                           const int32_t* d_tokens, int B,
+                           const int32_t* d_row_loops, int max_loops,
+                           int kv_mode, float* d_logits, int32_t* d_argmax,
+                           void* d_workspace, int64_t ws_bytes, void* stream);
 
 /* Copy the final residual state s (input of the LM head, f32) of the last
  * call that used this workspace: [B, T, d] for a logits_all prefill, else

@@ -49,6 +49,7 @@ SIGNATURES = {
     "dory_cache_length": (c_int, [_P, POINTER(c_int)]),
     "dory_cache_reset": (c_int, [_P, _P]),
     "dory_cache_fill_synthetic": (c_int, [_P, _P, c_int, ctypes.c_uint64, _P]),
+    "dory_cache_copy_prefix": (c_int, [_P, _P, _P, c_int, c_int, _P]),
     "dory_workspace_bytes": (c_int, [_P, c_int, c_int, _I64P]),
     "dory_prefill": (c_int, [_P, _P, _P, c_int, c_int, c_int, c_int, c_int,
                              _P, _P, _P, c_int64, _P]),
@@ -56,6 +57,10 @@ SIGNATURES = {
                                  c_int64, _P]),
     "dory_decode_step_static": (c_int, [_P, _P, _P, c_int, c_int, c_int, _P,
                                         _P, _P]),
+    "dory_prefill_mixed": (c_int, [_P, _P, _P, c_int, c_int, _P, c_int, c_int,
+                                   c_int, _P, _P, _P, c_int64, _P]),
+    "dory_decode_step_mixed": (c_int, [_P, _P, _P, c_int, _P, c_int, c_int,
+                                       _P, _P, _P, c_int64, _P]),
     "dory_debug_gemm_bf16": (c_int, [_P, c_int, _P, _P, c_int, c_int, c_int,
                                      _P]),
     "dory_debug_gemm_bf16_split": (c_int, [_P, c_int, _P, _P, c_int, c_int,

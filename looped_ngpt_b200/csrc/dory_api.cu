@@ -60,8 +60,11 @@ struct BlockW {
   const float *s_q, *s_k, *alpha_a, *alpha_m;
 };
 
+// (B, loops/T/logits_all, tokens, logits, argmax, workspace, row loop
+// counts, cache): the cache comes last.
 typedef std::tuple<int, int, const void*, const void*, const void*,
-                   const void*, const void*> GraphKey;
+                   const void*, const void*, const void*> GraphKey;
+constexpr size_t kKeyCache = std::tuple_size<GraphKey>::value - 1;
 
 struct GraphEntry {
   int seen = 0;
@@ -506,7 +509,7 @@ void dory_cache_free(dory_cache* c) {
   }
   m->caches.erase(c);
   for (auto it = m->graphs.begin(); it != m->graphs.end();) {
-    if (std::get<6>(it->first) == (const void*)c) {
+    if (std::get<kKeyCache>(it->first) == (const void*)c) {
       if (it->second.exec) cudaGraphExecDestroy(it->second.exec);
       it = m->graphs.erase(it);
     } else {
@@ -629,6 +632,7 @@ struct CallCtx {
   float* logits;
   int* argmax;
   cudaStream_t st;
+  const int* row_loops;   // device [B] per-sequence loop counts, or null
 };
 
 int slot_index(const dory_cache* c, int i, int t) {
@@ -717,8 +721,10 @@ void enqueue_forward(const CallCtx& x) {
     for (int i = m->n_in; i < m->n_in + m->n_rec; ++i) order.push_back({i, t});
   for (int i = m->n_in + m->n_rec; i < m->nblk; ++i) order.push_back({i, 0});
 
+  int prev_t = 0;        // loop of the previous layer pass (0: not recurrent)
   for (size_t k = 0; k < order.size(); ++k) {
     const int i = order[k].first, t = order[k].second;
+    const int rj_loop = (i == m->n_in && t > 1) ? t : 0;
     const BlockW& bw = m->blk[i];
     int rj = RJ_NONE;
     if (i == m->n_in) rj = (t == 1) ? RJ_FIRST : RJ_NEXT;
@@ -737,6 +743,7 @@ void enqueue_forward(const CallCtx& x) {
       } else {
         g.pro = PRO_UPDATE; g.s_in = cur; g.h_in = w.h; g.h_S = prev_S;
         g.alpha = prev_alpha; g.s_out = other; g.reinject = rj; g.x_buf = w.x;
+        g.row_loops = x.row_loops; g.upd_loop = prev_t; g.rj_loop = rj_loop;
         std::swap(cur, other);
       }
       S_qkvg = gemv_run(m, g, x.st, "gemv_qkvg", &bw.m_qkvg);
@@ -744,7 +751,8 @@ void enqueue_forward(const CallCtx& x) {
       if (k > 0) {
         Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
         launch_update_rows(cur, w.h, prev_alpha, other, w.s_bf, w.x, rj, x.M,
-                           dm.d, x.st, prev_S);
+                           dm.d, x.st, prev_S, x.row_loops, x.T, prev_t,
+                           rj_loop);
         std::swap(cur, other);
       }
       const float* osc = nullptr;
@@ -762,6 +770,7 @@ void enqueue_forward(const CallCtx& x) {
         qg.rope = w.rope + (full ? (size_t)x.T * half * 2 : 0);
         qg.q_scale = q_scale; qg.kv = kv; qg.g = geo;
         qg.q_out = w.qb; qg.gate_out = w.gate;
+        qg.row_loops = x.row_loops; qg.loop_t = t;
         Prof p(m, x.st, "gemm_qkv",
                (double)x.M * dm.d * 2 + (double)dm.rows_qkvg * dm.d * 2 +
                    (double)x.M * (dm.qdim * 6.0 + dm.kvdim * 4.0),
@@ -776,6 +785,7 @@ void enqueue_forward(const CallCtx& x) {
       da.rope = w.rope + (full ? (size_t)half * 2 : 0);
       da.q_scale = q_scale; da.window = full ? 0 : dm.window;
       da.kv = kv; da.g = geo; da.a_out = w.a; da.err = m->d_status;
+      da.row_loops = x.row_loops; da.loop_t = t;
       const double nk = full ? x.n_ctx0 + 1.0
                              : std::min(x.n_ctx0 + 1.0, (double)dm.window);
       if (gemv && x.B * dm.Hkv * nk * dm.hd * 4.0 < kL2pfMaxKvBytes)
@@ -822,6 +832,7 @@ void enqueue_forward(const CallCtx& x) {
       g.epi = EPI_SWIGLU; g.pair_off = dm.F; g.S = 1; g.out_bf = w.mact;
       g.pro = PRO_UPDATE; g.s_in = cur; g.h_in = w.h; g.h_S = S_o;
       g.alpha = bw.alpha_a; g.s_out = other; g.reinject = RJ_NONE; g.x_buf = w.x;
+      g.row_loops = x.row_loops; g.upd_loop = t;
       std::swap(cur, other);
       gemv_run(m, g, x.st, "gemv_gateup", &bw.m_gu);
       GemvArgs g2{};
@@ -833,7 +844,7 @@ void enqueue_forward(const CallCtx& x) {
       {
         Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
         launch_update_rows(cur, w.h, bw.alpha_a, other, w.s_bf, w.x, RJ_NONE,
-                           x.M, dm.d, x.st, S_o);
+                           x.M, dm.d, x.st, S_o, x.row_loops, x.T, t, 0);
       }
       std::swap(cur, other);
       {
@@ -853,6 +864,7 @@ void enqueue_forward(const CallCtx& x) {
                         nullptr, x.st, "gemm_down", slabs, osc);
     }
     prev_alpha = bw.alpha_m;
+    prev_t = t;
   }
 
   // ---- final update and LM head ------------------------------------------
@@ -862,6 +874,7 @@ void enqueue_forward(const CallCtx& x) {
     g.epi = EPI_LMHEAD; g.pro = PRO_UPDATE; g.s_in = cur; g.h_in = w.h;
     g.h_S = prev_S; g.alpha = prev_alpha; g.s_out = w.sfin;
     g.reinject = RJ_NONE; g.x_buf = w.x;
+    g.row_loops = x.row_loops; g.upd_loop = prev_t;
     g.out = x.logits; g.out_stride = dm.V; g.col_scale = m->s_z;
     g.amax_val = w.amax_val; g.amax_idx = w.amax_idx;
     const int grid = gemv_grid(g, m->num_sms);
@@ -876,7 +889,7 @@ void enqueue_forward(const CallCtx& x) {
     {
       Prof p(m, x.st, "update_rows", (double)x.M * dm.d * 14, 0);
       launch_update_rows(cur, w.h, prev_alpha, w.sfin, w.s_bf, w.x, RJ_NONE,
-                         x.M, dm.d, x.st, prev_S);
+                         x.M, dm.d, x.st, prev_S, x.row_loops, x.T, prev_t, 0);
     }
     if (x.logits_all) {
       gemm_run(m, w.s_bf, dm.d, m->lm_head, x.logits, dm.V, x.M, dm.V, dm.d,
@@ -931,7 +944,7 @@ constexpr int kMaxGraphT = 16;
 int run_call(dory_model* m, dory_cache* c, const int32_t* tokens, int B,
              int T, int n_loops, int kv_mode, int logits_all, float* logits,
              int32_t* argmax, void* ws, int64_t ws_bytes, void* stream,
-             int flags) {
+             int flags, const int* row_loops = nullptr) {
   const bool graphs_ok = (flags & kCallGraph) && T <= kMaxGraphT;
   const bool spec = (flags & kCallSpec) != 0;
   if (!m || !c || c->m != m || !tokens || !ws) return DORY_ERR_ARG;
@@ -947,14 +960,14 @@ int run_call(dory_model* m, dory_cache* c, const int32_t* tokens, int B,
   const WS w = ws_layout(m, B, T, (char*)ws);
   if ((int64_t)w.total > ws_bytes) return DORY_ERR_WORKSPACE;
   CallCtx x{m, c, w, B, T, B * T, n_loops, logits_all, c->n_ctx, tokens,
-            logits, argmax, (cudaStream_t)stream};
+            logits, argmax, (cudaStream_t)stream, row_loops};
   cudaGetLastError();   // clear stale errors from earlier, unrelated calls
   take_host_failure();
 
   bool done = false;
   if (graphs_ok && m->use_graphs && !m->prof) {
     const GraphKey key(B, n_loops + 256 * T + (logits_all << 24), tokens,
-                       logits, argmax, ws, c);
+                       logits, argmax, ws, row_loops, c);
     if (m->graphs.size() > 64 && !m->graphs.count(key)) {
       for (auto& kv : m->graphs)
         if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
@@ -1162,6 +1175,28 @@ int dory_debug_spec_accept(const int32_t* d_draft, const int32_t* d_target,
   cudaGetLastError();
   launch_spec_accept(a, (cudaStream_t)stream);
   return cuda_rc(cudaGetLastError());
+}
+
+int dory_prefill_mixed(dory_model* m, dory_cache* c, const int32_t* d_tokens,
+                       int B, int T, const int32_t* d_row_loops, int max_loops,
+                       int kv_mode, int logits_all, float* d_logits,
+                       int32_t* d_argmax, void* d_workspace, int64_t ws_bytes,
+                       void* stream) {
+  if (!d_row_loops) return DORY_ERR_ARG;
+  return run_call(m, c, d_tokens, B, T, max_loops, kv_mode, logits_all ? 1 : 0,
+                  d_logits, d_argmax, d_workspace, ws_bytes, stream, 0,
+                  d_row_loops);
+}
+
+int dory_decode_step_mixed(dory_model* m, dory_cache* c,
+                           const int32_t* d_tokens, int B,
+                           const int32_t* d_row_loops, int max_loops,
+                           int kv_mode, float* d_logits, int32_t* d_argmax,
+                           void* d_workspace, int64_t ws_bytes, void* stream) {
+  if (!d_row_loops) return DORY_ERR_ARG;
+  return run_call(m, c, d_tokens, B, 1, max_loops, kv_mode, 0, d_logits,
+                  d_argmax, d_workspace, ws_bytes, stream, kCallGraph,
+                  d_row_loops);
 }
 
 int dory_copy_state(const dory_model* m, const void* d_workspace, int B,
@@ -1397,6 +1432,52 @@ extern "C" int dory_debug_gemv(const dory_model* m, const char* tensor,
   launch_gemv(g, gemv_grid(g, m->num_sms), (cudaStream_t)stream);
   if (cudaGetLastError() != cudaSuccess) return DORY_ERR_CUDA;
   *n_partials = g.S;
+  return DORY_OK;
+}
+
+extern "C" int dory_cache_copy_prefix(dory_model* m, dory_cache* dst,
+                                      const dory_cache* src, int src_b,
+                                      int n_tokens, void* stream) {
+  if (!m || !dst || !src || dst == src || dst->m != m || src->m != m ||
+      src_b < 0 || src_b >= src->B || n_tokens < 0)
+    return DORY_ERR_ARG;
+  if (dst->kv_mode != src->kv_mode || n_tokens > src->n_ctx ||
+      n_tokens > dst->max_ctx)
+    return DORY_ERR_CACHE;
+  // the loops the source's per_loop slots hold
+  int loops = 1;
+  if (src->kv_mode == DORY_KV_PER_LOOP) {
+    loops = src->loops_bound;
+    if (n_tokens > 0 && loops == 0) return DORY_ERR_CACHE;
+    if (loops > dst->max_loops) return DORY_ERR_CACHE;
+  }
+  const Dims& dm = m->dm;
+  // a later query at position n_tokens sees sliding-window keys from
+  // n_tokens - W + 1 on; the source ring must still hold them
+  const int sw_lo = std::max(0, n_tokens - dm.window + 1);
+  if (n_tokens > 0 && src->n_ctx - src->swa_cap > sw_lo) return DORY_ERR_CACHE;
+  const cudaStream_t st = (cudaStream_t)stream;
+  const CacheGeo gs{src->d_nctx, src->d_block_table, src->pages_per_seq,
+                    src->max_ctx};
+  const CacheGeo gd{dst->d_nctx, dst->d_block_table, dst->pages_per_seq,
+                    dst->max_ctx};
+  cudaGetLastError();
+  for (int i = 0; i < m->nblk; ++i) {
+    const bool per_loop = is_rec(m, i) && src->kv_mode == DORY_KV_PER_LOOP;
+    const int ns = per_loop ? loops : 1;
+    for (int t = 0; t < ns; ++t) {
+      const KVSlot& a = src->slots[src->slot_base[i] + t];
+      const KVSlot& b = dst->slots[dst->slot_base[i] + t];
+      const int lo = a.ring ? sw_lo : 0;
+      launch_copy_prefix(a, gs, src_b, b, gd, dst->B, dm.Hkv, dm.hd, lo,
+                         n_tokens, st);
+    }
+  }
+  launch_set_nctx(dst->d_nctx, n_tokens, st);
+  if (cudaGetLastError() != cudaSuccess) return DORY_ERR_CUDA;
+  dst->n_ctx = n_tokens;
+  dst->loops_bound = src->kv_mode == DORY_KV_PER_LOOP && n_tokens > 0
+                         ? loops : 0;
   return DORY_OK;
 }
 

@@ -141,6 +141,11 @@ struct GemvArgs {
   float* amax_val;     // EPI_LMHEAD: [B][gridDim]
   int* amax_idx;
   int* err;            // device status word (bounded-wait timeouts)
+  // rows with their own loop counts (null: every row runs every loop)
+  const int* row_loops; // [B] loops of each row
+  int upd_loop;        // loop of the sublayer whose update the prologue
+                       // applies (0: a non-recurrent block)
+  int rj_loop;         // loop whose re-injection it applies (RJ_NEXT)
 };
 // K segments per row the launcher will use (outputs are [S][B][n] partials
 // for EPI_F32; 1 for the other epilogues).
@@ -171,10 +176,33 @@ void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
                   bf16* s_bf, int* err, int vocab, float* rope,
                   const int* n_ctx, int hd, double theta_swa,
                   double theta_full, cudaStream_t st);
-// Prefill: s_new = N(s + alpha (N(h) - s)) per row (+ loop re-injection).
+// Rows that run their own loop counts: row b of a call takes part in loop t
+// of the recurrent blocks iff t <= row_loops[b]; in the loops it sits out,
+// its state is kept and it writes no K/V.  The effective re-injection of a
+// pending update for row b: -1 = keep the state (the update belongs to a
+// loop the row sits out), else RJ_NONE / RJ_FIRST / RJ_NEXT (RJ_NEXT drops
+// to RJ_NONE when the row does not run loop rj_loop).
+__device__ __forceinline__ int row_reinject(const int* row_loops, int b,
+                                            int upd_loop, int rj_loop,
+                                            int reinject) {
+  if (!row_loops) return reinject;
+  const int k = row_loops[b];
+  if (upd_loop > k) return -1;
+  if (reinject == RJ_NEXT && rj_loop > k) return RJ_NONE;
+  return reinject;
+}
+__device__ __forceinline__ bool row_writes_kv(const int* row_loops, int b,
+                                              int loop_t) {
+  return !row_loops || loop_t <= row_loops[b];
+}
+
+// Prefill: s_new = N(s + alpha (N(h) - s)) per row (+ loop re-injection);
+// rows b * T + t belong to sequence b (row_loops: see row_reinject).
 void launch_update_rows(const float* s_in, const float* h, const float* alpha,
                         float* s_out, bf16* s_bf, float* x_buf, int reinject,
-                        int M, int d, cudaStream_t st, int h_S = 1);
+                        int M, int d, cudaStream_t st, int h_S = 1,
+                        const int* row_loops = nullptr, int T = 1,
+                        int upd_loop = 0, int rj_loop = 0);
 // Final greedy argmax over [B][n] partials or full logits rows.
 void launch_argmax_partials(const float* val, const int* idx, int B, int n,
                             int* out, int* n_ctx, int T, cudaStream_t st);
@@ -188,6 +216,11 @@ void launch_fill_kv(const KVSlot& kv, const CacheGeo& g, int B, int Hkv,
                     uint64_t seed, float ck, float cv, cudaStream_t st);
 void launch_cache_init(int* n_ctx, int* block_table, int B, int pages_per_seq,
                        cudaStream_t st);
+// K/V entries of positions [p_lo, p_hi) of sequence src_b of one layer slot
+// -> the same positions of every sequence of a layer slot of another cache.
+void launch_copy_prefix(const KVSlot& src, const CacheGeo& gs, int src_b,
+                        const KVSlot& dst, const CacheGeo& gd, int B_dst,
+                        int Hkv, int hd, int p_lo, int p_hi, cudaStream_t st);
 
 // ----------------------------------------------------------- attention ----
 struct AttnArgs {
@@ -240,6 +273,8 @@ struct DecAttnArgs {
   // weights of the following projections, fetched into L2 while this
   // kernel (latency-bound at short context) leaves HBM idle
   L2Range l2pf[kMaxL2Ranges];
+  const int* row_loops; // rows with their own loop counts, or null
+  int loop_t;          // loop of this layer pass (0: non-recurrent)
 };
 // kv_maps: the TMA maps of this layer slot's K and V (make_kv_tile_map).
 void launch_attn_decode(const DecAttnArgs& a, const CUtensorMap* kv_maps,
@@ -282,6 +317,8 @@ struct QkvGemmArgs {
   KVSlot kv; CacheGeo g;
   bf16* q_out;         // [M][qdim]
   float* gate_out;     // [M][qdim]
+  const int* row_loops; // rows with their own loop counts, or null
+  int loop_t;          // loop of this layer pass (0: non-recurrent)
 };
 void launch_gemm_qkv(const bf16* A, int lda, const bf16* W,
                      const QkvGemmArgs& q, cudaStream_t st,

@@ -325,8 +325,9 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     }
     cons_sync();
 
-    // (b) the block holding position p stores the new entry
-    if (has_p) {
+    // (b) the block holding position p stores the new entry (not for a row
+    // that sits out this loop)
+    if (has_p && row_writes_kv(a.row_loops, b, a.loop_t)) {
       const size_t off = kv_index(a.kv, a.g, dm.Hkv, HD, b, kvh, p);
       for (int c = ct; c < HD; c += CT) {
         a.kv.K[off + c] = __float2bfloat16_rn(kn_s[c]);

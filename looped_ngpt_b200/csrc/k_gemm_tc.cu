@@ -70,6 +70,8 @@ struct TcArgs {
   KVSlot kv; CacheGeo g;
   bf16* q_out;          // [M][qdim] bf16, scaled by sqrt(hd) log2 e
   float* gate_out;      // [M][qdim] sigmoid(gate)
+  const int* row_loops; // rows with their own loop counts, or null
+  int loop_t;           // loop of this layer pass (0: non-recurrent)
 };
 
 // Epilogue of a TC_QKV tile: this thread holds one row of one head (hd
@@ -103,6 +105,8 @@ __device__ __forceinline__ void qkv_epilogue(const TcArgs& a, int item,
     atomicOr(a.err, ERRBIT_BOUNDS);
     return;
   }
+  // a row that sits out this loop writes no K/V
+  if (kind != 0 && !row_writes_kv(a.row_loops, b, a.loop_t)) return;
   if (kind != 2) {
     constexpr int H2 = HD / 2;
     const float* rt = a.rope + (size_t)t * H2 * 2;
@@ -623,6 +627,8 @@ void launch_gemm_qkv(const bf16* A, int lda, const bf16* W, const QkvGemmArgs& q
   a.g = q.g;
   a.q_out = q.q_out;
   a.gate_out = q.gate_out;
+  a.row_loops = q.row_loops;
+  a.loop_t = q.loop_t;
   const int mt = (q.M + BM - 1) / BM, nt = rows / hd;
   switch (hd) {
     case 64: launch_tc<TC_QKV, 64>(ma, mb, a, mt, nt, st); break;

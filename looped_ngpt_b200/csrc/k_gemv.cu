@@ -368,14 +368,26 @@ __device__ __forceinline__ UpdScal upd_scalars(const float (&r)[7], bool next) {
 // RJ_FIRST), re-injected value to the activation row in shared memory.
 template <int FMT>
 __device__ __forceinline__ void upd_store(const GemvArgs& a, const UpdScal& q,
-                                          size_t row, int i, float al, float sv,
-                                          float hv, float xv, void* xs) {
+                                          int rj, size_t row, int i, float al,
+                                          float sv, float hv, float xv,
+                                          void* xs) {
   const bool lead = blockIdx.x == 0;
   float v = ((1.f - al) * sv + al * hv * q.inv_h) * q.inv_t;
-  if (a.reinject == RJ_FIRST && lead && a.x_buf) a.x_buf[row + i] = v;
-  if (a.reinject == RJ_NEXT) v = (v + xv) * q.inv_u;
+  if (rj == RJ_FIRST && lead && a.x_buf) a.x_buf[row + i] = v;
+  if (rj == RJ_NEXT) v = (v + xv) * q.inv_u;
   if (lead) a.s_out[row + i] = v;
   put_x<FMT>(xs, (int)(row + i), v);
+}
+
+// A row sitting out this loop keeps its state (row_reinject < 0).
+template <int FMT>
+__device__ __forceinline__ void keep_row(const GemvArgs& a, int b, void* xs) {
+  const size_t row = (size_t)b * a.K;
+  for (int i = threadIdx.x; i < a.K; i += kThreads) {
+    const float v = a.s_in[row + i];
+    if (blockIdx.x == 0) a.s_out[row + i] = v;
+    put_x<FMT>(xs, (int)(row + i), v);
+  }
 }
 
 // PRO_UPDATE for batch row b: the previous sublayer's nGPT update
@@ -393,7 +405,12 @@ __device__ __forceinline__ void stage_x_update(const GemvArgs& a, int b,
                                                const float (&al)[kU], void* xs,
                                                float* red) {
   const int K = a.K, tid = threadIdx.x;
-  const bool next = a.reinject == RJ_NEXT;
+  const int rj = row_reinject(a.row_loops, b, a.upd_loop, a.rj_loop, a.reinject);
+  if (rj < 0) {
+    keep_row<FMT>(a, b, xs);
+    return;
+  }
+  const bool next = rj == RJ_NEXT;
   const size_t row = (size_t)b * K, hs = (size_t)a.B * K;
   float sv[kU], hv[kU], xv[kU];
 #pragma unroll
@@ -436,7 +453,7 @@ __device__ __forceinline__ void stage_x_update(const GemvArgs& a, int b,
 #pragma unroll
   for (int u = 0; u < kU; ++u) {
     const int i = tid + u * kThreads;
-    if (i < K) upd_store<FMT>(a, q, row, i, al[u], sv[u], hv[u], xv[u], xs);
+    if (i < K) upd_store<FMT>(a, q, rj, row, i, al[u], sv[u], hv[u], xv[u], xs);
   }
 }
 
@@ -446,7 +463,12 @@ template <int FMT>
 __device__ void stage_x_update_2pass(const GemvArgs& a, int b, void* xs,
                                      float* tmp, float* red) {
   const int K = a.K, tid = threadIdx.x;
-  const bool next = a.reinject == RJ_NEXT;
+  const int rj = row_reinject(a.row_loops, b, a.upd_loop, a.rj_loop, a.reinject);
+  if (rj < 0) {
+    keep_row<FMT>(a, b, xs);
+    return;
+  }
+  const bool next = rj == RJ_NEXT;
   const size_t row = (size_t)b * K, hs = (size_t)a.B * K;
   float r[7] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   for (int i = tid; i < K; i += kThreads) {
@@ -467,7 +489,7 @@ __device__ void stage_x_update_2pass(const GemvArgs& a, int b, void* xs,
   block_sum_n<7>(r, red);
   const UpdScal q = upd_scalars(r, next);
   for (int i = tid; i < K; i += kThreads)
-    upd_store<FMT>(a, q, row, i, a.alpha[i], a.s_in[row + i], tmp[i],
+    upd_store<FMT>(a, q, rj, row, i, a.alpha[i], a.s_in[row + i], tmp[i],
                    next ? a.x_buf[row + i] : 0.f, xs);
 }
 

@@ -81,14 +81,36 @@ __global__ void embed_kernel(const int* tokens, const bf16* E, int d,
 // sublayer output, gridDim.x rows apart.  Requires d % 256 == 0, d <= 8192.
 __global__ void update_rows_kernel(const float* s_in, const float* h,
                                    const float* alpha, float* s_out,
-                                   bf16* s_bf, float* x_buf, int reinject,
-                                   int d, int h_S) {
+                                   bf16* s_bf, float* x_buf, int reinject0,
+                                   int d, int h_S, const int* row_loops, int T,
+                                   int upd_loop, int rj_loop) {
   __shared__ float red[7 * 32];
   const size_t o = (size_t)blockIdx.x * d;
   const size_t hs = (size_t)gridDim.x * d;
   const int half = d / 2;
-  const bool next = reinject == RJ_NEXT;
   pdl_wait();
+  // rows with their own loop counts (uniform over the block: one row)
+  const int reinject = row_reinject(row_loops, blockIdx.x / T, upd_loop,
+                                    rj_loop, reinject0);
+  if (reinject < 0) {
+    pdl_trigger();
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int i = 4 * threadIdx.x + k * half;
+      const float4 vo = *reinterpret_cast<const float4*>(s_in + o + i);
+      if (s_out) *reinterpret_cast<float4*>(s_out + o + i) = vo;
+      if (s_bf) {
+        uint2 u;
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(vo.x, vo.y);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(vo.z, vo.w);
+        u.x = *reinterpret_cast<const uint32_t*>(&lo);
+        u.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(s_bf + o + i) = u;
+      }
+    }
+    return;
+  }
+  const bool next = reinject == RJ_NEXT;
   float4 sv[2], av[2], hv[2], xv[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
@@ -251,6 +273,30 @@ __global__ void fill_kv_kernel(KVSlot kv, CacheGeo g, int B, int Hkv, int hd,
   }
 }
 
+// Copy positions [p_lo, p_hi) of sequence src_b of one layer slot into every
+// sequence of the same layer slot of another cache (rings and pages are
+// addressed through each cache's own geometry); 16 bytes per thread.
+__global__ void copy_prefix_kernel(KVSlot src, CacheGeo gs, int src_b,
+                                   KVSlot dst, CacheGeo gd, int B_dst, int Hkv,
+                                   int hd, int p_lo, int p_hi) {
+  const int vec = hd / 8, np = p_hi - p_lo;
+  const long total = (long)B_dst * Hkv * np * vec;
+  for (long id = blockIdx.x * (long)blockDim.x + threadIdx.x; id < total;
+       id += (long)gridDim.x * blockDim.x) {
+    const int v = (int)(id % vec);
+    long r = id / vec;
+    const int pos = p_lo + (int)(r % np);
+    r /= np;
+    const int kvh = (int)(r % Hkv), b = (int)(r / Hkv);
+    const size_t so = kv_index(src, gs, Hkv, hd, src_b, kvh, pos) + v * 8;
+    const size_t dof = kv_index(dst, gd, Hkv, hd, b, kvh, pos) + v * 8;
+    *reinterpret_cast<uint4*>(dst.K + dof) =
+        *reinterpret_cast<const uint4*>(src.K + so);
+    *reinterpret_cast<uint4*>(dst.V + dof) =
+        *reinterpret_cast<const uint4*>(src.V + so);
+  }
+}
+
 __global__ void set_nctx_kernel(int* n_ctx, int v) { *n_ctx = v; }
 
 __global__ void advance_kernel(int* n_ctx, int T) {
@@ -285,9 +331,12 @@ void launch_embed(const int* tokens, const bf16* E, int M, int d, float* s,
 
 void launch_update_rows(const float* s_in, const float* h, const float* alpha,
                         float* s_out, bf16* s_bf, float* x_buf, int reinject,
-                        int M, int d, cudaStream_t st, int h_S) {
+                        int M, int d, cudaStream_t st, int h_S,
+                        const int* row_loops, int T, int upd_loop,
+                        int rj_loop) {
   launch_k(update_rows_kernel, dim3(M), dim3(d / 8), 0, st, s_in, h, alpha,
-           s_out, s_bf, x_buf, reinject, d, h_S);
+           s_out, s_bf, x_buf, reinject, d, h_S, row_loops, T < 1 ? 1 : T,
+           upd_loop, rj_loop);
 }
 
 void launch_argmax_partials(const float* val, const int* idx, int B, int n,
@@ -315,6 +364,14 @@ void launch_set_nctx(int* n_ctx, int v, cudaStream_t st) {
 
 void launch_advance(int* n_ctx, int T, cudaStream_t st) {
   launch_k(advance_kernel, dim3(1), dim3(1), 0, st, n_ctx, T);
+}
+
+void launch_copy_prefix(const KVSlot& src, const CacheGeo& gs, int src_b,
+                        const KVSlot& dst, const CacheGeo& gd, int B_dst,
+                        int Hkv, int hd, int p_lo, int p_hi, cudaStream_t st) {
+  if (p_hi <= p_lo) return;
+  copy_prefix_kernel<<<148 * 4, 256, 0, st>>>(src, gs, src_b, dst, gd, B_dst,
+                                               Hkv, hd, p_lo, p_hi);
 }
 
 void launch_cache_init(int* n_ctx, int* block_table, int B, int pages_per_seq,

@@ -65,6 +65,13 @@ class KVCache:
                   self.model.handle, self.handle, n_ctx, seed,
                   _stream_ptr(stream)))
 
+    def copy_prefix_from(self, src, src_b, n_tokens, stream=None):
+        """dory_cache_copy_prefix: every sequence of this cache takes the
+        first n_tokens positions of sequence src_b of `src`."""
+        check("dory_cache_copy_prefix", _lib.load().dory_cache_copy_prefix(
+            self.model.handle, self.handle, src.handle, src_b, n_tokens,
+            _stream_ptr(stream)))
+
     def reset(self, stream=None):
         check("dory_cache_reset",
               _lib.load().dory_cache_reset(self.handle, _stream_ptr(stream)))
@@ -169,6 +176,48 @@ class DoryModel:
             ctypes.c_void_p(argmax.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
             ws.numel(), _stream_ptr(stream)))
         return logits, argmax
+
+    def prefill_mixed(self, cache, tokens, row_loops, ws, logits_all=False,
+                      stream=None):
+        """dory_prefill_mixed: sequence b runs row_loops[b] loops (device
+        int32 [B]); returns (logits, argmax)."""
+        B, T = tokens.shape
+        V = self.shape.vocab
+        logits = torch.empty((B, T, V) if logits_all else (B, V),
+                             dtype=torch.float32, device=self.device)
+        argmax = torch.empty((B, T) if logits_all else (B,), dtype=torch.int32,
+                             device=self.device)
+        check("dory_prefill_mixed", _lib.load().dory_prefill_mixed(
+            self.handle, cache.handle, ctypes.c_void_p(tokens.data_ptr()), B, T,
+            ctypes.c_void_p(row_loops.data_ptr()), int(row_loops.max()),
+            KV_MODES[cache.kv_mode], 1 if logits_all else 0,
+            ctypes.c_void_p(logits.data_ptr()),
+            ctypes.c_void_p(argmax.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+            ws.numel(), _stream_ptr(stream)))
+        return logits, argmax
+
+    def decode_step_mixed(self, cache, tokens, row_loops, max_loops, ws,
+                          stream=None):
+        """dory_decode_step_mixed on device tokens int32 [B] and per-row loop
+        counts row_loops int32 [B]; returns (logits, argmax)."""
+        B = tokens.shape[0]
+        if getattr(cache, "_mix_bufs", None) is None:
+            cache._mix_bufs = (
+                torch.empty((B,), dtype=torch.int32, device=self.device),
+                torch.empty((B, self.shape.vocab), dtype=torch.float32,
+                            device=self.device),
+                torch.empty((B,), dtype=torch.int32, device=self.device),
+                torch.empty((B,), dtype=torch.int32, device=self.device))
+        tok_buf, lg_buf, am_buf, rl_buf = cache._mix_bufs
+        tok_buf.copy_(tokens.reshape(B), non_blocking=True)
+        rl_buf.copy_(row_loops.reshape(B), non_blocking=True)
+        check("dory_decode_step_mixed", _lib.load().dory_decode_step_mixed(
+            self.handle, cache.handle, ctypes.c_void_p(tok_buf.data_ptr()), B,
+            ctypes.c_void_p(rl_buf.data_ptr()), max_loops,
+            KV_MODES[cache.kv_mode], ctypes.c_void_p(lg_buf.data_ptr()),
+            ctypes.c_void_p(am_buf.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+            ws.numel(), _stream_ptr(stream)))
+        return lg_buf, am_buf
 
     def spec_workspace(self, batch, gamma):
         n = ctypes.c_int64()
