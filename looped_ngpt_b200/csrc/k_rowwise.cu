@@ -79,49 +79,38 @@ __global__ void embed_kernel(const int* tokens, const bf16* E, int d,
 // row is read once and written once (16-byte accesses), with one block
 // reduction of the norm terms in between.  h: h_S K-split partials of the
 // sublayer output, gridDim.x rows apart.  Requires d % 256 == 0, d <= 8192.
-__global__ void update_rows_kernel(const float* s_in, const float* h,
-                                   const float* alpha, float* s_out,
-                                   bf16* s_bf, float* x_buf, int reinject0,
-                                   int d, int h_S, const int* row_loops, int T,
-                                   int upd_loop, int rj_loop) {
+// One row per block of d / 8 threads (d <= 8192: at most 1024 threads,
+// which also caps the registers at 64 and keeps three 320-thread blocks per
+// SM for d = 2560).
+__global__ void __launch_bounds__(1024)
+update_rows_kernel(const float* s_in, const float* h, const float* alpha,
+                   float* s_out, bf16* s_bf, float* x_buf, int reinject0,
+                   int d, int h_S, const int* row_loops, int T, int upd_loop,
+                   int rj_loop) {
   __shared__ float red[7 * 32];
   const size_t o = (size_t)blockIdx.x * d;
   const size_t hs = (size_t)gridDim.x * d;
   const int half = d / 2;
   pdl_wait();
-  // rows with their own loop counts (uniform over the block: one row)
-  const int reinject = row_reinject(row_loops, blockIdx.x / T, upd_loop,
-                                    rj_loop, reinject0);
-  if (reinject < 0) {
-    pdl_trigger();
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int i = 4 * threadIdx.x + k * half;
-      const float4 vo = *reinterpret_cast<const float4*>(s_in + o + i);
-      if (s_out) *reinterpret_cast<float4*>(s_out + o + i) = vo;
-      if (s_bf) {
-        uint2 u;
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(vo.x, vo.y);
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(vo.z, vo.w);
-        u.x = *reinterpret_cast<const uint32_t*>(&lo);
-        u.y = *reinterpret_cast<const uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(s_bf + o + i) = u;
-      }
-    }
-    return;
-  }
+  // rows with their own loop counts (uniform over the block: one row); a
+  // row sitting out this loop keeps its state
+  const int rj = row_reinject(row_loops, blockIdx.x / T, upd_loop, rj_loop,
+                              reinject0);
+  const bool frozen = rj < 0;
+  const int reinject = frozen ? RJ_NONE : rj;
   const bool next = reinject == RJ_NEXT;
   float4 sv[2], av[2], hv[2], xv[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int i = 4 * threadIdx.x + k * half;
     sv[k] = *reinterpret_cast<const float4*>(s_in + o + i);
-    av[k] = *reinterpret_cast<const float4*>(alpha + i);
-    hv[k] = *reinterpret_cast<const float4*>(h + o + i);
+    av[k] = frozen ? make_float4(0.f, 0.f, 0.f, 0.f)
+                   : *reinterpret_cast<const float4*>(alpha + i);
+    hv[k] = frozen ? sv[k] : *reinterpret_cast<const float4*>(h + o + i);
     xv[k] = next ? *reinterpret_cast<const float4*>(x_buf + o + i)
                  : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  for (int p = 1; p < h_S; ++p)
+  for (int p = 1; p < (frozen ? 1 : h_S); ++p)
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const float4 t = *reinterpret_cast<const float4*>(h + p * hs + o + 4 * threadIdx.x +
