@@ -126,6 +126,7 @@ struct Plan {
   int sh;       // log2(S)
   int NS;       // stages in the ring (8 items each)
   int tmp;      // PRO_UPDATE needs the two-pass prologue (K > kU * kThreads)
+  int bps;      // blocks per SM (the grid is up to bps x the SM count)
 };
 
 // ---- quantised weights (MXFP8 / NVFP4): decode 8 weights of one lane ----
@@ -569,8 +570,17 @@ __device__ __forceinline__ float row_dot_mma(const uint8_t* w,
 }
 
 // ---- the kernel -----------------------------------------------------------
+// Blocks per SM the kernel is compiled for: two for quantised weights, whose
+// SIMT decode loop is bound by the latency of its dependent chains (twice
+// the warps hide it: MXFP8 batch-1 decode 267 -> 328 tok/s, NVFP4
+// 285 -> 355, k = 2); one for BF16, whose batch-1 rows run on the warp MMA
+// and whose batched SIMT rows measured slower with two blocks (batch 4 at a
+// 131K context 461 -> 436 tok/s).
+template <int NB, int FMT>
+constexpr int kBlocksPerSm = FMT != WF_BF16 ? 2 : 1;
+
 template <int NB, int EPI, int FMT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, (kBlocksPerSm<NB, FMT>))
 gemv_kernel(const GemvArgs a, const Plan pl) {
   constexpr int R = (EPI == EPI_SWIGLU) ? 2 : 1;
   constexpr int LB = FmtInfo<FMT>::LB;       // bytes per 8 weights
@@ -829,15 +839,27 @@ int lane_bytes(int fmt) { return fmt == WF_BF16 ? 16 : fmt == WF_MXFP8 ? 8 : 4; 
 // Segments per row S (F32 only: SwiGLU and LM head need whole rows) and
 // ring depth: the largest segment <= kSeg whose 8-item stages still fit at
 // least 3 deep (2 as a last resort).
+// Blocks per SM wanted for these arguments (kBlocksPerSm of the variant the
+// launcher picks; DORY_GEMV_BPS = 1 or 2 overrides it for measurements).
+int bps_wanted(const GemvArgs& a, int nb) {
+  (void)nb;
+  const char* e = getenv("DORY_GEMV_BPS");
+  if (e && atoi(e) < 2) return 1;
+  return a.fmt != WF_BF16 ? 2 : 1;
+}
+
 Plan make_plan(const GemvArgs& a, int nb) {
   const int R = a.epi == EPI_SWIGLU ? 2 : 1;
   const size_t fixed = fixed_smem(a, nb);
   const int lb = lane_bytes(a.fmt);
+  int bps = bps_wanted(a, nb);
+  // two blocks share the SM's shared memory (and its 1 KB per block)
+  size_t budget = bps == 2 ? kSmemBudget / 2 - 2048 : kSmemBudget;
   int S = 1;
   if (a.epi == EPI_F32) {
     while (a.K / S > kSeg && (a.K / (2 * S)) % 256 == 0) S *= 2;
     while ((a.K / (2 * S)) % 256 == 0 &&
-           fixed + 3 * (size_t)kWarps * R * (a.K / S) / 8 * lb > kSmemBudget)
+           fixed + 3 * (size_t)kWarps * R * (a.K / S) / 8 * lb > budget)
       S *= 2;
   }
   const int sbytes = a.fmt == WF_BF16 ? 0
@@ -846,10 +868,14 @@ Plan make_plan(const GemvArgs& a, int nb) {
                                              (sbytes % 16 == 0 ? sbytes : 0));
   int NS = stages_default();
   if (a.fmt != WF_BF16) NS = kMaxStages;          // smaller items: go deeper
-  while (NS > 2 && fixed + NS * stage > kSmemBudget) --NS;
+  if (bps == 2 && fixed + 2 * stage > budget) {   // two rings do not fit
+    bps = 1;
+    budget = kSmemBudget;
+  }
+  while (NS > 2 && fixed + NS * stage > budget) --NS;
   int sh = 0;
   while ((1 << sh) < S) ++sh;
-  return Plan{S, sh, NS, needs_tmp(a) ? 1 : 0};
+  return Plan{S, sh, NS, needs_tmp(a) ? 1 : 0, bps};
 }
 
 size_t smem_bytes(const GemvArgs& a, const Plan& p, int nb) {
@@ -959,7 +985,8 @@ void launch_dequant_bf16(int fmt, const uint8_t* Wq, const uint8_t* Ws, long N,
 int gemv_splits(const GemvArgs& a) { return make_plan(a, nb_of(a.B)).S; }
 
 int gemv_grid(const GemvArgs& a, int num_sms) {
-  return a.n_items < num_sms ? a.n_items : num_sms;
+  const int n = num_sms * make_plan(a, nb_of(a.B)).bps;
+  return a.n_items < n ? a.n_items : n;
 }
 
 void launch_dequant_rows(int fmt, const uint8_t* Wq, const uint8_t* Ws, int K,
