@@ -25,11 +25,12 @@
 //                   stages are issued before the dependency wait (positions
 //                   < p were written by finished calls; row p is replaced in
 //                   shared memory);
-//   warps 1-2       (a) vector v of (q_0 .. q_{G-1}, k, v) is formed once in
-//                   the cluster, by warp v % 2 of block v / 2, from the QKVG
-//                   partials (rotate-half RoPE, per-head L2 norm, scales; k
-//                   and v rounded to BF16); after a cluster barrier every
-//                   block copies the vectors from their owners;
+//   warps 1-2       (a) every block forms the vectors it reads from the
+//                   QKVG partials (rotate-half RoPE, per-head L2 norm,
+//                   scales; k and v rounded to BF16): q_0 .. q_{G-1}, and in
+//                   the block holding position p also k and v (forming them
+//                   locally, all loads in one L2 round trip, is quicker than
+//                   a cluster barrier and a copy from owner blocks);
 //                   (b) the block holding position p stores k, v in the cache;
 //                   (c) per stage warp c takes keys 16c..16c+15: S^T = K Q^T
 //                   on m16n8k16 (K rows as A, the heads as the 8 columns),
@@ -109,77 +110,100 @@ __device__ __forceinline__ float4 ld_peer4(uint32_t addr) {
   return v;
 }
 
-// One warp forms vector v of (q_0 .. q_{G-1}, k, v) of KV head kvh from the
-// split-K partials of the fused QKVG output: q and k get rotate-half RoPE
-// (rope: [hd/2] cos, sin of this position), the L2 norm over the head and the
-// per-dim scale (q also q_scale); k and v are rounded to BF16, the precision
-// the cache holds.  All loads are issued before the first use.
-template <int HD, int G>
-__device__ __forceinline__ void form_vector(const DecAttnArgs& a,
-                                            const float* src, size_t pstride,
-                                            int kvh, int v, float* dst) {
+// One warp forms up to NW vectors v of (q_0 .. q_{G-1}, k, v) of KV head kvh
+// (vs[j] < 0: none) from the split-K partials of the fused QKVG output: q and
+// k get rotate-half RoPE (rope: [hd/2] cos, sin of this position), the L2
+// norm over the head and the per-dim scale (q also q_scale); k and v are
+// rounded to BF16, the precision the cache holds.  Every load of every
+// vector is issued before the first use (one L2 round trip).
+template <int HD, int G, int NW>
+__device__ __forceinline__ void form_vectors(const DecAttnArgs& a,
+                                             const float* src, size_t pstride,
+                                             int kvh, const int (&vs)[NW],
+                                             float* vec_s) {
   constexpr int HALF = HD / 2;
   constexpr int NPR = (HALF + 31) / 32;       // rotation pairs per lane
   const Dims& dm = a.dm;
   const int lane = threadIdx.x & 31;
-  const bool is_q = v < G, is_v = v == G + 1;
-  const int col0 = is_q ? (kvh * G + v) * HD
-                 : !is_v ? dm.qdim + kvh * HD : dm.qdim + dm.kvdim + kvh * HD;
-  const float* scale = is_q ? a.s_q + (kvh * G + v) * HD : a.s_k + kvh * HD;
-  float x1[NPR], x2[NPR], cs[NPR], sn[NPR], sc1[NPR], sc2[NPR];
+  float x1[NW][NPR], x2[NW][NPR], cs[NPR], sn[NPR], sc1[NW][NPR], sc2[NW][NPR];
 #pragma unroll
   for (int j = 0; j < NPR; ++j) {
     const int i = lane + 32 * j;
-    const bool in = i < HALF;
-    x1[j] = x2[j] = 0.f;
-    cs[j] = in && !is_v ? a.rope[2 * i] : 0.f;
-    sn[j] = in && !is_v ? a.rope[2 * i + 1] : 0.f;
-    sc1[j] = in && !is_v ? scale[i] : 0.f;
-    sc2[j] = in && !is_v ? scale[i + HALF] : 0.f;
+    cs[j] = i < HALF ? a.rope[2 * i] : 0.f;
+    sn[j] = i < HALF ? a.rope[2 * i + 1] : 0.f;
+  }
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const int v = vs[w];
+    const bool is_q = v < G, is_v = v == G + 1;
+    const float* scale = is_q ? a.s_q + (kvh * G + v) * HD : a.s_k + kvh * HD;
+#pragma unroll
+    for (int j = 0; j < NPR; ++j) {
+      const int i = lane + 32 * j;
+      const bool in = v >= 0 && i < HALF && !is_v;
+      x1[w][j] = x2[w][j] = 0.f;
+      sc1[w][j] = in ? scale[i] : 0.f;
+      sc2[w][j] = in ? scale[i + HALF] : 0.f;
+    }
   }
   for (int s = 0; s < a.S; ++s) {
-    const float* sp = src + s * pstride + col0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const int v = vs[w];
+      if (v < 0) continue;
+      const bool is_q = v < G, is_v = v == G + 1;
+      const int col0 = is_q ? (kvh * G + v) * HD
+                     : !is_v ? dm.qdim + kvh * HD : dm.qdim + dm.kvdim + kvh * HD;
+      const float* sp = src + s * pstride + col0;
+#pragma unroll
+      for (int j = 0; j < NPR; ++j) {
+        const int i = lane + 32 * j;
+        if (i < HALF) {
+          x1[w][j] += sp[i];
+          x2[w][j] += sp[i + HALF];
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const int v = vs[w];
+    if (v < 0) continue;
+    const bool is_q = v < G, is_v = v == G + 1;
+    float* dst = vec_s + v * HD;
+    if (is_v) {
+#pragma unroll
+      for (int j = 0; j < NPR; ++j) {
+        const int i = lane + 32 * j;
+        if (i < HALF) {
+          dst[i] = __bfloat162float(__float2bfloat16_rn(x1[w][j]));
+          dst[i + HALF] = __bfloat162float(__float2bfloat16_rn(x2[w][j]));
+        }
+      }
+      continue;
+    }
+    float r1[NPR], r2[NPR], ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < NPR; ++j) {
+      r1[j] = x1[w][j] * cs[j] - x2[w][j] * sn[j];
+      r2[j] = x2[w][j] * cs[j] + x1[w][j] * sn[j];
+      ss += r1[j] * r1[j] + r2[j] * r2[j];
+    }
+    const float inv = 1.f / fmaxf(sqrtf(warp_sum(ss)), 1e-12f);
+    const float extra = is_q ? a.q_scale : 1.f;
 #pragma unroll
     for (int j = 0; j < NPR; ++j) {
       const int i = lane + 32 * j;
       if (i < HALF) {
-        x1[j] += sp[i];
-        x2[j] += sp[i + HALF];
+        float u = r1[j] * inv * sc1[w][j] * extra;
+        float z = r2[j] * inv * sc2[w][j] * extra;
+        if (!is_q) {
+          u = __bfloat162float(__float2bfloat16_rn(u));
+          z = __bfloat162float(__float2bfloat16_rn(z));
+        }
+        dst[i] = u;
+        dst[i + HALF] = z;
       }
-    }
-  }
-  if (is_v) {
-#pragma unroll
-    for (int j = 0; j < NPR; ++j) {
-      const int i = lane + 32 * j;
-      if (i < HALF) {
-        dst[i] = __bfloat162float(__float2bfloat16_rn(x1[j]));
-        dst[i + HALF] = __bfloat162float(__float2bfloat16_rn(x2[j]));
-      }
-    }
-    return;
-  }
-  float r1[NPR], r2[NPR], ss = 0.f;
-#pragma unroll
-  for (int j = 0; j < NPR; ++j) {
-    r1[j] = x1[j] * cs[j] - x2[j] * sn[j];
-    r2[j] = x2[j] * cs[j] + x1[j] * sn[j];
-    ss += r1[j] * r1[j] + r2[j] * r2[j];
-  }
-  const float inv = 1.f / fmaxf(sqrtf(warp_sum(ss)), 1e-12f);
-  const float extra = is_q ? a.q_scale : 1.f;
-#pragma unroll
-  for (int j = 0; j < NPR; ++j) {
-    const int i = lane + 32 * j;
-    if (i < HALF) {
-      float u = r1[j] * inv * sc1[j] * extra;
-      float w = r2[j] * inv * sc2[j] * extra;
-      if (!is_q) {
-        u = __bfloat162float(__float2bfloat16_rn(u));
-        w = __bfloat162float(__float2bfloat16_rn(w));
-      }
-      dst[i] = u;
-      dst[i + HALF] = w;
     }
   }
 }
@@ -255,7 +279,6 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
     if (lane == 0)
       for (int i = 0; i < min(kStages, ntile); ++i) issue(i);
     __syncwarp();
-    cluster_arrive();                         // (1): nothing to publish
     pdl_wait();
     pdl_trigger();
     if (lane != 0) {
@@ -283,7 +306,6 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
       }
     }
     __syncwarp();
-    cluster_wait();                           // (1)
     cluster_arrive();                         // (2)
     cluster_wait();
     cluster_arrive();                         // (3)
@@ -309,19 +331,18 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
           gate[k] += src[s3 * pstride + dm.qdim + 2 * dm.kvdim + kvh * G * HD + idx];
     }
 
-    // (a) this warp's vector, if it owns one; then every block copies all
-    const int v_own = rank * kCons + cw;
-    if (v_own < NV) form_vector<HD, G>(a, src, pstride, kvh, v_own, vec_s + v_own * HD);
-    cluster_arrive();                         // (1): vectors published
-    cluster_wait();
+    // (a) every block forms the vectors it reads itself: the G query heads,
+    // and where p's tile is, the new k and v (warp cw takes vectors cw,
+    // cw + 2, ...); no cluster exchange is needed before the tiles
     {
-      constexpr int V4 = NV * HD / 4;
-      for (int e = ct; e < V4; e += CT) {
-        const int owner = ((4 * e) / HD) / kCons;
-        if (owner != rank)
-          *reinterpret_cast<float4*>(vec_s + 4 * e) =
-              ld_peer4(peer_addr(vec_s + 4 * e, owner));
+      constexpr int NW = (NV + kCons - 1) / kCons;
+      int vs[NW];
+#pragma unroll
+      for (int j = 0; j < NW; ++j) {
+        const int v = cw + kCons * j;
+        vs[j] = (v < G || (v < NV && has_p)) ? v : -1;
       }
+      form_vectors<HD, G, NW>(a, src, pstride, kvh, vs, vec_s);
     }
     cons_sync();
 
