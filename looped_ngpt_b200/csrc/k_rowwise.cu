@@ -79,14 +79,14 @@ __global__ void embed_kernel(const int* tokens, const bf16* E, int d,
 // row is read once and written once (16-byte accesses), with one block
 // reduction of the norm terms in between.  h: h_S K-split partials of the
 // sublayer output, gridDim.x rows apart.  Requires d % 256 == 0, d <= 8192.
-// One row per block of d / 8 threads (d <= 8192: at most 1024 threads,
-// which also caps the registers at 64 and keeps three 320-thread blocks per
-// SM for d = 2560).
-__global__ void __launch_bounds__(1024)
-update_rows_kernel(const float* s_in, const float* h, const float* alpha,
-                   float* s_out, bf16* s_bf, float* x_buf, int reinject0,
-                   int d, int h_S, const int* row_loops, int T, int upd_loop,
-                   int rj_loop) {
+// MIXED: rows carry their own loop counts (row_loops non-null); the plain
+// variant has no per-row test at all.
+template <bool MIXED>
+__global__ void update_rows_kernel(const float* s_in, const float* h,
+                                   const float* alpha, float* s_out,
+                                   bf16* s_bf, float* x_buf, int reinject0,
+                                   int d, int h_S, const int* row_loops, int T,
+                                   int upd_loop, int rj_loop) {
   __shared__ float red[7 * 32];
   const size_t o = (size_t)blockIdx.x * d;
   const size_t hs = (size_t)gridDim.x * d;
@@ -94,9 +94,10 @@ update_rows_kernel(const float* s_in, const float* h, const float* alpha,
   pdl_wait();
   // rows with their own loop counts (uniform over the block: one row); a
   // row sitting out this loop keeps its state
-  const int rj = row_reinject(row_loops, blockIdx.x / T, upd_loop, rj_loop,
-                              reinject0);
-  const bool frozen = rj < 0;
+  const int rj = MIXED ? row_reinject(row_loops, blockIdx.x / T, upd_loop,
+                                      rj_loop, reinject0)
+                       : reinject0;
+  const bool frozen = MIXED && rj < 0;
   const int reinject = frozen ? RJ_NONE : rj;
   const bool next = reinject == RJ_NEXT;
   float4 sv[2], av[2], hv[2], xv[2];
@@ -323,9 +324,14 @@ void launch_update_rows(const float* s_in, const float* h, const float* alpha,
                         int M, int d, cudaStream_t st, int h_S,
                         const int* row_loops, int T, int upd_loop,
                         int rj_loop) {
-  launch_k(update_rows_kernel, dim3(M), dim3(d / 8), 0, st, s_in, h, alpha,
-           s_out, s_bf, x_buf, reinject, d, h_S, row_loops, T < 1 ? 1 : T,
-           upd_loop, rj_loop);
+  if (row_loops)
+    launch_k(update_rows_kernel<true>, dim3(M), dim3(d / 8), 0, st, s_in, h,
+             alpha, s_out, s_bf, x_buf, reinject, d, h_S, row_loops,
+             T < 1 ? 1 : T, upd_loop, rj_loop);
+  else
+    launch_k(update_rows_kernel<false>, dim3(M), dim3(d / 8), 0, st, s_in, h,
+             alpha, s_out, s_bf, x_buf, reinject, d, h_S, row_loops,
+             T < 1 ? 1 : T, upd_loop, rj_loop);
 }
 
 void launch_argmax_partials(const float* val, const int* idx, int B, int n,
