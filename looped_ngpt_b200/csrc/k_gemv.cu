@@ -322,12 +322,13 @@ __device__ __forceinline__ uint4 bf8_to_h8(uint4 v) {
 // PRO_BF16: copy the caller's bf16 rows (zero rows past B), all loads of a
 // thread in flight together.
 template <int FMT, int NB>
-__device__ __forceinline__ void stage_x_copy(const GemvArgs& a, void* xs) {
+__device__ __forceinline__ void stage_x_copy(const GemvArgs& a, int XS,
+                                             void* xs) {
   const int vec = a.K / 8, tid = threadIdx.x;
 #pragma unroll 1
   for (int b = 0; b < NB; ++b) {
     uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(xs) +
-                                          (size_t)b * a.K);
+                                          (size_t)b * XS);
     const uint4* src = reinterpret_cast<const uint4*>(
         a.xin + (size_t)(b < a.B ? b : 0) * a.xin_stride);
 #pragma unroll 1
@@ -369,25 +370,26 @@ __device__ __forceinline__ UpdScal upd_scalars(const float (&r)[7], bool next) {
 // RJ_FIRST), re-injected value to the activation row in shared memory.
 template <int FMT>
 __device__ __forceinline__ void upd_store(const GemvArgs& a, const UpdScal& q,
-                                          int rj, size_t row, int i, float al,
-                                          float sv, float hv, float xv,
-                                          void* xs) {
+                                          int rj, size_t row, size_t xrow,
+                                          int i, float al, float sv, float hv,
+                                          float xv, void* xs) {
   const bool lead = blockIdx.x == 0;
   float v = ((1.f - al) * sv + al * hv * q.inv_h) * q.inv_t;
   if (rj == RJ_FIRST && lead && a.x_buf) a.x_buf[row + i] = v;
   if (rj == RJ_NEXT) v = (v + xv) * q.inv_u;
   if (lead) a.s_out[row + i] = v;
-  put_x<FMT>(xs, (int)(row + i), v);
+  put_x<FMT>(xs, (int)(xrow + i), v);
 }
 
 // A row sitting out this loop keeps its state (row_reinject < 0).
 template <int FMT>
-__device__ __forceinline__ void keep_row(const GemvArgs& a, int b, void* xs) {
+__device__ __forceinline__ void keep_row(const GemvArgs& a, int b, int XS,
+                                         void* xs) {
   const size_t row = (size_t)b * a.K;
   for (int i = threadIdx.x; i < a.K; i += kThreads) {
     const float v = a.s_in[row + i];
     if (blockIdx.x == 0) a.s_out[row + i] = v;
-    put_x<FMT>(xs, (int)(row + i), v);
+    put_x<FMT>(xs, (int)((size_t)b * XS + i), v);
   }
 }
 
@@ -402,13 +404,13 @@ __device__ __forceinline__ void keep_row(const GemvArgs& a, int b, void* xs) {
 // the whole update costs one round trip to L2.  `al` holds this thread's
 // alpha values (loaded before the programmatic-dependent-launch wait).
 template <int FMT>
-__device__ __forceinline__ void stage_x_update(const GemvArgs& a, int b,
+__device__ __forceinline__ void stage_x_update(const GemvArgs& a, int b, int XS,
                                                const float (&al)[kU], void* xs,
                                                float* red) {
   const int K = a.K, tid = threadIdx.x;
   const int rj = row_reinject(a.row_loops, b, a.upd_loop, a.rj_loop, a.reinject);
   if (rj < 0) {
-    keep_row<FMT>(a, b, xs);
+    keep_row<FMT>(a, b, XS, xs);
     return;
   }
   const bool next = rj == RJ_NEXT;
@@ -454,19 +456,21 @@ __device__ __forceinline__ void stage_x_update(const GemvArgs& a, int b,
 #pragma unroll
   for (int u = 0; u < kU; ++u) {
     const int i = tid + u * kThreads;
-    if (i < K) upd_store<FMT>(a, q, rj, row, i, al[u], sv[u], hv[u], xv[u], xs);
+    if (i < K)
+      upd_store<FMT>(a, q, rj, row, (size_t)b * XS, i, al[u], sv[u], hv[u],
+                     xv[u], xs);
   }
 }
 
 // PRO_UPDATE for K > kU * kThreads: the same update in two passes, the
 // summed h kept in shared memory (tmp [K]) in between.
 template <int FMT>
-__device__ void stage_x_update_2pass(const GemvArgs& a, int b, void* xs,
+__device__ void stage_x_update_2pass(const GemvArgs& a, int b, int XS, void* xs,
                                      float* tmp, float* red) {
   const int K = a.K, tid = threadIdx.x;
   const int rj = row_reinject(a.row_loops, b, a.upd_loop, a.rj_loop, a.reinject);
   if (rj < 0) {
-    keep_row<FMT>(a, b, xs);
+    keep_row<FMT>(a, b, XS, xs);
     return;
   }
   const bool next = rj == RJ_NEXT;
@@ -490,8 +494,8 @@ __device__ void stage_x_update_2pass(const GemvArgs& a, int b, void* xs,
   block_sum_n<7>(r, red);
   const UpdScal q = upd_scalars(r, next);
   for (int i = tid; i < K; i += kThreads)
-    upd_store<FMT>(a, q, rj, row, i, a.alpha[i], a.s_in[row + i], tmp[i],
-                   next ? a.x_buf[row + i] : 0.f, xs);
+    upd_store<FMT>(a, q, rj, row, (size_t)b * XS, i, a.alpha[i],
+                   a.s_in[row + i], tmp[i], next ? a.x_buf[row + i] : 0.f, xs);
 }
 
 // ---- batch-1 BF16 rows on the tensor cores ---------------------------------
@@ -569,6 +573,41 @@ __device__ __forceinline__ float row_dot_mma(const uint8_t* w,
   return warp_sum(v);
 }
 
+// ---- several BF16 activation rows on the tensor cores -----------------------
+// Whole-row items (no K split) of BF16 weights with 2..8 activation rows:
+// m16n8k16 with the activation rows as the M rows (NB of 16 used) and the 8
+// weight rows of a stage as the N = 8 columns, so every product but those of
+// the unused M rows counts.  Warp w takes the w-th eighth of K of all 8 rows
+// (its activation fragments stay in registers for the whole launch), and the
+// eight warps' partial sums meet in shared memory once per stage.
+template <int NB, int EPI, int FMT>
+constexpr bool kMmaB = FMT == WF_BF16 && NB >= 2 && EPI != EPI_LMHEAD;
+
+// Row stride (elements) of the activation rows in shared memory: padded by
+// 16 bytes where the batched MMA path reads them, so that the 8 rows of a
+// fragment load fall in different banks.
+__host__ __device__ constexpr int x_stride_of(int fmt, int nb, int K) {
+  return (fmt == WF_BF16 && nb >= 2) ? K + 8 : K;
+}
+template <int NB, int FMT>
+__device__ __forceinline__ int x_stride(int K) { return x_stride_of(FMT, NB, K); }
+
+// Partial-sum buffer of the batched MMA path: two stages x kWarps x R x 64.
+constexpr int kRedFloats = 2 * kWarps * 2 * 64;
+
+// Barrier of the consumer warps (named barrier 1) that also ORs a flag over
+// them, so that all take the same branch afterwards.
+__device__ __forceinline__ bool cons_bar_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+      " bar.red.or.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kWarps * 32)
+      : "memory");
+  return r != 0;
+}
+
 // ---- the kernel -----------------------------------------------------------
 // Blocks per SM the kernel is compiled for: two for quantised weights, whose
 // SIMT decode loop is bound by the latency of its dependent chains (twice
@@ -594,13 +633,19 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
   // else the consumers read them from global memory
   const int sb = FMT == WF_BF16 ? 0 : seg / GROUP;
   const bool sc_tma = FMT != WF_BF16 && (sb % 16) == 0;
-  const uint32_t codes_bytes = (uint32_t)kWarps * R * item_bytes;
+  // several BF16 activation rows with whole-row items: the 8 rows of a
+  // stage are the 8 MMA columns (see mma_rows8), each item copied to its own
+  // 16-byte-padded slot so that ldmatrix reads them without bank conflicts
+  const bool mmab = kMmaB<NB, EPI, FMT> && S == 1;
+  const uint32_t item_pitch = item_bytes + (mmab ? 16u : 0u);
+  const uint32_t codes_bytes = (uint32_t)kWarps * R * item_pitch;
   const uint32_t stage_bytes =
       codes_bytes + (sc_tma ? (uint32_t)(kWarps * R * sb) : 0u);
+  const int XS = x_stride<NB, FMT>(K);                    // activation row
   uint8_t* ring = smem;                                   // NS stages
-  void* xs = ring + (size_t)NS * stage_bytes;             // [NB][K] 16-bit
+  void* xs = ring + (size_t)NS * stage_bytes;             // [NB][XS] 16-bit
   float* tmp = reinterpret_cast<float*>(reinterpret_cast<uint16_t*>(xs) +
-                                        (size_t)NB * K);  // [K] if 2-pass
+                                        (size_t)NB * XS); // [K] if 2-pass
   uint64_t* full = reinterpret_cast<uint64_t*>(tmp + (pl.tmp ? K : 0));
   uint64_t* empty = full + NS;
   __shared__ float red[7 * (kWarps + 1)];
@@ -628,11 +673,22 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
                                    : reinterpret_cast<const char*>(a.Wq);
     const uint32_t sbytes = sc_tma ? (uint32_t)(cnt * sb) : 0u;
     mbar_expect_tx(bar, (bytes + sbytes) * R);
-    tma_load_1d_hint(dst, w + (size_t)it * item_bytes, bytes, bar, pol);
-    if (R == 2)
-      tma_load_1d_hint(dst + kWarps * item_bytes,
-                       w + ((size_t)it + (size_t)a.pair_off * S) * item_bytes, bytes,
-                       bar, pol);
+    if (mmab) {
+      for (int k = 0; k < cnt; ++k) {
+        tma_load_1d_hint(dst + k * item_pitch, w + (size_t)(it + k) * item_bytes,
+                         item_bytes, bar, pol);
+        if (R == 2)
+          tma_load_1d_hint(dst + (kWarps + k) * item_pitch,
+                           w + ((size_t)it + k + (size_t)a.pair_off) * item_bytes,
+                           item_bytes, bar, pol);
+      }
+    } else {
+      tma_load_1d_hint(dst, w + (size_t)it * item_bytes, bytes, bar, pol);
+      if (R == 2)
+        tma_load_1d_hint(dst + kWarps * item_bytes,
+                         w + ((size_t)it + (size_t)a.pair_off * S) * item_bytes,
+                         bytes, bar, pol);
+    }
     if (sc_tma) {
       // scales of item it start at byte it * sb (rows are K / GROUP bytes)
       const char* ws = reinterpret_cast<const char*>(a.Ws);
@@ -669,14 +725,14 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
 #pragma unroll 1
     for (int b = 0; b < NB; ++b) {
       if (b < a.B) {
-        if (upd_reg) stage_x_update<FMT>(a, b, al, xs, red);
-        else stage_x_update_2pass<FMT>(a, b, xs, tmp, red);
+        if (upd_reg) stage_x_update<FMT>(a, b, XS, al, xs, red);
+        else stage_x_update_2pass<FMT>(a, b, XS, xs, tmp, red);
       } else {
-        for (int i = tid; i < K; i += kThreads) put_x<FMT>(xs, b * K + i, 0.f);
+        for (int i = tid; i < K; i += kThreads) put_x<FMT>(xs, b * XS + i, 0.f);
       }
     }
   } else {
-    stage_x_copy<FMT, NB>(a, xs);
+    stage_x_copy<FMT, NB>(a, XS, xs);
   }
   __syncthreads();
 
@@ -700,10 +756,104 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
       }
     }
   } else {
-    // ---- consumers: warp w owns item w of every stage ------------------
+    // ---- consumers -----------------------------------------------------
     const int sbrow = FMT == WF_BF16 ? 0 : K / GROUP;
     int slot = 0;
     uint32_t phase = 0;
+    bool done = false;
+    if constexpr (kMmaB<NB, EPI, FMT>) {
+      if (mmab) {
+        done = true;
+        constexpr int KSW = kSeg / (16 * kWarps);   // k-steps per warp, max
+        const int ksw = seg / (16 * kWarps);        // even: seg % 256 == 0
+        const int kb = warp * ksw * 16;             // this warp's first k
+        const int g = lane >> 2, t = lane & 3, ct = tid;
+        uint32_t af[KSW][2];
+        const uint16_t* xh = reinterpret_cast<const uint16_t*>(xs);
+#pragma unroll
+        for (int q = 0; q < KSW; ++q) {
+          af[q][0] = af[q][1] = 0u;
+          if (q < ksw && g < NB) {
+            const uint16_t* xr = xh + (size_t)g * XS + kb + 16 * q + 2 * t;
+            af[q][0] = *reinterpret_cast<const uint32_t*>(xr);
+            af[q][1] = *reinterpret_cast<const uint32_t*>(xr + 8);
+          }
+        }
+        float* redm = reinterpret_cast<float*>(full + 2 * kMaxStages);
+        // ldmatrix.x4 of two k-steps: lane l addresses row l % 8 of matrix
+        // l / 8 (k offsets 0, 8, 16, 24)
+        const uint32_t loff = (uint32_t)(lane & 7) * item_pitch +
+                              (uint32_t)(kb + 8 * (lane >> 3)) * 2;
+        for (int s = 0; s < n_stages; ++s) {
+          const int it0 = j0 + s * kWarps;
+          const int cnt = j1 - it0 < kWarps ? j1 - it0 : kWarps;
+          const bool got = mbar_wait(full + slot, phase);
+          if (!got && lane == 0) atomicOr(&s_fail, 1);
+          float d[R][4];
+#pragma unroll
+          for (int r = 0; r < R; ++r) d[r][0] = d[r][1] = d[r][2] = d[r][3] = 0.f;
+          if (got) {
+            const uint32_t sbase = smem_addr(ring + (size_t)slot * stage_bytes);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              const uint32_t rb = sbase + (uint32_t)(r * kWarps) * item_pitch + loff;
+#pragma unroll
+              for (int q = 0; q < KSW; q += 2) {
+                if (q < ksw) {
+                  uint32_t b[4];
+                  asm volatile(
+                      "ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                      : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
+                      : "r"(rb + q * 32));
+                  const uint32_t a0[4] = {af[q][0], 0u, af[q][1], 0u};
+                  const uint32_t a1[4] = {af[q + 1][0], 0u, af[q + 1][1], 0u};
+                  mma_bf16_16816(d[r], a0, b[0], b[1]);
+                  mma_bf16_16816(d[r], a1, b[2], b[3]);
+                }
+              }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + slot);   // stage read
+          }
+          // partial sums: lane (g, t) holds D[g][2t], D[g][2t + 1] (batch
+          // row g, weight rows 2t, 2t + 1 of the stage)
+          float* rbuf = redm + ((size_t)(s & 1) * kWarps + warp) * R * 64;
+          if (g < NB) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              rbuf[r * 64 + g * 8 + 2 * t] = d[r][0];
+              rbuf[r * 64 + g * 8 + 2 * t + 1] = d[r][1];
+            }
+          }
+          if (cons_bar_or(*fail != 0)) break;
+          if (ct < NB * 8) {
+            const int bb = ct >> 3, n8 = ct & 7;
+            if (n8 < cnt && bb < a.B) {
+              float acc[R];
+#pragma unroll
+              for (int r = 0; r < R; ++r) {
+                acc[r] = 0.f;
+#pragma unroll
+                for (int w2 = 0; w2 < kWarps; ++w2)
+                  acc[r] += redm[((size_t)(s & 1) * kWarps + w2) * R * 64 +
+                                 r * 64 + bb * 8 + n8];
+              }
+              const int n = it0 + n8;
+              if (EPI == EPI_F32) {
+                a.out[(size_t)bb * a.n_items + n] = acc[0];
+              } else {
+                const float gv = acc[0];
+                a.out_bf[(size_t)bb * a.pair_off + n] =
+                    __float2bfloat16_rn(gv * sigmoidf_(gv) * acc[R - 1]);
+              }
+            }
+          }
+          if (++slot == NS) { slot = 0; phase ^= 1u; }
+        }
+      }
+    }
+    if (!done) {
+    // ---- warp w owns item w of every stage ---------------------------------
     // batch 1, BF16: tensor-core row dots with x (this warp's segment
     // w % S) held as MMA fragments for the whole launch
     constexpr bool kMma = FMT == WF_BF16 && NB == 1;
@@ -741,7 +891,7 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
         } else {
           item_dot<FMT, NB, R>(wr, sr, gr,
                                reinterpret_cast<const uint16_t*>(xs) + sidx * seg,
-                               K, nch, lane, acc);
+                               XS, nch, lane, acc);
 #pragma unroll
           for (int r = 0; r < R; ++r)
 #pragma unroll
@@ -777,6 +927,7 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
       if (lane == 0) mbar_arrive(empty + slot);
       if (++slot == NS) { slot = 0; phase ^= 1u; }
       if (*fail) break;
+    }
     }
   }
   __syncthreads();
@@ -828,13 +979,26 @@ bool needs_tmp(const GemvArgs& a) {
   return a.pro == PRO_UPDATE && a.K > kU * kThreads;
 }
 
-size_t fixed_smem(const GemvArgs& a, int nb) {
-  return (size_t)nb * a.K * 2 + (needs_tmp(a) ? (size_t)a.K * 4 : 0) +
-         2 * kMaxStages * 8;
-}
-
 // Bytes of one lane chunk (8 weights) of a format.
 int lane_bytes(int fmt) { return fmt == WF_BF16 ? 16 : fmt == WF_MXFP8 ? 8 : 4; }
+
+// Host view of kMmaB (the batched MMA path needs whole-row items, S = 1).
+bool mmab_kernel(const GemvArgs& a, int nb) {
+  return a.fmt == WF_BF16 && nb >= 2 && a.epi != EPI_LMHEAD;
+}
+
+size_t fixed_smem(const GemvArgs& a, int nb) {
+  return (size_t)nb * x_stride_of(a.fmt, nb, a.K) * 2 +
+         (needs_tmp(a) ? (size_t)a.K * 4 : 0) + 2 * kMaxStages * 8 +
+         (mmab_kernel(a, nb) ? (size_t)kRedFloats * 4 : 0);
+}
+
+// Bytes of one item slot in a stage (padded on the batched MMA path).
+size_t item_slot(const GemvArgs& a, int nb, int S) {
+  return (size_t)(a.K / S) / 8 * lane_bytes(a.fmt) +
+         (mmab_kernel(a, nb) && S == 1 ? 16 : 0);
+}
+
 
 // Segments per row S (F32 only: SwiGLU and LM head need whole rows) and
 // ring depth: the largest segment <= kSeg whose 8-item stages still fit at
@@ -864,7 +1028,7 @@ Plan make_plan(const GemvArgs& a, int nb) {
   }
   const int sbytes = a.fmt == WF_BF16 ? 0
                      : (a.K / S) / (a.fmt == WF_MXFP8 ? 32 : 16);
-  const size_t stage = (size_t)kWarps * R * ((a.K / S) / 8 * lb +
+  const size_t stage = (size_t)kWarps * R * (item_slot(a, nb, S) +
                                              (sbytes % 16 == 0 ? sbytes : 0));
   int NS = stages_default();
   if (a.fmt != WF_BF16) NS = kMaxStages;          // smaller items: go deeper
@@ -883,8 +1047,7 @@ size_t smem_bytes(const GemvArgs& a, const Plan& p, int nb) {
   const int sbytes = a.fmt == WF_BF16 ? 0
                      : (a.K / p.S) / (a.fmt == WF_MXFP8 ? 32 : 16);
   return (size_t)p.NS * kWarps * R *
-             ((a.K / p.S) / 8 * lane_bytes(a.fmt) +
-              (sbytes % 16 == 0 ? sbytes : 0)) +
+             (item_slot(a, nb, p.S) + (sbytes % 16 == 0 ? sbytes : 0)) +
          fixed_smem(a, nb);
 }
 

@@ -154,3 +154,27 @@ def test_quantised_prefill_dory_widths(qmodel):
     torch.cuda.empty_cache()
     zr = Model(QSHAPE, qw, kv_mode="per_loop").forward(prompt, k, True)
     compare(zg, zr, f"{fmt} prefill T={T} Dory widths")
+
+
+@pytest.mark.parametrize("B", [2, 3, 4, 8])
+@pytest.mark.parametrize("name", ["blk0.w_qkvg", "blk1.w_o", "blk2.w_gu",
+                                  "blk1.w_down"])
+def test_bf16_batched_gemv_matches_float64(bf16_weights, name, B):
+    """The BF16 decode GEMV for 2..8 activation rows (whole-row projections
+    on the warp MMA, the 8 weight rows of a stage as the MMA columns; the
+    K-split down projection on the SIMT loop) against a float64 product of
+    the same bf16 values."""
+    import looped_ngpt_b200 as lb
+    from synthetic.gen import bf16_bits_to_f32, f32_to_bf16_bits
+    gm = lb.DoryModel(QSHAPE, bf16_weights, device="cuda:0")
+    W = bf16_bits_to_f32(bf16_weights[name]).astype(np.float64)
+    K = W.shape[1]
+    rng = np.random.default_rng(B * 7 + K)
+    x = f32_to_bf16_bits(rng.standard_normal((B, K)).astype(np.float32) /
+                         np.float32(np.sqrt(K)))
+    dx = torch.from_numpy(x.view(np.int16)).to("cuda:0")
+    got = gm.debug_gemv(name, dx).cpu().numpy().astype(np.float64).sum(0)
+    want = bf16_bits_to_f32(x).astype(np.float64) @ W.T
+    assert gm.sync_status() == 0
+    tol = 2e-5 * np.sqrt(K) * (np.abs(want).max() + 1e-3)
+    assert np.abs(got - want).max() <= tol, np.abs(got - want).max()
