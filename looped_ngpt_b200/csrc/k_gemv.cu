@@ -574,7 +574,8 @@ __device__ __forceinline__ float row_dot_mma(const uint8_t* w,
 }
 
 // ---- several BF16 activation rows on the tensor cores -----------------------
-// Whole-row items (no K split) of BF16 weights with 2..8 activation rows:
+// BF16 weights with 2..8 activation rows (whole rows, or K segments taken
+// segment-major so that the 8 rows of a stage share one segment):
 // m16n8k16 with the activation rows as the M rows (NB of 16 used) and the 8
 // weight rows of a stage as the N = 8 columns, so every product but those of
 // the unused M rows counts.  Warp w takes the w-th eighth of K of all 8 rows
@@ -636,7 +637,10 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
   // several BF16 activation rows with whole-row items: the 8 rows of a
   // stage are the 8 MMA columns (see mma_rows8), each item copied to its own
   // 16-byte-padded slot so that ldmatrix reads them without bank conflicts
-  const bool mmab = kMmaB<NB, EPI, FMT> && S == 1;
+  // (K-split items only from 4 rows on: with 2 rows the per-segment
+  // fragment reloads cost more than the SIMT loop, 531 -> 495 tok/s)
+  const bool mmab = kMmaB<NB, EPI, FMT> && a.n_items % 8 == 0 &&
+                    (S == 1 || NB >= 4);
   const uint32_t item_pitch = item_bytes + (mmab ? 16u : 0u);
   const uint32_t codes_bytes = (uint32_t)kWarps * R * item_pitch;
   const uint32_t stage_bytes =
@@ -654,10 +658,19 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
   __shared__ int s_fail, s_issued;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // row-aligned item range: a stage of 8 items starts at a multiple of S,
-  // so warp w always works on K segment w % S
-  const int j0 = (int)((long)a.n_items * blockIdx.x / gridDim.x) * S;
-  const int j1 = (int)((long)a.n_items * (blockIdx.x + 1) / gridDim.x) * S;
+  // item range.  Row-major items (row it >> sh, segment it & (S - 1)): a
+  // stage of 8 items starts at a multiple of S, so warp w always works on K
+  // segment w % S.  Batched MMA path with S > 1: segment-major items
+  // (segment it / n_items, row it % n_items) in ranges aligned to 8, so the
+  // 8 rows of a stage share one K segment.
+  int j0 = (int)((long)a.n_items * blockIdx.x / gridDim.x) * S;
+  int j1 = (int)((long)a.n_items * (blockIdx.x + 1) / gridDim.x) * S;
+  if (mmab && S > 1) {
+    const long tot = (long)a.n_items * S;
+    j0 = (int)(tot * blockIdx.x / gridDim.x) & ~7;
+    j1 = blockIdx.x + 1 == gridDim.x ? (int)tot
+                                     : (int)(tot * (blockIdx.x + 1) / gridDim.x) & ~7;
+  }
   const int n_stages = (j1 - j0 + kWarps - 1) / kWarps;
   const bool producer = tid == kWarps * 32;
 
@@ -675,8 +688,10 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
     mbar_expect_tx(bar, (bytes + sbytes) * R);
     if (mmab) {
       for (int k = 0; k < cnt; ++k) {
-        tma_load_1d_hint(dst + k * item_pitch, w + (size_t)(it + k) * item_bytes,
-                         item_bytes, bar, pol);
+        // segment-major item it + k: row (it + k) % n_items, segment (it + k) / n_items
+        const size_t src = (size_t)((it + k) % a.n_items) * S + (it + k) / a.n_items;
+        tma_load_1d_hint(dst + k * item_pitch, w + src * item_bytes, item_bytes,
+                         bar, pol);
         if (R == 2)
           tma_load_1d_hint(dst + (kWarps + k) * item_pitch,
                            w + ((size_t)it + k + (size_t)a.pair_off) * item_bytes,
@@ -770,15 +785,21 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
         const int g = lane >> 2, t = lane & 3, ct = tid;
         uint32_t af[KSW][2];
         const uint16_t* xh = reinterpret_cast<const uint16_t*>(xs);
+        // activation fragments of K segment sg (kept while the segment lasts)
+        int aseg = -1;
+        auto load_af = [&](int sg) {
 #pragma unroll
-        for (int q = 0; q < KSW; ++q) {
-          af[q][0] = af[q][1] = 0u;
-          if (q < ksw && g < NB) {
-            const uint16_t* xr = xh + (size_t)g * XS + kb + 16 * q + 2 * t;
-            af[q][0] = *reinterpret_cast<const uint32_t*>(xr);
-            af[q][1] = *reinterpret_cast<const uint32_t*>(xr + 8);
+          for (int q = 0; q < KSW; ++q) {
+            af[q][0] = af[q][1] = 0u;
+            if (q < ksw && g < NB) {
+              const uint16_t* xr =
+                  xh + (size_t)g * XS + (size_t)sg * seg + kb + 16 * q + 2 * t;
+              af[q][0] = *reinterpret_cast<const uint32_t*>(xr);
+              af[q][1] = *reinterpret_cast<const uint32_t*>(xr + 8);
+            }
           }
-        }
+          aseg = sg;
+        };
         float* redm = reinterpret_cast<float*>(full + 2 * kMaxStages);
         // ldmatrix.x4 of two k-steps: lane l addresses row l % 8 of matrix
         // l / 8 (k offsets 0, 8, 16, 24)
@@ -787,6 +808,8 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
         for (int s = 0; s < n_stages; ++s) {
           const int it0 = j0 + s * kWarps;
           const int cnt = j1 - it0 < kWarps ? j1 - it0 : kWarps;
+          const int sg = it0 / a.n_items, row0 = it0 - sg * a.n_items;
+          if (sg != aseg) load_af(sg);
           const bool got = mbar_wait(full + slot, phase);
           if (!got && lane == 0) atomicOr(&s_fail, 1);
           float d[R][4];
@@ -838,9 +861,9 @@ gemv_kernel(const GemvArgs a, const Plan pl) {
                   acc[r] += redm[((size_t)(s & 1) * kWarps + w2) * R * 64 +
                                  r * 64 + bb * 8 + n8];
               }
-              const int n = it0 + n8;
+              const int n = row0 + n8;
               if (EPI == EPI_F32) {
-                a.out[(size_t)bb * a.n_items + n] = acc[0];
+                a.out[((size_t)sg * a.B + bb) * a.n_items + n] = acc[0];
               } else {
                 const float gv = acc[0];
                 a.out_bf[(size_t)bb * a.pair_off + n] =
@@ -982,9 +1005,10 @@ bool needs_tmp(const GemvArgs& a) {
 // Bytes of one lane chunk (8 weights) of a format.
 int lane_bytes(int fmt) { return fmt == WF_BF16 ? 16 : fmt == WF_MXFP8 ? 8 : 4; }
 
-// Host view of kMmaB (the batched MMA path needs whole-row items, S = 1).
+// Host view of the batched MMA path (kMmaB and 8 | n_items).
 bool mmab_kernel(const GemvArgs& a, int nb) {
-  return a.fmt == WF_BF16 && nb >= 2 && a.epi != EPI_LMHEAD;
+  return a.fmt == WF_BF16 && nb >= 2 && a.epi != EPI_LMHEAD &&
+         a.n_items % 8 == 0;
 }
 
 size_t fixed_smem(const GemvArgs& a, int nb) {
@@ -996,7 +1020,7 @@ size_t fixed_smem(const GemvArgs& a, int nb) {
 // Bytes of one item slot in a stage (padded on the batched MMA path).
 size_t item_slot(const GemvArgs& a, int nb, int S) {
   return (size_t)(a.K / S) / 8 * lane_bytes(a.fmt) +
-         (mmab_kernel(a, nb) && S == 1 ? 16 : 0);
+         (mmab_kernel(a, nb) && (S == 1 || nb >= 4) ? 16 : 0);
 }
 
 
