@@ -22,6 +22,7 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <cstdlib>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -135,6 +136,90 @@ __device__ __forceinline__ void qkv_epilogue(const TcArgs& a, int item,
     u.x = pack2(v[i], v[i + 1]); u.y = pack2(v[i + 2], v[i + 3]);
     u.z = pack2(v[i + 4], v[i + 5]); u.w = pack2(v[i + 6], v[i + 7]);
     *reinterpret_cast<uint4*>(dst + i) = u;
+  }
+}
+
+// Epilogue of one output row of a tile: this thread owns TMEM lane `trow`
+// (row `row` of C), columns n0 .. of the tile (column tile ni, K split z).
+template <int MODE, int TN>
+__device__ __forceinline__ void epilogue_row(const TcArgs& a, uint32_t trow,
+                                             int row, int n0, int ni, int z) {
+  constexpr int OUTC = MODE == TC_SWIGLU ? TN / 2 : TN;   // output columns
+  if (MODE == TC_PLAIN) {
+    for (int c0 = 0; c0 < TN; c0 += 32) {
+      float v[32];
+      tmem_ld32(trow + c0, v);
+      if (a.out_scale) {
+        const float os = *a.out_scale;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v[k] *= os;
+      }
+      const int col = n0 + c0;
+      if (row < a.M && col < a.N) {
+        float* dst = a.C + z * a.slab + (size_t)row * a.ldc + col;
+        if (a.col_scale) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (col + k < a.N) v[k] *= a.col_scale[col + k];
+        }
+        // 16-byte stores only when every row start stays 16-byte aligned
+        if (col + 32 <= a.N && (a.ldc & 3) == 0) {
+#pragma unroll
+          for (int k = 0; k < 32; k += 4)
+            *reinterpret_cast<float4*>(dst + k) =
+                make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+        } else {
+          for (int k = 0; k < 32 && col + k < a.N; ++k) dst[k] = v[k];
+        }
+      }
+    }
+  } else if (MODE == TC_SWIGLU) {
+    for (int c0 = 0; c0 < TN / 2; c0 += 32) {
+      float gt[32], u[32];
+      tmem_ld32(trow + c0, gt);
+      tmem_ld32(trow + TN / 2 + c0, u);
+      if (a.out_scale) {
+        const float os = *a.out_scale;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          gt[k] *= os;
+          u[k] *= os;
+        }
+      }
+      const int col = n0 + c0;
+      // columns of this tile only (TN / 2 need not be a multiple of 32)
+      const int lim = min(32, min(OUTC - c0, a.N - col));
+      if (row < a.M && lim > 0) {
+        bf16* dst = a.Cb + (size_t)row * a.ldc + col;
+        if (lim == 32 && (a.ldc & 1) == 0) {
+#pragma unroll
+          for (int k = 0; k < 32; k += 2)
+            *reinterpret_cast<__nv_bfloat162*>(dst + k) = __floats2bfloat162_rn(
+                gt[k] * sigmoidf_(gt[k]) * u[k],
+                gt[k + 1] * sigmoidf_(gt[k + 1]) * u[k + 1]);
+        } else {
+          // unrolled with a predicate so that gt and u stay in registers
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (k < lim) dst[k] = __float2bfloat16_rn(gt[k] * sigmoidf_(gt[k]) * u[k]);
+        }
+      }
+    }
+  } else {
+    float v[TN];
+#pragma unroll
+    for (int c0 = 0; c0 < TN; c0 += 32) {
+      float t32[32];
+      tmem_ld32(trow + c0, t32);
+#pragma unroll
+      for (int k = 0; k < 32; ++k) v[c0 + k] = t32[k];
+    }
+    if (a.out_scale) {
+      const float os = *a.out_scale;
+#pragma unroll
+      for (int k = 0; k < TN; ++k) v[k] *= os;
+    }
+    if (row < a.M) qkv_epilogue<TN>(a, ni, row, v);
   }
 }
 
@@ -300,80 +385,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       const int m0 = mi * BM, n0 = ni * OUTC;
       const int row = m0 + q * 32 + lane;
       const uint32_t trow = tmem + buf * kAccCols + ((uint32_t)(q * 32) << 16);
-      if (MODE == TC_PLAIN) {
-        for (int c0 = 0; c0 < TN; c0 += 32) {
-          float v[32];
-          tmem_ld32(trow + c0, v);
-          if (a.out_scale) {
-            const float os = *a.out_scale;
-#pragma unroll
-            for (int k = 0; k < 32; ++k) v[k] *= os;
-          }
-          const int col = n0 + c0;
-          if (row < a.M && col < a.N) {
-            float* dst = a.C + z * a.slab + (size_t)row * a.ldc + col;
-            if (a.col_scale) {
-#pragma unroll
-              for (int k = 0; k < 32; ++k)
-                if (col + k < a.N) v[k] *= a.col_scale[col + k];
-            }
-            // 16-byte stores only when every row start stays 16-byte aligned
-            if (col + 32 <= a.N && (a.ldc & 3) == 0) {
-#pragma unroll
-              for (int k = 0; k < 32; k += 4)
-                *reinterpret_cast<float4*>(dst + k) =
-                    make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
-            } else {
-              for (int k = 0; k < 32 && col + k < a.N; ++k) dst[k] = v[k];
-            }
-          }
-        }
-      } else if (MODE == TC_SWIGLU) {
-        for (int c0 = 0; c0 < TN / 2; c0 += 32) {
-          float gt[32], u[32];
-          tmem_ld32(trow + c0, gt);
-          tmem_ld32(trow + TN / 2 + c0, u);
-          if (a.out_scale) {
-            const float os = *a.out_scale;
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              gt[k] *= os;
-              u[k] *= os;
-            }
-          }
-          const int col = n0 + c0;
-          // columns of this tile only (TN / 2 need not be a multiple of 32)
-          const int lim = min(32, min(OUTC - c0, a.N - col));
-          if (row < a.M && lim > 0) {
-            bf16* dst = a.Cb + (size_t)row * a.ldc + col;
-            if (lim == 32 && (a.ldc & 1) == 0) {
-#pragma unroll
-              for (int k = 0; k < 32; k += 2)
-                *reinterpret_cast<__nv_bfloat162*>(dst + k) = __floats2bfloat162_rn(
-                    gt[k] * sigmoidf_(gt[k]) * u[k],
-                    gt[k + 1] * sigmoidf_(gt[k + 1]) * u[k + 1]);
-            } else {
-              for (int k = 0; k < lim; ++k)
-                dst[k] = __float2bfloat16_rn(gt[k] * sigmoidf_(gt[k]) * u[k]);
-            }
-          }
-        }
-      } else {
-        float v[TN];
-#pragma unroll
-        for (int c0 = 0; c0 < TN; c0 += 32) {
-          float t32[32];
-          tmem_ld32(trow + c0, t32);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) v[c0 + k] = t32[k];
-        }
-        if (a.out_scale) {
-          const float os = *a.out_scale;
-#pragma unroll
-          for (int k = 0; k < TN; ++k) v[k] *= os;
-        }
-        if (row < a.M) qkv_epilogue<TN>(a, ni, row, v);
-      }
+      epilogue_row<MODE, TN>(a, trow, row, n0, ni, z);
       // this warp's lanes are read: the buffer may take tile i + 2
       tc_fence_before();
       __syncwarp();
@@ -400,6 +412,183 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   if (warp == 0) {
     tc_fence_after();
     tmem_free(tmem, 2 * kAccCols);
+  }
+}
+
+// CTA-pair variant for many-row GEMMs (prefill): a cluster of two CTAs on
+// one TPC computes a 256 x 256 output tile with tcgen05 cta_group::2 MMAs
+// (M = 256, N = 256, K = 16).  Each CTA stages its own 128 rows of A and
+// half of the tile's W rows (128: the first or second half of the column
+// tile; SwiGLU: the gate rows in the even CTA, the up rows in the odd one),
+// so a CTA moves 32 KB per 64-deep K block instead of 48 KB and the ring
+// holds PSTAGES = 6 stages in the same shared memory.  Per K block each SM
+// reads 16 KB of operands for 2 x 128 x 256 x 64 products, two thirds of
+// what a one-CTA 128 x 256 tile reads: the single-CTA kernel is limited by
+// the shared-memory bandwidth that the TMA fill and the MMA operand reads
+// share.
+//   both CTAs, warp 0 lane 0: TMA producer for its own halves; the copies
+//       count on the even CTA's `full` barrier (the even producer arms it
+//       with both CTAs' bytes), stages are released to both producers by
+//       the MMA commit (multicast to both CTAs' `empty` barriers);
+//   even CTA, warp 1 lane 0: MMA issuer (cta_group::2) into one of two
+//       256-column accumulators of both CTAs' TMEM;
+//   both CTAs, warps 2-5: epilogue of their own 128 rows (TMEM lanes), then
+//       an arrival on the even CTA's `acc_empty` (8 arrivals per use).
+// Every wait is bounded; a final cluster barrier keeps either CTA from
+// leaving while the other may still address its shared memory or TMEM.
+constexpr int PSTAGES = 6;
+constexpr uint32_t kPairB = (BN / 2) * BK * 2;     // 16 KB: half the W rows
+constexpr uint32_t kPairStage = kStageA + kPairB;  // 32 KB per CTA and stage
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB, const TcArgs a,
+                    const TileGrid tg) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = su32(smem_raw);
+  uint8_t* base = smem_raw + ((1024 - (raw & 1023)) & 1023);
+  uint8_t* sA = base;
+  uint8_t* sB = base + PSTAGES * kStageA;
+  __shared__ __align__(8) uint64_t full[PSTAGES], empty[PSTAGES];
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
+  __shared__ uint32_t tmem_base;
+  __shared__ int s_fail, s_issued;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();             // 0: MMA issuer
+  constexpr int OUTC = MODE == TC_SWIGLU ? BN / 2 : BN;
+  const int KB = a.K / BK;
+  volatile int* fail = &s_fail;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < PSTAGES; ++i) {
+      mbar_init(full + i, 1);
+      mbar_init(empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(acc_full + i, 1);
+      mbar_init(acc_empty + i, 2 * kEpiWarps);
+    }
+    mbar_init(&mma_done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
+    s_fail = 0;
+    s_issued = 0;
+  }
+  if (warp == 0) tmem_alloc_pair(&tmem_base, 2 * kAccCols);
+  tc_fence_before();
+  cluster_sync_all();             // both CTAs' barriers initialised, TMEM held
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  pdl_wait();
+  pdl_trigger();
+  const int ntiles = tg.count();
+  const int c0 = blockIdx.x >> 1, nc = gridDim.x >> 1;   // cluster index, count
+  const uint32_t full0 = cluster_addr(full, 0);          // the even CTA's
+  const uint32_t acc_empty0 = cluster_addr(acc_empty, 0);
+
+  if (warp == 0) {
+    // ---- TMA producer (both CTAs) -----------------------------------------
+    if (lane == 0) {
+      int g = 0;
+      for (int t = c0; t < ntiles && !*fail; t += nc) {
+        int mi, ni, z;
+        tg.at(t, mi, ni, z);
+        const int m0 = mi * 2 * BM + (int)rank * BM;
+        const int nb = MODE == TC_SWIGLU ? (rank ? a.up_off : 0) + ni * OUTC
+                                         : ni * BN + (int)rank * (BN / 2);
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          const int s = g % PSTAGES, use = g / PSTAGES;
+          if (use > 0 && !mbar_wait(empty + s, (uint32_t)((use - 1) & 1))) {
+            atomicOr(&s_fail, 1);
+            break;
+          }
+          if (rank == 0) mbar_expect_tx(full + s, 2 * kPairStage);
+          tma_load_2d_pair(sA + s * kStageA, &tmA, kb * BK, m0, full0 + 8 * s);
+          tma_load_2d_pair(sB + s * kPairB, &tmB, kb * BK, nb, full0 + 8 * s);
+          s_issued = g + 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer (even CTA) --------------------------------------------
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16(2 * BM, BN);
+      int g = 0, i = 0;
+      for (int t = c0; t < ntiles && !*fail; t += nc, ++i) {
+        const int buf = i & 1, ub = i >> 1;
+        // both CTAs' epilogues have drained this buffer (tile i - 2)
+        if (ub > 0 && !mbar_wait_cluster(acc_empty + buf, (uint32_t)((ub - 1) & 1))) {
+          atomicOr(&s_fail, 1);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + buf * kAccCols;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          const int s = g % PSTAGES, use = g / PSTAGES;
+          if (!mbar_wait(full + s, (uint32_t)(use & 1))) {
+            atomicOr(&s_fail, 1);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = su32(sA + s * kStageA), b0 = su32(sB + s * kPairB);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16_pair(acc, smem_desc(a0 + kk * 32), smem_desc(b0 + kk * 32),
+                           idesc, (kb | kk) != 0);
+          umma_commit_pair(empty + s);           // both CTAs' stage s is free
+        }
+        umma_commit_pair(acc_full + buf);
+        if (!ok) break;
+      }
+      umma_commit_pair(&mma_done);
+    }
+  } else {
+    // ---- epilogue warps (both CTAs): own 128 rows --------------------------
+    const int q = warp & 3;
+    int i = 0;
+    for (int t = c0; t < ntiles; t += nc, ++i) {
+      const int buf = i & 1, ub = i >> 1;
+      const bool got = !*fail && mbar_wait(acc_full + buf, (uint32_t)(ub & 1));
+      if (!got) {
+        if (lane == 0) atomicOr(&s_fail, 1);
+        break;
+      }
+      tc_fence_after();
+      int mi, ni, z;
+      tg.at(t, mi, ni, z);
+      const int row = mi * 2 * BM + (int)rank * BM + q * 32 + lane;
+      const uint32_t trow = tmem + buf * kAccCols + ((uint32_t)(q * 32) << 16);
+      epilogue_row<MODE, BN>(a, trow, row, ni * OUTC, ni, 0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8 * buf);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // the pair's MMAs read this CTA's shared memory and write its TMEM: all
+    // of them must be done before either is released (the commit reaches
+    // both CTAs)
+    if (!mbar_wait(&mma_done, 0)) atomicOr(&s_fail, 1);
+    if (*fail) {
+      atomicOr(a.err, ERRBIT_TIMEOUT);
+      if (rank == 0) {
+        const int hi = s_issued, lo = hi > PSTAGES ? hi - PSTAGES : 0;
+        for (int g = lo; g < hi; ++g)
+          if (!mbar_wait(full + g % PSTAGES, (uint32_t)((g / PSTAGES) & 1), kSpin / 16))
+            break;
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_free_pair(tmem, 2 * kAccCols);
   }
 }
 
@@ -484,6 +673,16 @@ bool weight_map(CUtensorMap* m, const void* ptr, long rows, long cols,
   return true;
 }
 
+// CTA-pair tiles for many-row GEMMs (DORY_PAIR_GEMM=0 keeps one CTA per
+// 128 x 256 tile everywhere).
+bool pair_gemm_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("DORY_PAIR_GEMM");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 int* g_err_ptr = nullptr;
 
 size_t tc_smem() { return (size_t)STAGES * (kStageA + kStageB) + 1024; }
@@ -517,6 +716,51 @@ bool launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const TcArgs& a,
   const int grid = tiles < num_sms() ? tiles : num_sms();
   return launch_k(gemm_tc_kernel<MODE, TN>, dim3(grid), dim3(kGemmThreads),
                   tc_smem(), st, ma, mb, a, tg) == cudaSuccess;
+}
+
+size_t tc_pair_smem() { return (size_t)PSTAGES * kPairStage + 1024; }
+
+// Clusters of two co-resident at once (one CTA per SM), at most.
+template <int MODE>
+int pair_clusters() {
+  static int n = [] {
+    cudaFuncSetAttribute(gemm_tc_pair_kernel<MODE>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)tc_pair_smem());
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 74);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = tc_pair_smem();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int v = 0;
+    if (cudaOccupancyMaxActiveClusters(&v, gemm_tc_pair_kernel<MODE>, &cfg) !=
+            cudaSuccess || v < 1) {
+      cudaGetLastError();
+      v = num_sms() / 2;
+    }
+    return v;
+  }();
+  return n;
+}
+
+// Pair tiles: mt2 row tiles of 256 rows x nt column tiles.
+template <int MODE>
+bool launch_tc_pair(const CUtensorMap& ma, const CUtensorMap& mb,
+                    const TcArgs& a, int mt2, int nt, cudaStream_t st) {
+  const int clusters = pair_clusters<MODE>();
+  const int KB = a.K / BK;
+  const TileGrid tg{mt2, nt, 1, KB};
+  const int tiles = mt2 * nt;
+  const int grid = 2 * (tiles < clusters ? tiles : clusters);
+  return launch_k_cluster(gemm_tc_pair_kernel<MODE>, dim3(grid),
+                          dim3(kGemmThreads), tc_pair_smem(), st, 2, ma, mb, a,
+                          tg) == cudaSuccess;
 }
 
 TcArgs base_args(int M, int N, int K) {
@@ -553,7 +797,10 @@ int launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
   a.out_scale = out_scale;
   const int mt = (M + BM - 1) / BM, nt = (N + BN - 1) / BN;
   const int ks = gemm_split_count(M, N, K, col_scale ? 1 : max_splits);
-  launch_tc<TC_PLAIN, BN>(ma, mb, a, mt, nt, st, ks);
+  if (ks == 1 && mt > 1 && pair_gemm_enabled())
+    launch_tc_pair<TC_PLAIN>(ma, mb, a, (M + 2 * BM - 1) / (2 * BM), nt, st);
+  else
+    launch_tc<TC_PLAIN, BN>(ma, mb, a, mt, nt, st, ks);
   return ks;
 }
 
@@ -598,7 +845,11 @@ void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
                                          (F + kSmallPair - 1) / kSmallPair, st);
     return;
   }
-  launch_tc<TC_SWIGLU, BN>(ma, mb, a, mt, (F + BN / 2 - 1) / (BN / 2), st);
+  if (pair_gemm_enabled())
+    launch_tc_pair<TC_SWIGLU>(ma, mb, a, (M + 2 * BM - 1) / (2 * BM),
+                              (F + BN / 2 - 1) / (BN / 2), st);
+  else
+    launch_tc<TC_SWIGLU, BN>(ma, mb, a, mt, (F + BN / 2 - 1) / (BN / 2), st);
 }
 
 // Fused q/k/v/gate projection with the RoPE / QK-norm / KV-write epilogue.

@@ -56,6 +56,49 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// CTA-pair forms (cta_group::2, a cluster of two CTAs on one TPC): one MMA
+// of M = 256 rows issued by the even CTA reads A rows 0-127 and B columns
+// 0 .. N/2-1 from its own shared memory and A rows 128-255 and the other N/2
+// B columns from the odd CTA's shared memory at the same offsets, and writes
+// rows 0-127 of D to the even CTA's TMEM and rows 128-255 to the odd CTA's,
+// at the same TMEM address.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t a,
+                                               uint64_t b, uint32_t idesc,
+                                               uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+// Arrive on the mbarrier at `bar`'s offset in both CTAs of the pair once
+// every tcgen05 operation issued so far by this thread has completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster."
+      "multicast::cluster.b64 [%0], %1;" ::"r"(su32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
+// Pair allocation: one warp of each CTA of the pair issues it, with the same
+// destination offset; the columns are allocated in both CTAs' TMEM.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t cols) {
+  asm volatile(
+      "tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+          su32(dst)),
+      "r"(cols)
+      : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ void tmem_free_pair(uint32_t base, uint32_t cols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(base),
+               "r"(cols)
+               : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
