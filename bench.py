@@ -395,7 +395,7 @@ def run_gpu(args, rank, world, local):
                 hbm_peak=hbm_peak, tc_peak=tc_peak, peak_kind=peak_kind)
 
 
-def run_spec(gm, prompt, steps=16, gamma=4, k_draft=1, k_verify=4):
+def run_spec(gm, prompt, steps=64, gamma=4, k_draft=1, k_verify=4):
     """Self-speculative greedy decoding after the prompt (per_loop cache):
     gamma drafts at k_draft loops, one verify pass at k_verify.  Every step
     synchronises once (the emitted count); wall-clock timing."""

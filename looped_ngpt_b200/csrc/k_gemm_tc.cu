@@ -436,11 +436,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
 //       an arrival on the even CTA's `acc_empty` (8 arrivals per use).
 // Every wait is bounded; a final cluster barrier keeps either CTA from
 // leaving while the other may still address its shared memory or TMEM.
-constexpr int PSTAGES = 6;
-constexpr uint32_t kPairB = (BN / 2) * BK * 2;     // 16 KB: half the W rows
-constexpr uint32_t kPairStage = kStageA + kPairB;  // 32 KB per CTA and stage
+// Stage bytes per CTA (A rows + half the W rows) and ring depth for tile
+// width TN (6 stages of 32 KB at TN = 256).
+constexpr uint32_t pair_b_bytes(int TN) { return (uint32_t)(TN / 2) * BK * 2; }
+constexpr uint32_t pair_stage_bytes(int TN) { return kStageA + pair_b_bytes(TN); }
+constexpr int pair_stages(int TN) {
+  return (int)(212992u / pair_stage_bytes(TN)) < 8 ? (int)(212992u / pair_stage_bytes(TN)) : 8;
+}
 
-template <int MODE>
+template <int MODE, int TN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB, const TcArgs a,
@@ -449,6 +453,8 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   const uint32_t raw = su32(smem_raw);
   uint8_t* base = smem_raw + ((1024 - (raw & 1023)) & 1023);
   uint8_t* sA = base;
+  constexpr int PSTAGES = pair_stages(TN);
+  constexpr uint32_t kPairB = pair_b_bytes(TN), kPairStage = pair_stage_bytes(TN);
   uint8_t* sB = base + PSTAGES * kStageA;
   __shared__ __align__(8) uint64_t full[PSTAGES], empty[PSTAGES];
   __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
@@ -456,7 +462,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   __shared__ int s_fail, s_issued;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();             // 0: MMA issuer
-  constexpr int OUTC = MODE == TC_SWIGLU ? BN / 2 : BN;
+  constexpr int OUTC = MODE == TC_SWIGLU ? TN / 2 : TN;
   const int KB = a.K / BK;
   volatile int* fail = &s_fail;
 
@@ -497,7 +503,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA,
         tg.at(t, mi, ni, z);
         const int m0 = mi * 2 * BM + (int)rank * BM;
         const int nb = MODE == TC_SWIGLU ? (rank ? a.up_off : 0) + ni * OUTC
-                                         : ni * BN + (int)rank * (BN / 2);
+                                         : ni * TN + (int)rank * (TN / 2);
         for (int kb = 0; kb < KB; ++kb, ++g) {
           const int s = g % PSTAGES, use = g / PSTAGES;
           if (use > 0 && !mbar_wait(empty + s, (uint32_t)((use - 1) & 1))) {
@@ -514,7 +520,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   } else if (warp == 1) {
     // ---- MMA issuer (even CTA) --------------------------------------------
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_bf16(2 * BM, BN);
+      constexpr uint32_t idesc = idesc_bf16(2 * BM, TN);
       int g = 0, i = 0;
       for (int t = c0; t < ntiles && !*fail; t += nc, ++i) {
         const int buf = i & 1, ub = i >> 1;
@@ -562,7 +568,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       tg.at(t, mi, ni, z);
       const int row = mi * 2 * BM + (int)rank * BM + q * 32 + lane;
       const uint32_t trow = tmem + buf * kAccCols + ((uint32_t)(q * 32) << 16);
-      epilogue_row<MODE, BN>(a, trow, row, ni * OUTC, ni, 0);
+      epilogue_row<MODE, TN>(a, trow, row, ni * OUTC, ni, 0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8 * buf);
@@ -718,19 +724,22 @@ bool launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const TcArgs& a,
                   tc_smem(), st, ma, mb, a, tg) == cudaSuccess;
 }
 
-size_t tc_pair_smem() { return (size_t)PSTAGES * kPairStage + 1024; }
+template <int TN>
+size_t tc_pair_smem() {
+  return (size_t)pair_stages(TN) * pair_stage_bytes(TN) + 1024;
+}
 
 // Clusters of two co-resident at once (one CTA per SM), at most.
-template <int MODE>
+template <int MODE, int TN>
 int pair_clusters() {
   static int n = [] {
-    cudaFuncSetAttribute(gemm_tc_pair_kernel<MODE>,
+    cudaFuncSetAttribute(gemm_tc_pair_kernel<MODE, TN>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)tc_pair_smem());
+                         (int)tc_pair_smem<TN>());
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 74);
     cfg.blockDim = dim3(kGemmThreads);
-    cfg.dynamicSmemBytes = tc_pair_smem();
+    cfg.dynamicSmemBytes = tc_pair_smem<TN>();
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -739,7 +748,7 @@ int pair_clusters() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int v = 0;
-    if (cudaOccupancyMaxActiveClusters(&v, gemm_tc_pair_kernel<MODE>, &cfg) !=
+    if (cudaOccupancyMaxActiveClusters(&v, gemm_tc_pair_kernel<MODE, TN>, &cfg) !=
             cudaSuccess || v < 1) {
       cudaGetLastError();
       v = num_sms() / 2;
@@ -749,18 +758,18 @@ int pair_clusters() {
   return n;
 }
 
-// Pair tiles: mt2 row tiles of 256 rows x nt column tiles.
-template <int MODE>
+// Pair tiles: mt2 row tiles of 256 rows x nt column tiles of TN.
+template <int MODE, int TN>
 bool launch_tc_pair(const CUtensorMap& ma, const CUtensorMap& mb,
                     const TcArgs& a, int mt2, int nt, cudaStream_t st) {
-  const int clusters = pair_clusters<MODE>();
+  const int clusters = pair_clusters<MODE, TN>();
   const int KB = a.K / BK;
   const TileGrid tg{mt2, nt, 1, KB};
   const int tiles = mt2 * nt;
   const int grid = 2 * (tiles < clusters ? tiles : clusters);
-  return launch_k_cluster(gemm_tc_pair_kernel<MODE>, dim3(grid),
-                          dim3(kGemmThreads), tc_pair_smem(), st, 2, ma, mb, a,
-                          tg) == cudaSuccess;
+  return launch_k_cluster(gemm_tc_pair_kernel<MODE, TN>, dim3(grid),
+                          dim3(kGemmThreads), tc_pair_smem<TN>(), st, 2, ma, mb,
+                          a, tg) == cudaSuccess;
 }
 
 TcArgs base_args(int M, int N, int K) {
@@ -798,7 +807,7 @@ int launch_gemm_bf16(const bf16* A, int lda, const bf16* W, float* C, int ldc,
   const int mt = (M + BM - 1) / BM, nt = (N + BN - 1) / BN;
   const int ks = gemm_split_count(M, N, K, col_scale ? 1 : max_splits);
   if (ks == 1 && mt > 1 && pair_gemm_enabled())
-    launch_tc_pair<TC_PLAIN>(ma, mb, a, (M + 2 * BM - 1) / (2 * BM), nt, st);
+    launch_tc_pair<TC_PLAIN, BN>(ma, mb, a, (M + 2 * BM - 1) / (2 * BM), nt, st);
   else
     launch_tc<TC_PLAIN, BN>(ma, mb, a, mt, nt, st, ks);
   return ks;
@@ -846,8 +855,8 @@ void launch_gemm_swiglu(const bf16* A, int lda, const bf16* W, bf16* m,
     return;
   }
   if (pair_gemm_enabled())
-    launch_tc_pair<TC_SWIGLU>(ma, mb, a, (M + 2 * BM - 1) / (2 * BM),
-                              (F + BN / 2 - 1) / (BN / 2), st);
+    launch_tc_pair<TC_SWIGLU, BN>(ma, mb, a, (M + 2 * BM - 1) / (2 * BM),
+                                  (F + BN / 2 - 1) / (BN / 2), st);
   else
     launch_tc<TC_SWIGLU, BN>(ma, mb, a, mt, (F + BN / 2 - 1) / (BN / 2), st);
 }

@@ -74,23 +74,24 @@ __global__ void embed_kernel(const int* tokens, const bf16* E, int d,
 }
 
 // The nGPT update of whole rows (see ngpt_update_row for the algebra), one
-// row per block of d / 8 threads: thread i holds elements 4i..4i+3 and
-// d/2 + 4i..d/2 + 4i+3 in registers from the first read to the store, so a
-// row is read once and written once (16-byte accesses), with one block
+// row per block of d / (4 NV) threads: thread i holds the 4-element groups
+// at 4i + k d / NV (k < NV) in registers from the first read to the store,
+// so a row is read once and written once (16-byte accesses), with one block
 // reduction of the norm terms in between.  h: h_S K-split partials of the
-// sublayer output, gridDim.x rows apart.  Requires d % 256 == 0, d <= 8192.
+// sublayer output, gridDim.x rows apart.  NV = 2 needs d % 256 == 0 and
+// d <= 8192; NV = 4 (d % 512 == 0 and d <= 2560: 160 threads at d = 2560)
+// halves the block so that four rows per SM are in flight instead of three.
 // MIXED: rows carry their own loop counts (row_loops non-null); the plain
 // variant has no per-row test at all.
-template <bool MIXED>
-__global__ void update_rows_kernel(const float* s_in, const float* h,
-                                   const float* alpha, float* s_out,
-                                   bf16* s_bf, float* x_buf, int reinject0,
-                                   int d, int h_S, const int* row_loops, int T,
-                                   int upd_loop, int rj_loop) {
+template <bool MIXED, int NV>
+__device__ __forceinline__ void update_row_body(
+    const float* s_in, const float* h, const float* alpha, float* s_out,
+    bf16* s_bf, float* x_buf, int reinject0, int d, int h_S,
+    const int* row_loops, int T, int upd_loop, int rj_loop) {
   __shared__ float red[7 * 32];
   const size_t o = (size_t)blockIdx.x * d;
   const size_t hs = (size_t)gridDim.x * d;
-  const int half = d / 2;
+  const int part = d / NV;
   pdl_wait();
   // rows with their own loop counts (uniform over the block: one row); a
   // row sitting out this loop keeps its state
@@ -100,10 +101,10 @@ __global__ void update_rows_kernel(const float* s_in, const float* h,
   const bool frozen = MIXED && rj < 0;
   const int reinject = frozen ? RJ_NONE : rj;
   const bool next = reinject == RJ_NEXT;
-  float4 sv[2], av[2], hv[2], xv[2];
+  float4 sv[NV], av[NV], hv[NV], xv[NV];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int i = 4 * threadIdx.x + k * half;
+  for (int k = 0; k < NV; ++k) {
+    const int i = 4 * threadIdx.x + k * part;
     sv[k] = *reinterpret_cast<const float4*>(s_in + o + i);
     av[k] = frozen ? make_float4(0.f, 0.f, 0.f, 0.f)
                    : *reinterpret_cast<const float4*>(alpha + i);
@@ -113,9 +114,9 @@ __global__ void update_rows_kernel(const float* s_in, const float* h,
   }
   for (int p = 1; p < (frozen ? 1 : h_S); ++p)
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < NV; ++k) {
       const float4 t = *reinterpret_cast<const float4*>(h + p * hs + o + 4 * threadIdx.x +
-                                                        k * half);
+                                                        k * part);
       hv[k].x += t.x; hv[k].y += t.y; hv[k].z += t.z; hv[k].w += t.w;
     }
   pdl_trigger();
@@ -131,7 +132,7 @@ __global__ void update_rows_kernel(const float* s_in, const float* h,
     r[6] += x * x;
   };
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
+  for (int k = 0; k < NV; ++k) {
     acc(sv[k].x, av[k].x, hv[k].x, xv[k].x);
     acc(sv[k].y, av[k].y, hv[k].y, xv[k].y);
     acc(sv[k].z, av[k].z, hv[k].z, xv[k].z);
@@ -153,8 +154,8 @@ __global__ void update_rows_kernel(const float* s_in, const float* h,
     return v;
   };
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int i = 4 * threadIdx.x + k * half;
+  for (int k = 0; k < NV; ++k) {
+    const int i = 4 * threadIdx.x + k * part;
     float4 xo, vo;
     vo.x = upd(sv[k].x, av[k].x, hv[k].x, xv[k].x, &xo.x);
     vo.y = upd(sv[k].y, av[k].y, hv[k].y, xv[k].y, &xo.y);
@@ -171,6 +172,27 @@ __global__ void update_rows_kernel(const float* s_in, const float* h,
       *reinterpret_cast<uint2*>(s_bf + o + i) = u;
     }
   }
+}
+
+template <bool MIXED>
+__global__ void update_rows_kernel(const float* s_in, const float* h,
+                                   const float* alpha, float* s_out,
+                                   bf16* s_bf, float* x_buf, int reinject0,
+                                   int d, int h_S, const int* row_loops, int T,
+                                   int upd_loop, int rj_loop) {
+  update_row_body<MIXED, 2>(s_in, h, alpha, s_out, s_bf, x_buf, reinject0, d,
+                            h_S, row_loops, T, upd_loop, rj_loop);
+}
+
+// d = 2560: 160 threads, four blocks (rows) per SM without spills
+template <bool MIXED>
+__global__ void __launch_bounds__(160, 4)
+update_rows_wide_kernel(const float* s_in, const float* h, const float* alpha,
+                        float* s_out, bf16* s_bf, float* x_buf, int reinject0,
+                        int d, int h_S, const int* row_loops, int T,
+                        int upd_loop, int rj_loop) {
+  update_row_body<MIXED, 4>(s_in, h, alpha, s_out, s_bf, x_buf, reinject0, d,
+                            h_S, row_loops, T, upd_loop, rj_loop);
 }
 
 // Lowest index among the maxima; NaN entries never win.
@@ -324,14 +346,25 @@ void launch_update_rows(const float* s_in, const float* h, const float* alpha,
                         int M, int d, cudaStream_t st, int h_S,
                         const int* row_loops, int T, int upd_loop,
                         int rj_loop) {
-  if (row_loops)
+  const int Tp = T < 1 ? 1 : T;
+  if (d % 512 == 0 && d <= 2560) {
+    if (row_loops)
+      launch_k(update_rows_wide_kernel<true>, dim3(M), dim3(d / 16), 0, st, s_in,
+               h, alpha, s_out, s_bf, x_buf, reinject, d, h_S, row_loops, Tp,
+               upd_loop, rj_loop);
+    else
+      launch_k(update_rows_wide_kernel<false>, dim3(M), dim3(d / 16), 0, st, s_in,
+               h, alpha, s_out, s_bf, x_buf, reinject, d, h_S, row_loops, Tp,
+               upd_loop, rj_loop);
+  } else if (row_loops) {
     launch_k(update_rows_kernel<true>, dim3(M), dim3(d / 8), 0, st, s_in, h,
-             alpha, s_out, s_bf, x_buf, reinject, d, h_S, row_loops,
-             T < 1 ? 1 : T, upd_loop, rj_loop);
-  else
+             alpha, s_out, s_bf, x_buf, reinject, d, h_S, row_loops, Tp,
+             upd_loop, rj_loop);
+  } else {
     launch_k(update_rows_kernel<false>, dim3(M), dim3(d / 8), 0, st, s_in, h,
-             alpha, s_out, s_bf, x_buf, reinject, d, h_S, row_loops,
-             T < 1 ? 1 : T, upd_loop, rj_loop);
+             alpha, s_out, s_bf, x_buf, reinject, d, h_S, row_loops, Tp,
+             upd_loop, rj_loop);
+  }
 }
 
 void launch_argmax_partials(const float* val, const int* idx, int B, int n,
