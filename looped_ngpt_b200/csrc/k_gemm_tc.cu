@@ -17,6 +17,11 @@
 //                  so epilogues overlap the next tile's MMAs.
 // Every mbarrier wait is bounded: on timeout the CTA records ERRBIT_TIMEOUT,
 // waits (bounded) for its outstanding copies and MMAs, frees TMEM and exits.
+//
+// Many-row plain and SwiGLU GEMMs (prefill) run on CTA pairs instead
+// (gemm_tc_pair_kernel below: clusters of two, tcgen05 cta_group::2,
+// 256 x 256 tiles, each CTA staging half of every operand tile), which halves
+// the shared-memory operand traffic per FLOP that limits the one-CTA tile.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
