@@ -20,8 +20,9 @@
 //
 // Many-row plain and SwiGLU GEMMs (prefill) run on CTA pairs instead
 // (gemm_tc_pair_kernel below: clusters of two, tcgen05 cta_group::2,
-// 256 x 256 tiles, each CTA staging half of every operand tile), which halves
-// the shared-memory operand traffic per FLOP that limits the one-CTA tile.
+// 256 x 256 tiles, each CTA staging its own A rows and half of the W rows),
+// which cuts by a third the shared-memory operand traffic per FLOP that
+// limits the one-CTA tile.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
