@@ -743,7 +743,7 @@ int pair_clusters() {
                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)tc_pair_smem<TN>());
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * 74);
+    cfg.gridDim = dim3(num_sms() >= 2 ? num_sms() & ~1 : 2);   // whole pairs
     cfg.blockDim = dim3(kGemmThreads);
     cfg.dynamicSmemBytes = tc_pair_smem<TN>();
     cudaLaunchAttribute attr[1];
